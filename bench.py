@@ -1,0 +1,467 @@
+"""Benchmark of the hybrid-head sparse decode-attention step (libychee) on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl lychee|reference]
+                    [--workload qwen3_stack_128k|llama3_ragged_stack|qwen3_stack_<N>x<L>]
+
+One step = one decode step of the whole hot path: lychee_decode_stack over all
+layers of the workload (per layer: hybrid attention, top-k of the retrieval
+heads, combine; the sets chained layer to layer), on seeded synthetic inputs
+already resident in HBM.  The default workload is the Qwen3-8B-shaped 36-layer
+stack at 128K context (19.3 GB of K/V per step, far larger than L2, so no L2
+flush is needed between steps).  Rank 0 prints one JSON line.
+
+Under torchrun (N > 1) every rank runs an independent replica (its own sequence,
+seeded by rank); there is no collective on the data path.  Ranks meet at a
+barrier around the timed region and the slowest rank's time is reported.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import sys
+import threading
+import time
+
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "µs/decode-step & achieved HBM GB/s (% of roofline) at 128K ctx, 1 B200"
+UNIT = "µs/decode-step"
+NOMINAL_HBM_GBS = 8000.0
+FALLBACK_HBM_GBS = 6650.0
+
+
+# ---------------------------------------------------------------- helpers
+def measured_peak():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(p) as f:
+            return float(json.load(f)["hbm_gbs"]), "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+class ClockSampler:
+    """Samples SM clock, max clock, power and throttle reasons through NVML while
+    running (reads only; changes no setting)."""
+    REASONS = {
+        0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap",
+        0x8: "hw_slowdown", 0x10: "sync_boost", 0x20: "sw_thermal_slowdown",
+        0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown",
+        0x100: "display_clock_setting",
+    }
+
+    def __init__(self, device_index, period_s=0.01):
+        self.period = period_s
+        self.samples = []
+        self.max_mhz = None
+        self.ok = False
+        self._stop = threading.Event()
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            uuid = str(torch.cuda.get_device_properties(device_index).uuid)
+            handle = None
+            for i in range(pynvml.nvmlDeviceGetCount()):
+                h = pynvml.nvmlDeviceGetHandleByIndex(i)
+                u = pynvml.nvmlDeviceGetUUID(h)
+                u = u.decode() if isinstance(u, bytes) else u
+                if u.replace("GPU-", "") == uuid.replace("GPU-", ""):
+                    handle = h
+            if handle is None:
+                handle = pynvml.nvmlDeviceGetHandleByIndex(device_index)
+            self.nv, self.h = pynvml, handle
+            self.max_mhz = float(pynvml.nvmlDeviceGetMaxClockInfo(handle, pynvml.NVML_CLOCK_SM))
+            self.ok = True
+        except Exception as e:  # no NVML: report the absence, do not fail the bench
+            self.err = str(e)
+
+    def _run(self):
+        nv, h = self.nv, self.h
+        while not self._stop.is_set():
+            try:
+                mhz = nv.nvmlDeviceGetClockInfo(h, nv.NVML_CLOCK_SM)
+                try:
+                    rs = nv.nvmlDeviceGetCurrentClocksEventReasons(h)
+                except Exception:
+                    rs = nv.nvmlDeviceGetCurrentClocksThrottleReasons(h)
+                pw = nv.nvmlDeviceGetPowerUsage(h) / 1000.0
+                self.samples.append((float(mhz), int(rs), pw))
+            except Exception:
+                pass
+            time.sleep(self.period)
+
+    def __enter__(self):
+        if self.ok:
+            self._t = threading.Thread(target=self._run, daemon=True)
+            self._t.start()
+        return self
+
+    def __exit__(self, *a):
+        if self.ok:
+            self._stop.set()
+            self._t.join()
+
+    def summary(self):
+        if not self.ok:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvml unavailable"]}
+        if not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": [], "samples": 0}
+        mhz = [s[0] for s in self.samples]
+        bits = 0
+        for s in self.samples:
+            bits |= s[1]
+        reasons = sorted(n for b, n in self.REASONS.items() if bits & b and n != "gpu_idle")
+        return {"sm_mhz": statistics.median(mhz), "sm_max_mhz": self.max_mhz, "reasons": reasons,
+                "samples": len(mhz), "power_w_max": max(s[2] for s in self.samples)}
+
+
+def make_workload(name, device, seed_offset=0):
+    from hybrid_head_sparse_decode_b200 import inputs
+    if name == "qwen3_stack_128k":
+        return inputs.qwen3_stack_128k(device=device, seed=inputs.BASE_SEED + 2 + seed_offset)
+    if name == "llama3_ragged_stack":
+        return inputs.llama3_ragged_stack(device=device, seed=inputs.BASE_SEED + 3 + seed_offset)
+    if name.startswith("qwen3_stack_"):      # qwen3_stack_<N>x<L>, for small profiling cases
+        n, l = name[len("qwen3_stack_"):].split("x")
+        return inputs.make_stack(int(l), 1, 32, 8, 128, int(n), seed=inputs.BASE_SEED + 2,
+                                 device=device, k_frac=0.3, n_planted=64,
+                                 n_extra_retrieval=min(32, (int(l) - 1) * 32))
+    raise SystemExit(f"unknown workload {name}")
+
+
+def describe(name, prob):
+    from hybrid_head_sparse_decode_b200.inputs import StackProblem
+    if isinstance(prob, StackProblem):
+        L, B, Hq, Hkv, d, N = prob.shape
+        return {"workload": name, "layers": L, "B": B, "Hq": Hq, "Hkv": Hkv, "d": d,
+                "N": N, "seqlens": [int(x) for x in prob.seqlens.cpu()], "k": prob.k,
+                "retrieval_heads": int(prob.roles.sum()), "layer0": "all retrieval",
+                "io_dtype": "bf16",
+                "l2": "no flush: each step reads %.1f GB of K/V (> 126 MB L2)" % (
+                    2 * L * B * Hkv * N * d * 2 / 1e9)}
+    B, Hq, Hkv, d, N = prob.shape
+    return {"workload": name, "layers": 1, "B": B, "Hq": Hq, "Hkv": Hkv, "d": d, "N": N,
+            "k": prob.k, "retrieval_heads": int(prob.role.sum()), "io_dtype": "bf16",
+            "l2": "flushed between steps by writing a 256 MB buffer"}
+
+
+def union_rows(prob, idx_layers):
+    """Rows the method must read per layer and group: n_b for a group holding a
+    retrieval head, |union of the heads' incoming sets| for a sparse-only group.
+    Returns (union_rows_per_layer, literal_rows_per_layer, dense_rows_per_layer)."""
+    L, B, Hq, Hkv, d, N = prob.shape
+    G = Hq // Hkv
+    dev = idx_layers.device
+    union, literal, dense = [], [], []
+    for l in range(L):
+        u = lit = 0
+        roles = prob.roles[l]
+        for b in range(B):
+            n = int(prob.seqlens[b])
+            kb = int(prob.meta["kb"][b])
+            for g in range(Hkv):
+                hs = list(range(g * G, g * G + G))
+                if any(int(roles[h]) == 1 for h in hs):
+                    u += n
+                    lit += n
+                else:
+                    mark = torch.zeros(n, dtype=torch.bool, device=dev)
+                    for h in hs:
+                        row = idx_layers[l - 1, b, h, :kb].long()
+                        mark[row] = True
+                    u += int(mark.sum())
+                    lit += kb
+        union.append(u)
+        literal.append(lit)
+        dense.append(Hkv * int(prob.seqlens.sum()))
+    return union, literal, dense
+
+
+# ---------------------------------------------------------------- our arm
+def run_lychee(args, rank, world, device):
+    from hybrid_head_sparse_decode_b200 import ops
+    from hybrid_head_sparse_decode_b200.inputs import StackProblem
+
+    torch.manual_seed(0)
+    prob = make_workload(args.workload, device, seed_offset=rank)
+    is_stack = isinstance(prob, StackProblem)
+    if not is_stack:
+        raise SystemExit("the step benchmark needs a stack workload")
+    L, B, Hq, Hkv, d, N = prob.shape
+    dt = prob.q.dtype
+    row_bytes = 2 * d * prob.q.element_size()
+    ws = ops.alloc_workspace(B, Hq, Hkv, d, N, prob.k, dt, device)
+    out = torch.empty((L, B, Hq, d), dtype=dt, device=device)
+    fin = torch.empty((B, Hq, prob.k), dtype=torch.int32, device=device)
+    idx_layers = torch.empty((L, B, Hq, prob.k), dtype=torch.int32, device=device)
+    roles = prob.roles
+
+    def step(r=roles, o=out):
+        ops.decode_stack(prob.q, prob.k_caches, prob.v_caches, prob.seqlens, r, prob.k,
+                         k_per_seq=prob.k_per_seq, out=o, idx_final=fin, workspace=ws)
+
+    # untimed pass that also records every layer's sets, to count algorithmic bytes
+    ops.decode_stack(prob.q, prob.k_caches, prob.v_caches, prob.seqlens, roles, prob.k,
+                     k_per_seq=prob.k_per_seq, out=out, idx_final=fin, idx_layers=idx_layers,
+                     workspace=ws)
+    st, bits = ops.check_device_error(ws)
+    if st != 0:
+        raise SystemExit(f"device error {st} bits {bits}")
+    urows, lrows, drows = union_rows(prob, idx_layers)
+    union_bytes = [u * row_bytes for u in urows]
+    literal_bytes = [x * row_bytes for x in lrows]
+    dense_bytes = [x * row_bytes for x in drows]
+    del idx_layers
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+
+    def barrier():
+        if world > 1:
+            torch.distributed.barrier()
+
+    stream = torch.cuda.current_stream()
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    sampler = ClockSampler(device.index)
+    prof = ops.Profile(max_launches=args.steps * (3 * L + 2) + 16)
+    barrier()
+    torch.cuda.synchronize()
+    with sampler, prof:
+        t0.record(stream)
+        for _ in range(args.steps):
+            step()
+        t1.record(stream)
+        torch.cuda.synchronize()
+    barrier()
+    ms_total = t0.elapsed_time(t1)
+    if world > 1:
+        t = torch.tensor([ms_total], device=device, dtype=torch.float64)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        ms_total = float(t.item())
+    ms_step = ms_total / args.steps
+    recs = prof.records
+    attn = [ms for k, ms in recs if k == "attn"]
+    kinds = {}
+    for k, ms in recs:
+        kinds.setdefault(k, [0, 0.0])
+        kinds[k][0] += 1
+        kinds[k][1] += ms
+    # per-launch algorithmic bytes of the attention kernel, layer by layer
+    attn_bytes_per_step = sum(union_bytes)
+    attn_ms_per_step = sum(attn) / args.steps if attn else float("nan")
+    achieved = attn_bytes_per_step / (attn_ms_per_step * 1e-3) / 1e9
+    peak, peak_kind = measured_peak()
+
+    # dense comparator: the same kernels with every head a retrieval head
+    dense_roles = torch.ones_like(roles)
+    dense_out = torch.empty_like(out)
+    for _ in range(max(1, args.warmup // 2)):
+        step(dense_roles, dense_out)
+    dsteps = max(3, args.steps // 4)
+    torch.cuda.synchronize()
+    d0, d1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    d0.record(stream)
+    for _ in range(dsteps):
+        step(dense_roles, dense_out)
+    d1.record(stream)
+    torch.cuda.synchronize()
+    dense_ms = d0.elapsed_time(d1) / dsteps
+
+    # end to end through the public call with host buffers: q (and the per-sequence
+    # lengths and budgets) copied in from pinned memory, out and the final sets read
+    # back every step.  The K/V caches are the model's resident decode state.
+    q_h = prob.q.cpu().pin_memory()
+    sl_h = prob.seqlens.cpu().pin_memory()
+    kb_h = prob.k_per_seq.cpu().pin_memory()
+    out_h = torch.empty(out.shape, dtype=dt).pin_memory()
+    fin_h = torch.empty(fin.shape, dtype=torch.int32).pin_memory()
+    q_d = torch.empty_like(prob.q)
+    sl_d = torch.empty_like(prob.seqlens)
+    kb_d = torch.empty_like(prob.k_per_seq)
+
+    def e2e_step():
+        q_d.copy_(q_h, non_blocking=True)
+        sl_d.copy_(sl_h, non_blocking=True)
+        kb_d.copy_(kb_h, non_blocking=True)
+        ops.decode_stack(q_d, prob.k_caches, prob.v_caches, sl_d, roles, prob.k, k_per_seq=kb_d,
+                         out=out, idx_final=fin, workspace=ws)
+        out_h.copy_(out, non_blocking=True)
+        fin_h.copy_(fin, non_blocking=True)
+
+    for _ in range(2):
+        e2e_step()
+    torch.cuda.synchronize()
+    barrier()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(args.steps):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    e_ms = e0.elapsed_time(e1)
+    if world > 1:
+        t = torch.tensor([e_ms], device=device, dtype=torch.float64)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        e_ms = float(t.item())
+    h2d = (q_h.numel() * q_h.element_size() + sl_h.numel() * 4 + kb_h.numel() * 4)
+    d2h = out_h.numel() * out_h.element_size() + fin_h.numel() * 4
+
+    us_step_job = ms_step * 1e3 / world
+    result = {
+        "metric": METRIC, "value": round(us_step_job, 3), "unit": UNIT, "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_step, 5),
+        "higher_is_better": False, "scaling": "weak", "vs_baseline": None,
+        "dtype": "fp32", "data": "synthetic (seeded; planted high-affinity keys)",
+        "config": describe(args.workload, prob),
+        "us_per_layer": round(ms_step * 1e3 / L, 3),
+        "step_hbm_gbs_union": round(sum(union_bytes) / (ms_step * 1e-3) / 1e9, 1),
+        "step_hbm_gbs_literal": round(sum(literal_bytes) / (ms_step * 1e-3) / 1e9, 1),
+        "bytes_per_step": {"union": sum(union_bytes), "literal": sum(literal_bytes),
+                           "dense": sum(dense_bytes)},
+        "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak,
+                     "unit": "GB/s", "frac": round(achieved / peak, 4), "traffic": None,
+                     "kernel": "attn_kernel (hybrid attention, all layers)",
+                     "peak_source": peak_kind, "frac_of_nominal_8tbs": round(achieved / NOMINAL_HBM_GBS, 4),
+                     "bytes_rule": "union rows x 512 B per launch"},
+        "kernels_ms_per_step": {k: round(v[1] / args.steps, 4) for k, v in kinds.items()},
+        "dense_comparator": {"ms_per_step": round(dense_ms, 4),
+                             "hbm_gbs": round(sum(dense_bytes) / (dense_ms * 1e-3) / 1e9, 1),
+                             "speedup_hybrid_vs_dense": round(dense_ms / ms_step, 3)},
+        "e2e": {"value": round(e_ms * 1e3 / args.steps / world, 3), "unit": UNIT,
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+        "gpu_launches": sum(v[0] for v in kinds.values()),
+        "clocks": sampler.summary(),
+    }
+    return result, prob, union_bytes
+
+
+# ---------------------------------------------------------------- the oracle arm
+def oracle_chain_time(prob, layers, nthreads):
+    """Time the oracle's own chain over the given leading layers of the stack;
+    returns per-layer seconds."""
+    import numpy as np
+
+    import oracle
+
+    def bits(t):
+        t = t.detach().contiguous().cpu()
+        return t.view(torch.int16).numpy().view(np.uint16)
+
+    L, B, Hq, Hkv, d, N = prob.shape
+    seqlens = prob.seqlens.cpu().numpy()
+    kps = prob.k_per_seq.cpu().numpy()
+    idx = np.full((B, Hq, prob.k), -1, np.int32)
+    times = []
+    for l in range(layers):
+        q, K, V = bits(prob.q[l]), bits(prob.k_caches[l]), bits(prob.v_caches[l])
+        t = time.perf_counter()
+        _, idx, _ = oracle.hybrid_layer(q, K, V, seqlens, prob.roles[l].numpy(), idx, prob.k,
+                                        k_per_seq=kps, nthreads=nthreads)
+        times.append(time.perf_counter() - t)
+    return times
+
+
+def scale_to_step(times, L):
+    """Layer 0 (all retrieval) timed as is; the other layers by the mean of the
+    sampled ones."""
+    rest = times[1:] if len(times) > 1 else times
+    return times[0] + sum(rest) / len(rest) * (L - 1)
+
+
+def cpu_baseline(prob, sample_layers=4):
+    import oracle
+    oracle.build()
+    L = prob.shape[0]
+    nthreads = os.cpu_count() or 1
+    B, Hq = prob.shape[1], prob.shape[2]
+    times = oracle_chain_time(prob, min(sample_layers, L), nthreads)
+    est = scale_to_step(times, L)
+    return {"value": round(est * 1e6, 1), "unit": UNIT, "cores": min(nthreads, B * Hq),
+            "kind": "oracle",
+            "sample": f"oracle's own chain over layers 0..{len(times) - 1} of the same "
+                      f"workload ({sum(times):.1f} s of CPU work), scaled to {L} layers: "
+                      f"layer 0 as timed + mean of layers 1..{len(times) - 1} x {L - 1}"}
+
+
+def run_reference(args, rank, world):
+    """The reference arm: the fp64 oracle as it stands, on host cores, each step a
+    bounded sample (the oracle's own chain over the first layers), scaled to a
+    whole decode step.  Rank 0 only."""
+    if rank != 0:
+        return None
+    import oracle
+    oracle.build()
+    device = torch.device("cuda", 0) if torch.cuda.is_available() else torch.device("cpu")
+    prob = make_workload(args.workload, device)
+    L = prob.shape[0]
+    nthreads = os.cpu_count() or 1
+    layers = 2
+    for _ in range(args.warmup if args.warmup < 3 else 1):
+        oracle_chain_time(prob, 1, nthreads)
+    per = []
+    for _ in range(args.steps):
+        per.append(scale_to_step(oracle_chain_time(prob, layers, nthreads), L))
+    us = statistics.median(per) * 1e6
+    B, Hq = prob.shape[1], prob.shape[2]
+    cb = {"value": round(us, 1), "unit": UNIT, "cores": min(nthreads, B * Hq), "kind": "oracle",
+          "sample": f"per step: the oracle's own chain over layers 0..{layers - 1}, scaled to "
+                    f"{L} layers (layer 0 as timed + layer 1 x {L - 1}); median of {args.steps}"}
+    return {"impl": "reference", "metric": METRIC, "value": round(us, 1), "unit": UNIT,
+            "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": round(us / 1e3, 3), "higher_is_better": False, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f64", "data": "synthetic (seeded)",
+            "config": describe(args.workload, prob), "cpu_baseline": cb,
+            "e2e": {"value": round(us, 1), "unit": UNIT, "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+
+
+# ---------------------------------------------------------------- main
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="lychee", choices=["lychee", "reference"])
+    ap.add_argument("--workload", default="qwen3_stack_128k")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3 and args.impl == "lychee":
+        args.warmup = 3
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        # the oracle runs on host cores, on rank 0 only; other ranks leave at once
+        res = run_reference(args, rank, world)
+        if res is not None:
+            print(json.dumps(res), flush=True)
+        return
+    if world > 1:
+        import datetime
+        torch.cuda.set_device(local)
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                             device_id=torch.device("cuda", local))
+
+    device = torch.device("cuda", local)
+    torch.cuda.set_device(device)
+    res, prob, _ = run_lychee(args, rank, world, device)
+    if rank == 0:
+        if world == 1 and not args.no_cpu_baseline:
+            res["cpu_baseline"] = cpu_baseline(prob)
+        print(json.dumps(res), flush=True)
+    if world > 1:
+        torch.distributed.barrier()
+        torch.distributed.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

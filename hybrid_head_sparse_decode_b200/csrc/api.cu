@@ -1,0 +1,378 @@
+// api.cu -- the C ABI of libychee (declared in include/lychee.h): argument
+// validation, workspace layout and the launch sequence of one layer and of an
+// L-layer decode step.  Host code only; no memory is allocated here.
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+#include <vector>
+
+#include "common.cuh"
+#include "kernels.h"
+#include "lychee.h"
+
+using namespace lychee;
+
+namespace {
+
+constexpr int kVersion = 100;   // 0.1.0
+
+struct Layout {
+  size_t logits, part_ml, part_acc, bitmaps, total;
+  int nchunk, nwords;
+};
+
+size_t align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
+
+lychee_status check_shape(const lychee_shape* s) {
+  if (!s) return LYCHEE_ERR_INVALID_ARG;
+  if (s->B < 1 || s->Hq < 1 || s->Hkv < 1 || s->d < 1 || s->N_max < 1 || s->k < 1)
+    return LYCHEE_ERR_INVALID_ARG;
+  if (s->dtype != LYCHEE_BF16 && s->dtype != LYCHEE_FP32) return LYCHEE_ERR_INVALID_ARG;
+  if (s->Hq % s->Hkv != 0) return LYCHEE_ERR_INVALID_ARG;
+  if (s->k > s->N_max) return LYCHEE_ERR_INVALID_ARG;
+  const int G = s->Hq / s->Hkv;
+  if (G != 1 && G != 2 && G != 4 && G != 8) return LYCHEE_ERR_UNSUPPORTED;
+  if (s->Hq > kMaxHq) return LYCHEE_ERR_UNSUPPORTED;
+  if (s->d != 64 && s->d != 128) return LYCHEE_ERR_UNSUPPORTED;
+  if (s->N_max > (1 << 24)) return LYCHEE_ERR_UNSUPPORTED;
+  const long long nchunk = (s->N_max + kChunk - 1) / kChunk;
+  if ((long long)s->B * s->Hkv * nchunk >= (1LL << 31)) return LYCHEE_ERR_UNSUPPORTED;
+  if ((long long)s->B * s->Hq >= (1LL << 24)) return LYCHEE_ERR_UNSUPPORTED;
+  return LYCHEE_OK;
+}
+
+Layout layout_of(const lychee_shape* s) {
+  Layout L{};
+  L.nchunk = (s->N_max + kChunk - 1) / kChunk;
+  L.nwords = (s->N_max + 31) / 32;
+  const size_t bh = (size_t)s->B * s->Hq;
+  size_t off = sizeof(WsHeader);
+  L.logits = off;
+  off += align256(bh * s->N_max * 4);
+  L.part_ml = off;
+  off += align256(bh * L.nchunk * 2 * 4);
+  L.part_acc = off;
+  off += align256(bh * L.nchunk * s->d * 4);
+  L.bitmaps = off;
+  off += align256(bh * L.nwords * 4);
+  L.total = off;
+  return L;
+}
+
+bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0; }
+
+size_t elem_size(const lychee_shape* s) { return s->dtype == LYCHEE_BF16 ? 2 : 4; }
+
+lychee_status check_roles(const uint8_t* role, int Hq, int* n_sparse) {
+  if (!role) return LYCHEE_ERR_INVALID_ARG;
+  int ns = 0;
+  for (int h = 0; h < Hq; ++h) {
+    if (role[h] != LYCHEE_ROLE_SPARSE && role[h] != LYCHEE_ROLE_RETRIEVAL)
+      return LYCHEE_ERR_INVALID_ARG;
+    ns += role[h] == LYCHEE_ROLE_SPARSE;
+  }
+  if (n_sparse) *n_sparse = ns;
+  return LYCHEE_OK;
+}
+
+// ---- device properties -----------------------------------------------------------
+int num_sms_current() {
+  static std::mutex mu;
+  static std::vector<int> cache;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return -1;
+  std::lock_guard<std::mutex> g(mu);
+  if ((int)cache.size() <= dev) cache.resize(dev + 1, 0);
+  if (cache[dev] == 0) {
+    int n = 0;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return -1;
+    cache[dev] = n;
+  }
+  return cache[dev];
+}
+
+// ---- optional launch profiler ----------------------------------------------------
+struct Profiler {
+  std::mutex mu;
+  bool on = false;
+  int cap = 0, n = 0;
+  std::vector<cudaEvent_t> ev;
+  std::vector<int32_t> kinds;
+};
+Profiler g_prof;
+
+enum { kKindAttn = 0, kKindTopk = 1, kKindCombine = 2, kKindBuildBits = 3, kKindExport = 4 };
+
+template <typename F>
+cudaError_t timed(int kind, cudaStream_t st, F&& launch) {
+  if (!g_prof.on) return launch();
+  std::lock_guard<std::mutex> g(g_prof.mu);
+  if (!g_prof.on || g_prof.n >= g_prof.cap) return launch();
+  const int i = g_prof.n++;
+  g_prof.kinds[i] = kind;
+  cudaEventRecord(g_prof.ev[2 * i], st);
+  const cudaError_t e = launch();
+  cudaEventRecord(g_prof.ev[2 * i + 1], st);
+  return e;
+}
+
+void fill_roles(uint32_t (&bits)[4], const uint8_t* role, int Hq) {
+  bits[0] = bits[1] = bits[2] = bits[3] = 0;
+  for (int h = 0; h < Hq; ++h)
+    if (role[h] == LYCHEE_ROLE_RETRIEVAL) bits[h >> 5] |= 1u << (h & 31);
+}
+
+struct Ctx {
+  const lychee_shape* s;
+  Layout L;
+  unsigned char* ws;
+  cudaStream_t st;
+  int sms;
+  WsHeader* hdr() const { return reinterpret_cast<WsHeader*>(ws); }
+};
+
+// One layer's launches.  bitmaps carry the sets of sparse heads in and (when
+// write_bits) the sets of retrieval heads out.
+lychee_status run_layer(const Ctx& c, const void* q, const void* kc, const void* vc,
+                        const int32_t* seqlens, const int32_t* k_per_seq, const uint8_t* role,
+                        const int32_t* idx_in, void* out, int32_t* idx_out, bool build_bits,
+                        bool write_bits) {
+  const lychee_shape* s = c.s;
+  const int Hq = s->Hq, G = Hq / s->Hkv;
+  uint32_t* err = &c.hdr()->err;
+  uint32_t* counter = &c.hdr()->counters[0];
+  float* logits = reinterpret_cast<float*>(c.ws + c.L.logits);
+  float* part_ml = reinterpret_cast<float*>(c.ws + c.L.part_ml);
+  float* part_acc = reinterpret_cast<float*>(c.ws + c.L.part_acc);
+  uint32_t* bitmaps = reinterpret_cast<uint32_t*>(c.ws + c.L.bitmaps);
+  uint8_t rheads[kMaxHq], sheads[kMaxHq];
+  int nr = 0, ns = 0;
+  for (int h = 0; h < Hq; ++h) {
+    if (role[h] == LYCHEE_ROLE_RETRIEVAL) rheads[nr++] = (uint8_t)h;
+    else sheads[ns++] = (uint8_t)h;
+  }
+  cudaError_t e = cudaSuccess;
+  if (build_bits && ns > 0) {
+    BuildBitsParams bp{};
+    bp.idx_in = idx_in;
+    bp.seqlens = seqlens;
+    bp.k_per_seq = k_per_seq;
+    bp.bitmaps = bitmaps;
+    bp.err = err;
+    bp.B = s->B; bp.Hq = Hq; bp.N_max = s->N_max; bp.nwords = c.L.nwords; bp.k = s->k;
+    bp.nheads = ns;
+    std::memcpy(bp.heads, sheads, ns);
+    e = timed(kKindBuildBits, c.st, [&] { return launch_build_bits(bp, c.st); });
+    if (e != cudaSuccess) return LYCHEE_ERR_CUDA;
+  }
+  AttnParams ap{};
+  ap.q = q; ap.k = kc; ap.v = vc;
+  ap.seqlens = seqlens;
+  ap.bitmaps = bitmaps;
+  ap.logits = logits;
+  ap.part_ml = part_ml;
+  ap.part_acc = part_acc;
+  ap.err = err;
+  ap.counter = counter;
+  ap.B = s->B; ap.Hq = Hq; ap.Hkv = s->Hkv; ap.N_max = s->N_max;
+  ap.nwords = c.L.nwords; ap.nchunk = c.L.nchunk;
+  ap.n_items = s->B * s->Hkv * c.L.nchunk;
+  ap.scale_log2 = (float)(1.4426950408889634 / std::sqrt((double)s->d));
+  fill_roles(ap.role, role, Hq);
+  e = timed(kKindAttn, c.st, [&] { return launch_attn(ap, s->dtype, s->d, G, c.sms, c.st); });
+  if (e != cudaSuccess) return LYCHEE_ERR_CUDA;
+  if (nr > 0) {
+    TopkParams tp{};
+    tp.logits = logits;
+    tp.seqlens = seqlens;
+    tp.k_per_seq = k_per_seq;
+    tp.bitmaps = write_bits ? bitmaps : nullptr;
+    tp.idx_out = idx_out;
+    tp.err = err;
+    tp.B = s->B; tp.Hq = Hq; tp.N_max = s->N_max; tp.nwords = c.L.nwords; tp.k = s->k;
+    tp.nheads = nr;
+    std::memcpy(tp.heads, rheads, nr);
+    e = timed(kKindTopk, c.st, [&] { return launch_topk(tp, c.st); });
+    if (e != cudaSuccess) return LYCHEE_ERR_CUDA;
+  }
+  CombineParams cp{};
+  cp.part_ml = part_ml;
+  cp.part_acc = part_acc;
+  cp.seqlens = seqlens;
+  cp.k_per_seq = k_per_seq;
+  cp.out = out;
+  cp.idx_in = idx_in;
+  cp.idx_out = idx_in ? idx_out : nullptr;
+  cp.err = err;
+  cp.counter = counter;
+  cp.B = s->B; cp.Hq = Hq; cp.N_max = s->N_max; cp.nchunk = c.L.nchunk; cp.k = s->k;
+  cp.scale_log2 = ap.scale_log2;
+  std::memcpy(cp.role, ap.role, sizeof(cp.role));
+  e = timed(kKindCombine, c.st, [&] { return launch_combine(cp, s->dtype, s->d, c.st); });
+  if (e != cudaSuccess) return LYCHEE_ERR_CUDA;
+  return LYCHEE_OK;
+}
+
+lychee_status export_sets(const Ctx& c, const int32_t* seqlens, int32_t* idx) {
+  ExportParams xp{};
+  xp.bitmaps = reinterpret_cast<const uint32_t*>(c.ws + c.L.bitmaps);
+  xp.seqlens = seqlens;
+  xp.idx = idx;
+  xp.B = c.s->B; xp.Hq = c.s->Hq; xp.N_max = c.s->N_max; xp.nwords = c.L.nwords; xp.k = c.s->k;
+  const cudaError_t e = timed(kKindExport, c.st, [&] { return launch_export(xp, c.st); });
+  return e == cudaSuccess ? LYCHEE_OK : LYCHEE_ERR_CUDA;
+}
+
+}  // namespace
+
+extern "C" {
+
+size_t lychee_workspace_size(const lychee_shape* s) {
+  if (check_shape(s) != LYCHEE_OK) return 0;
+  return layout_of(s).total;
+}
+
+lychee_status lychee_workspace_offsets(const lychee_shape* s, size_t* logits_off,
+                                      size_t* bitmaps_off, int32_t* nwords) {
+  if (check_shape(s) != LYCHEE_OK || !logits_off || !bitmaps_off || !nwords)
+    return LYCHEE_ERR_INVALID_ARG;
+  const Layout L = layout_of(s);
+  *logits_off = L.logits;
+  *bitmaps_off = L.bitmaps;
+  *nwords = L.nwords;
+  return LYCHEE_OK;
+}
+
+lychee_status lychee_hybrid_decode_attn(const lychee_shape* s, const void* q,
+                                        const void* k_cache, const void* v_cache,
+                                        const int32_t* seqlens, const int32_t* k_per_seq,
+                                        const uint8_t* head_role, const int32_t* idx_in,
+                                        void* out, int32_t* idx_out, void* workspace,
+                                        size_t workspace_bytes, void* stream) {
+  lychee_status st = check_shape(s);
+  if (st != LYCHEE_OK) return st;
+  int ns = 0;
+  if ((st = check_roles(head_role, s->Hq, &ns)) != LYCHEE_OK) return st;
+  if (!q || !k_cache || !v_cache || !seqlens || !out || !idx_out) return LYCHEE_ERR_INVALID_ARG;
+  if (ns > 0 && !idx_in) return LYCHEE_ERR_INVALID_ARG;
+  if (!aligned(q, 16) || !aligned(k_cache, 16) || !aligned(v_cache, 16) || !aligned(out, 16))
+    return LYCHEE_ERR_INVALID_ARG;
+  const Layout L = layout_of(s);
+  if (!workspace || workspace_bytes < L.total || !aligned(workspace, 256))
+    return LYCHEE_ERR_WORKSPACE;
+  Ctx c{s, L, static_cast<unsigned char*>(workspace), static_cast<cudaStream_t>(stream), 0};
+  if ((c.sms = num_sms_current()) <= 0) return LYCHEE_ERR_CUDA;
+  if (cudaMemsetAsync(workspace, 0, sizeof(WsHeader), c.st) != cudaSuccess) return LYCHEE_ERR_CUDA;
+  return run_layer(c, q, k_cache, v_cache, seqlens, k_per_seq, head_role, ns > 0 ? idx_in : nullptr,
+                   out, idx_out, /*build_bits=*/true, /*write_bits=*/false);
+}
+
+lychee_status lychee_decode_stack(const lychee_shape* s, int32_t L, const void* q,
+                                  const void* const* k_caches, const void* const* v_caches,
+                                  const int32_t* seqlens, const int32_t* k_per_seq,
+                                  const uint8_t* head_role, void* out, int32_t* idx_final,
+                                  int32_t* idx_layers, void* workspace, size_t workspace_bytes,
+                                  void* stream) {
+  lychee_status st = check_shape(s);
+  if (st != LYCHEE_OK) return st;
+  if (L < 1 || !q || !k_caches || !v_caches || !seqlens || !head_role || !out || !idx_final)
+    return LYCHEE_ERR_INVALID_ARG;
+  if (!aligned(q, 16) || !aligned(out, 16)) return LYCHEE_ERR_INVALID_ARG;
+  for (int l = 0; l < L; ++l) {
+    if ((st = check_roles(head_role + (size_t)l * s->Hq, s->Hq, nullptr)) != LYCHEE_OK) return st;
+    if (!k_caches[l] || !v_caches[l] || !aligned(k_caches[l], 16) || !aligned(v_caches[l], 16))
+      return LYCHEE_ERR_INVALID_ARG;
+  }
+  for (int h = 0; h < s->Hq; ++h)
+    if (head_role[h] != LYCHEE_ROLE_RETRIEVAL) return LYCHEE_ERR_INVALID_ARG;
+  const Layout lay = layout_of(s);
+  if (!workspace || workspace_bytes < lay.total || !aligned(workspace, 256))
+    return LYCHEE_ERR_WORKSPACE;
+  Ctx c{s, lay, static_cast<unsigned char*>(workspace), static_cast<cudaStream_t>(stream), 0};
+  if ((c.sms = num_sms_current()) <= 0) return LYCHEE_ERR_CUDA;
+  if (cudaMemsetAsync(workspace, 0, sizeof(WsHeader), c.st) != cudaSuccess) return LYCHEE_ERR_CUDA;
+  const size_t layer_elems = (size_t)s->B * s->Hq * s->d;
+  const size_t esz = elem_size(s);
+  for (int l = 0; l < L; ++l) {
+    const char* ql = static_cast<const char*>(q) + (size_t)l * layer_elems * esz;
+    char* ol = static_cast<char*>(out) + (size_t)l * layer_elems * esz;
+    st = run_layer(c, ql, k_caches[l], v_caches[l], seqlens, k_per_seq,
+                   head_role + (size_t)l * s->Hq, nullptr, ol, nullptr, /*build_bits=*/false,
+                   /*write_bits=*/true);
+    if (st != LYCHEE_OK) return st;
+    if (idx_layers) {
+      st = export_sets(c, seqlens, idx_layers + (size_t)l * s->B * s->Hq * s->k);
+      if (st != LYCHEE_OK) return st;
+    }
+  }
+  return export_sets(c, seqlens, idx_final);
+}
+
+lychee_status lychee_check_device_error(void* workspace, void* stream, uint32_t* detail) {
+  if (!workspace) return LYCHEE_ERR_INVALID_ARG;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  uint32_t v = 0;
+  if (cudaStreamSynchronize(st) != cudaSuccess) return LYCHEE_ERR_CUDA;
+  if (cudaMemcpy(&v, workspace, sizeof(v), cudaMemcpyDeviceToHost) != cudaSuccess)
+    return LYCHEE_ERR_CUDA;
+  if (cudaMemset(workspace, 0, sizeof(v)) != cudaSuccess) return LYCHEE_ERR_CUDA;
+  if (detail) *detail = v;
+  if (v & kErrTimeout) return LYCHEE_ERR_TIMEOUT;
+  if (v) return LYCHEE_ERR_BAD_INDEX;
+  return LYCHEE_OK;
+}
+
+const char* lychee_status_string(lychee_status st) {
+  switch (st) {
+    case LYCHEE_OK: return "ok";
+    case LYCHEE_ERR_INVALID_ARG: return "invalid argument";
+    case LYCHEE_ERR_UNSUPPORTED: return "unsupported shape";
+    case LYCHEE_ERR_WORKSPACE: return "workspace missing, misaligned or too small";
+    case LYCHEE_ERR_CUDA: return "CUDA error";
+    case LYCHEE_ERR_BAD_INDEX: return "bad incoming index, sequence length or budget";
+    case LYCHEE_ERR_TIMEOUT: return "device wait timed out";
+  }
+  return "unknown status";
+}
+
+int32_t lychee_version(void) { return kVersion; }
+
+lychee_status lychee_profile_begin(int32_t max_launches) {
+  if (max_launches < 1) return LYCHEE_ERR_INVALID_ARG;
+  std::lock_guard<std::mutex> g(g_prof.mu);
+  if (g_prof.on) return LYCHEE_ERR_INVALID_ARG;
+  if ((int)g_prof.ev.size() < 2 * max_launches) {
+    const size_t old = g_prof.ev.size();
+    g_prof.ev.resize(2 * (size_t)max_launches);
+    for (size_t i = old; i < g_prof.ev.size(); ++i)
+      if (cudaEventCreate(&g_prof.ev[i]) != cudaSuccess) {
+        g_prof.ev.resize(i);
+        return LYCHEE_ERR_CUDA;
+      }
+  }
+  g_prof.kinds.assign(max_launches, -1);
+  g_prof.cap = max_launches;
+  g_prof.n = 0;
+  g_prof.on = true;
+  return LYCHEE_OK;
+}
+
+lychee_status lychee_profile_end(int32_t capacity, int32_t* kinds, float* ms, int32_t* n_out) {
+  std::lock_guard<std::mutex> g(g_prof.mu);
+  if (!g_prof.on) return LYCHEE_ERR_INVALID_ARG;
+  g_prof.on = false;
+  const int n = g_prof.n;
+  if (n_out) *n_out = n;
+  for (int i = 0; i < n && i < capacity; ++i) {
+    if (cudaEventSynchronize(g_prof.ev[2 * i + 1]) != cudaSuccess) return LYCHEE_ERR_CUDA;
+    float t = 0.f;
+    if (cudaEventElapsedTime(&t, g_prof.ev[2 * i], g_prof.ev[2 * i + 1]) != cudaSuccess)
+      return LYCHEE_ERR_CUDA;
+    if (kinds) kinds[i] = g_prof.kinds[i];
+    if (ms) ms[i] = t;
+  }
+  return LYCHEE_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,173 @@
+// common.cuh -- device helpers shared by the libychee kernels (sm_100a).
+//
+// Everything here is plain inline PTX for the Hopper/Blackwell asynchronous
+// copy machinery (mbarrier, 1-D bulk copies into shared memory, cluster
+// barriers and distributed shared memory) plus the workspace layout.  No TMA
+// copy here uses cluster multicast, and every source address is this GPU's own
+// global memory.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace lychee {
+
+// ---- device error word (workspace header) ---------------------------------
+enum : uint32_t {
+  kErrBadIndex = 1u,    // incoming index out of range or not strictly ascending
+  kErrBadSeqlen = 2u,   // n_b outside [1, N_max] (clamped)
+  kErrBadBudget = 4u,   // k_per_seq[b] < 1 (clamped to 1)
+  kErrTimeout = 8u,     // a pipeline wait gave up
+};
+
+// Workspace header: 256 bytes at offset 0.
+struct WsHeader {
+  uint32_t err;          // error bits (above)
+  uint32_t pad0[15];
+  uint32_t counters[48]; // per-launch work counters (zeroed at the start of a call)
+};
+static_assert(sizeof(WsHeader) == 256, "header is 256 bytes");
+
+constexpr int kChunk = 1024;          // positions per attention work item
+constexpr int kMaxHq = 128;           // query heads supported
+constexpr uint64_t kWaitLimitNs = 2000000000ull;   // 2 s: a wait this long is a fault
+
+__device__ __forceinline__ uint64_t globaltimer() {
+  uint64_t t;
+  asm volatile("mov.u64 %0, %globaltimer;" : "=l"(t));
+  return t;
+}
+
+__device__ __forceinline__ void flag_error(uint32_t* err, uint32_t bits) {
+  if (err) atomicOr(err, bits);
+}
+
+// ---- shared-memory addresses -----------------------------------------------
+__device__ __forceinline__ uint32_t smem_u32(const void* p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+// ---- mbarrier ------------------------------------------------------------------
+__device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count)
+               : "memory");
+}
+
+__device__ __forceinline__ void fence_mbar_init() {
+  asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.release.cta.shared::cta.b64 _, [%0], %1;" ::"r"(
+                   smem_u32(bar)),
+               "r"(bytes)
+               : "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
+  asm volatile("mbarrier.arrive.release.cta.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar))
+               : "memory");
+}
+
+__device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.acquire.cta.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
+// Wait for the phase with the given parity to complete.  Gives up after
+// kWaitLimitNs, sets kErrTimeout and returns false; the caller then leaves.
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, uint32_t* err) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = globaltimer();
+  uint32_t spins = 0;
+  while (!mbar_try_wait(bar, parity)) {
+    if ((++spins & 255u) == 0u && globaltimer() - t0 > kWaitLimitNs) {
+      flag_error(err, kErrTimeout);
+      return false;
+    }
+  }
+  return true;
+}
+
+// ---- 1-D bulk copy global -> shared (TMA, no tensor map, no multicast) ------
+// dst and src 16-byte aligned, bytes a multiple of 16.  Completion is signalled
+// as transaction bytes on `bar`.  The L2 policy marks the streamed cache rows
+// evict-first: they are read once per step.
+__device__ __forceinline__ uint64_t l2_evict_first_policy() {
+  uint64_t pol;
+  asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(pol));
+  return pol;
+}
+
+__device__ __forceinline__ void bulk_g2s(void* dst, const void* src, uint32_t bytes,
+                                         uint64_t* bar, uint64_t policy) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint"
+      " [%0], [%1], %2, [%3], %4;" ::"r"(smem_u32(dst)),
+      "l"(src), "r"(bytes), "r"(smem_u32(bar)), "l"(policy)
+      : "memory");
+}
+
+// ---- named barriers (a subset of the CTA's warps) ------------------------------
+__device__ __forceinline__ void named_bar_sync(uint32_t id, uint32_t nthreads) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
+}
+
+// ---- clusters / distributed shared memory ---------------------------------------
+__device__ __forceinline__ uint32_t cluster_ctarank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return r;
+}
+
+__device__ __forceinline__ void cluster_sync() {
+  asm volatile("barrier.cluster.arrive.release.aligned;\n\t"
+               "barrier.cluster.wait.acquire.aligned;" ::
+                   : "memory");
+}
+
+// Address of `p` (a shared variable of this CTA) in the shared window of CTA
+// `rank` of the cluster.
+__device__ __forceinline__ uint32_t dsmem_addr(const void* p, uint32_t rank) {
+  uint32_t out;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(out) : "r"(smem_u32(p)), "r"(rank));
+  return out;
+}
+
+__device__ __forceinline__ uint32_t dsmem_ld_u32(uint32_t addr) {
+  uint32_t v;
+  asm volatile("ld.shared::cluster.u32 %0, [%1];" : "=r"(v) : "r"(addr) : "memory");
+  return v;
+}
+
+// ---- numeric helpers --------------------------------------------------------------
+// 2^x on the special-function unit (PTX ex2.approx; max relative error about
+// 2^-22 over the range used here).
+__device__ __forceinline__ float fast_exp2(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
+// Order-preserving map of an fp32 value to uint32 (larger float -> larger key).
+// -0.0 is folded onto +0.0 so that equal values compare equal.
+__device__ __forceinline__ uint32_t float_to_key(float f) {
+  uint32_t u = __float_as_uint(f);
+  if (u == 0x80000000u) u = 0u;
+  return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+
+// bf16x2 in one 32-bit word -> two fp32 (exact widening).
+__device__ __forceinline__ float2 bf16x2_to_float2(uint32_t w) {
+  return make_float2(__uint_as_float(w << 16), __uint_as_float(w & 0xffff0000u));
+}
+
+}  // namespace lychee

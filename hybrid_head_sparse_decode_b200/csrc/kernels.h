@@ -1,0 +1,79 @@
+// kernels.h -- parameter blocks and launchers of the libychee kernels (internal).
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace lychee {
+
+// Hybrid attention over one layer (attn.cu).
+struct AttnParams {
+  const void* q;            // [B, Hq, D]
+  const void* k;            // [B, Hkv, N_max, D]
+  const void* v;            // [B, Hkv, N_max, D]
+  const int32_t* seqlens;   // [B]
+  const uint32_t* bitmaps;  // [B, Hq, nwords]: incoming sets of sparse heads
+  float* logits;            // [B, Hq, N_max]: raw q.k of retrieval heads
+  float* part_ml;           // [B, Hq, nchunk, 2]: (max raw dot, sum of weights)
+  float* part_acc;          // [B, Hq, nchunk, D]: unnormalised weighted values
+  uint32_t* err;
+  uint32_t* counter;        // work-item counter, 0 at launch
+  int B, Hq, Hkv, N_max, nwords, nchunk, n_items;
+  float scale_log2;         // log2(e) / sqrt(D)
+  uint32_t role[4];         // bit h set: head h is a retrieval head
+};
+cudaError_t launch_attn(const AttnParams& p, int dtype, int D, int G, int num_sms,
+                        cudaStream_t st);
+
+// argsTopK of retrieval heads (topk.cu).
+struct TopkParams {
+  const float* logits;       // [B, Hq, N_max]
+  const int32_t* seqlens;    // [B]
+  const int32_t* k_per_seq;  // [B] or null
+  uint32_t* bitmaps;         // [B, Hq, nwords] or null: selected set as bits
+  int32_t* idx_out;          // [B, Hq, k] or null: selected set, ascending, -1 padded
+  uint32_t* err;
+  int B, Hq, N_max, nwords, k, nheads;
+  uint8_t heads[128];        // the retrieval heads handled by this launch
+};
+cudaError_t launch_topk(const TopkParams& p, cudaStream_t st);
+
+// Merge of split partials, output rounding, set pass-through (combine.cu).
+struct CombineParams {
+  const float* part_ml;
+  const float* part_acc;
+  const int32_t* seqlens;
+  const int32_t* k_per_seq;  // [B] or null (validated here)
+  void* out;                 // [B, Hq, D]
+  const int32_t* idx_in;     // [B, Hq, k] or null
+  int32_t* idx_out;          // [B, Hq, k] or null: rows of sparse heads copied from idx_in
+  uint32_t* err;
+  uint32_t* counter;         // reset to 0 for the next attention launch
+  int B, Hq, N_max, nchunk, k;
+  float scale_log2;
+  uint32_t role[4];
+};
+cudaError_t launch_combine(const CombineParams& p, int dtype, int D, cudaStream_t st);
+
+// Incoming index sets -> membership bitmaps, with validation (sets.cu).
+struct BuildBitsParams {
+  const int32_t* idx_in;     // [B, Hq, k]
+  const int32_t* seqlens;
+  const int32_t* k_per_seq;
+  uint32_t* bitmaps;         // [B, Hq, nwords]
+  uint32_t* err;
+  int B, Hq, N_max, nwords, k, nheads;
+  uint8_t heads[128];        // the sparse heads whose sets are built
+};
+cudaError_t launch_build_bits(const BuildBitsParams& p, cudaStream_t st);
+
+// Membership bitmaps -> index rows (ascending, -1 padded) for every head (sets.cu).
+struct ExportParams {
+  const uint32_t* bitmaps;
+  const int32_t* seqlens;
+  int32_t* idx;              // [B, Hq, k]
+  int B, Hq, N_max, nwords, k;
+};
+cudaError_t launch_export(const ExportParams& p, cudaStream_t st);
+
+}  // namespace lychee

@@ -1,0 +1,201 @@
+"""Torch-facing calls of libychee: the hybrid-head sparse decode-attention step.
+
+    out, idx_out = hybrid_decode_attn(q, k_cache, v_cache, seqlens, head_role, idx_in, k)
+    out, idx_final, idx_layers = decode_stack(q, k_caches, v_caches, seqlens, head_roles, k)
+
+Method: page "LycheeDecode: Accelerating Long-Context LLM Inference via
+Hybrid-Head Sparse Decoding" (paper.rainbus.top/paper/2602.04541), steps (1),
+(3), (4), (7).  Shapes and conventions are those of include/lychee.h; this module
+only checks that tensors live on a CUDA device with the expected dtype and
+layout, allocates outputs/workspace with torch when the caller does not pass
+them, and hands raw pointers to the library on the current (or given) stream.
+"""
+from __future__ import annotations
+
+import ctypes
+
+import torch
+
+from . import _native as N
+
+_DT = {torch.bfloat16: N.BF16, torch.float32: N.FP32}
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream_handle(stream):
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _need_cuda(name, t, dtype=None, shape=None):
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch.Tensor")
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be on a CUDA device (there is no CPU path)")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if dtype is not None and t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    if shape is not None and tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} must have shape {tuple(shape)}, got {tuple(t.shape)}")
+
+
+def make_shape(B, Hq, Hkv, d, N_max, k, dtype) -> N.Shape:
+    code = _DT.get(dtype, dtype)
+    return N.Shape(int(B), int(Hq), int(Hkv), int(d), int(N_max), int(code), int(k))
+
+
+def workspace_size(B, Hq, Hkv, d, N_max, k, dtype) -> int:
+    sh = make_shape(B, Hq, Hkv, d, N_max, k, dtype)
+    n = N.load().lychee_workspace_size(ctypes.byref(sh))
+    if n == 0:
+        raise N.LycheeError(N.ERR_INVALID_ARG, "workspace_size")
+    return int(n)
+
+
+def alloc_workspace(B, Hq, Hkv, d, N_max, k, dtype, device=None) -> torch.Tensor:
+    n = workspace_size(B, Hq, Hkv, d, N_max, k, dtype)
+    return torch.empty(n, dtype=torch.uint8, device=device or "cuda")
+
+
+def _roles_host(role, n_expected):
+    r = torch.as_tensor(role, dtype=torch.uint8).contiguous().cpu()
+    if r.numel() != n_expected:
+        raise ValueError(f"head_role must have {n_expected} entries")
+    return r
+
+
+def _check(st, what):
+    if st != N.OK:
+        raise N.LycheeError(st, what)
+
+
+def hybrid_decode_attn(q, k_cache, v_cache, seqlens, head_role, idx_in, k, *, k_per_seq=None,
+                       out=None, idx_out=None, workspace=None, stream=None):
+    """One hybrid-head layer.  q [B,Hq,d]; caches [B,Hkv,N_max,d] (bf16 or fp32);
+    seqlens [B] int32 (device); head_role [Hq] (host, 1 = retrieval);
+    idx_in [B,Hq,k] int32 (device, or None when every head is retrieval).
+    Returns (out [B,Hq,d], idx_out [B,Hq,k])."""
+    B, Hq, d = q.shape
+    _, Hkv, N_max, _ = k_cache.shape
+    _need_cuda("q", q)
+    dt = q.dtype
+    _need_cuda("k_cache", k_cache, dt, (B, Hkv, N_max, d))
+    _need_cuda("v_cache", v_cache, dt, (B, Hkv, N_max, d))
+    _need_cuda("seqlens", seqlens, torch.int32, (B,))
+    if k_per_seq is not None:
+        _need_cuda("k_per_seq", k_per_seq, torch.int32, (B,))
+    if idx_in is not None:
+        _need_cuda("idx_in", idx_in, torch.int32, (B, Hq, k))
+    role = _roles_host(head_role, Hq)
+    if out is None:
+        out = torch.empty((B, Hq, d), dtype=dt, device=q.device)
+    _need_cuda("out", out, dt, (B, Hq, d))
+    if idx_out is None:
+        idx_out = torch.empty((B, Hq, k), dtype=torch.int32, device=q.device)
+    _need_cuda("idx_out", idx_out, torch.int32, (B, Hq, k))
+    sh = make_shape(B, Hq, Hkv, d, N_max, k, dt)
+    if workspace is None:
+        workspace = alloc_workspace(B, Hq, Hkv, d, N_max, k, dt, q.device)
+    _need_cuda("workspace", workspace, torch.uint8)
+    st = N.load().lychee_hybrid_decode_attn(
+        ctypes.byref(sh), _ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(seqlens), _ptr(k_per_seq),
+        ctypes.c_void_p(role.data_ptr()), _ptr(idx_in), _ptr(out), _ptr(idx_out),
+        _ptr(workspace), ctypes.c_size_t(workspace.numel()), _stream_handle(stream))
+    _check(st, "lychee_hybrid_decode_attn")
+    return out, idx_out
+
+
+def decode_stack(q, k_caches, v_caches, seqlens, head_roles, k, *, k_per_seq=None, out=None,
+                 idx_final=None, idx_layers=None, want_layers=False, workspace=None, stream=None):
+    """L chained layers of one decode step.  q [L,B,Hq,d]; k_caches / v_caches:
+    sequences of L tensors [B,Hkv,N_max,d]; head_roles [L,Hq] (host, row 0 all
+    retrieval).  Returns (out [L,B,Hq,d], idx_final [B,Hq,k], idx_layers or None)."""
+    L, B, Hq, d = q.shape
+    if len(k_caches) != L or len(v_caches) != L:
+        raise ValueError("need one K and one V cache per layer")
+    _need_cuda("q", q)
+    dt = q.dtype
+    _, Hkv, N_max, _ = k_caches[0].shape
+    for l in range(L):
+        _need_cuda(f"k_caches[{l}]", k_caches[l], dt, (B, Hkv, N_max, d))
+        _need_cuda(f"v_caches[{l}]", v_caches[l], dt, (B, Hkv, N_max, d))
+    _need_cuda("seqlens", seqlens, torch.int32, (B,))
+    if k_per_seq is not None:
+        _need_cuda("k_per_seq", k_per_seq, torch.int32, (B,))
+    roles = _roles_host(head_roles, L * Hq)
+    if out is None:
+        out = torch.empty((L, B, Hq, d), dtype=dt, device=q.device)
+    _need_cuda("out", out, dt, (L, B, Hq, d))
+    if idx_final is None:
+        idx_final = torch.empty((B, Hq, k), dtype=torch.int32, device=q.device)
+    _need_cuda("idx_final", idx_final, torch.int32, (B, Hq, k))
+    if idx_layers is None and want_layers:
+        idx_layers = torch.empty((L, B, Hq, k), dtype=torch.int32, device=q.device)
+    if idx_layers is not None:
+        _need_cuda("idx_layers", idx_layers, torch.int32, (L, B, Hq, k))
+    sh = make_shape(B, Hq, Hkv, d, N_max, k, dt)
+    if workspace is None:
+        workspace = alloc_workspace(B, Hq, Hkv, d, N_max, k, dt, q.device)
+    _need_cuda("workspace", workspace, torch.uint8)
+    kp = (ctypes.c_void_p * L)(*[t.data_ptr() for t in k_caches])
+    vp = (ctypes.c_void_p * L)(*[t.data_ptr() for t in v_caches])
+    st = N.load().lychee_decode_stack(
+        ctypes.byref(sh), ctypes.c_int32(L), _ptr(q), ctypes.cast(kp, ctypes.c_void_p),
+        ctypes.cast(vp, ctypes.c_void_p), _ptr(seqlens), _ptr(k_per_seq),
+        ctypes.c_void_p(roles.data_ptr()), _ptr(out), _ptr(idx_final), _ptr(idx_layers),
+        _ptr(workspace), ctypes.c_size_t(workspace.numel()), _stream_handle(stream))
+    _check(st, "lychee_decode_stack")
+    return out, idx_final, idx_layers
+
+
+def check_device_error(workspace, stream=None):
+    """Synchronise, read and clear the device error word.  Returns (status, bits)."""
+    _need_cuda("workspace", workspace, torch.uint8)
+    bits = ctypes.c_uint32(0)
+    st = N.load().lychee_check_device_error(_ptr(workspace), _stream_handle(stream),
+                                            ctypes.byref(bits))
+    return int(st), int(bits.value)
+
+
+def workspace_views(workspace, B, Hq, Hkv, d, N_max, k, dtype):
+    """Views into the documented workspace regions (for inspection in tests):
+    logits [B,Hq,N_max] fp32 (raw q.k of the most recent layer's retrieval
+    heads) and bitmaps [B,Hq,ceil(N_max/32)] int32 (bit patterns of the sets)."""
+    sh = make_shape(B, Hq, Hkv, d, N_max, k, dtype)
+    lo, bo, nw = ctypes.c_size_t(0), ctypes.c_size_t(0), ctypes.c_int32(0)
+    _check(N.load().lychee_workspace_offsets(ctypes.byref(sh), ctypes.byref(lo), ctypes.byref(bo),
+                                             ctypes.byref(nw)), "lychee_workspace_offsets")
+    lo, bo, nw = lo.value, bo.value, nw.value
+    logits = workspace[lo: lo + B * Hq * N_max * 4].view(torch.float32).view(B, Hq, N_max)
+    bitmaps = workspace[bo: bo + B * Hq * nw * 4].view(torch.int32).view(B, Hq, nw)
+    return logits, bitmaps
+
+
+class Profile:
+    """Context manager around lychee_profile_begin / lychee_profile_end.
+    After exit, ``records`` is a list of (kind, ms) per library launch."""
+    KINDS = {0: "attn", 1: "topk", 2: "combine", 3: "build_bits", 4: "export"}
+
+    def __init__(self, max_launches=4096):
+        self.max_launches = int(max_launches)
+        self.records = []
+
+    def __enter__(self):
+        _check(N.load().lychee_profile_begin(self.max_launches), "lychee_profile_begin")
+        return self
+
+    def __exit__(self, *exc):
+        cap = self.max_launches
+        kinds = (ctypes.c_int32 * cap)()
+        ms = (ctypes.c_float * cap)()
+        n = ctypes.c_int32(0)
+        _check(N.load().lychee_profile_end(cap, ctypes.cast(kinds, ctypes.c_void_p),
+                                           ctypes.cast(ms, ctypes.c_void_p), ctypes.byref(n)),
+               "lychee_profile_end")
+        self.records = [(self.KINDS.get(kinds[i], str(kinds[i])), float(ms[i]))
+                        for i in range(min(n.value, cap))]
+        return False

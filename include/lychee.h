@@ -1,0 +1,174 @@
+/*
+ * lychee.h -- C ABI of libychee, a B200 (sm_100a) implementation of the
+ * hybrid-head sparse decode-attention step of LycheeDecode.
+ *
+ * The operation (page "LycheeDecode: Accelerating Long-Context LLM Inference
+ * via Hybrid-Head Sparse Decoding", paper.rainbus.top/paper/2602.04541, method
+ * steps (1), (3), (4), (7)): at one new token, for every layer,
+ *   - a retrieval head h computes s_j = q_h . K_{g,j} / sqrt(d) over every
+ *     position j < n_b of its KV group g, O_h = softmax(s) V_g, and hands
+ *     S' = argsTopK(s, k_b) to the head at the same index h of the next layer;
+ *   - a sparse head h computes O_h = softmax(q_h . K_{g,S}^T / sqrt(d)) V_{g,S}
+ *     over its incoming set S only and hands S on unchanged;
+ *   - layer 0 is all retrieval (step (1)); roles are fixed inputs (step (7)).
+ * The budget k_b = 30% of the sequence length comes from the same page's
+ * reproduction paragraph; the caller passes it.
+ *
+ * Conventions shared by every entry point
+ *   - GQA: query head h reads KV head g = h / G with G = Hq / Hkv (consecutive
+ *     query heads share a KV head).
+ *   - Index sets are int32 rows of capacity k: the first k_b entries are the
+ *     set in strictly ascending position order, the rest are -1.
+ *     k_b = min(k_per_seq[b] (or k when k_per_seq is NULL), k, n_b).
+ *   - argsTopK ranks positions by larger logit first and, on equal logits, by
+ *     lower position; the returned set is in ascending position order.
+ *   - Element types: LYCHEE_BF16 (16-bit bfloat16) or LYCHEE_FP32.  Arithmetic
+ *     is fp32 with fp32 accumulation; outputs are rounded to the input type
+ *     (round to nearest even).
+ *   - Ownership: the caller owns every buffer.  The library allocates no
+ *     memory, never synchronises inside a call, and launches only on `stream`
+ *     (a cudaStream_t; NULL = the legacy default stream), so a call can be
+ *     captured into a CUDA graph.  Calls sharing one workspace must be ordered
+ *     on the same stream.
+ *   - Errors found on the host (NULL pointers, unsupported shapes, short
+ *     workspace, misaligned pointers, a sparse role in layer 0 of a stack) are
+ *     returned before anything is launched.  Errors only visible on the device
+ *     (an incoming index out of range or not strictly ascending, a sequence
+ *     length outside [1, N_max], a budget below 1, a wait that gave up) never
+ *     trap: the offending entry is skipped or clamped, a flag is set in the
+ *     workspace, and lychee_check_device_error() reports it.
+ *   - Device pointers must be 16-byte aligned (q, caches, out, workspace).
+ */
+#ifndef LYCHEE_H
+#define LYCHEE_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(LYCHEE_BUILD) && defined(__GNUC__)
+#define LYCHEE_API __attribute__((visibility("default")))
+#else
+#define LYCHEE_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  LYCHEE_OK = 0,
+  LYCHEE_ERR_INVALID_ARG = 1, /* NULL pointer, bad shape, bad role value, misalignment */
+  LYCHEE_ERR_UNSUPPORTED = 2, /* shape outside what the kernels are built for      */
+  LYCHEE_ERR_WORKSPACE = 3,   /* workspace NULL or smaller than lychee_workspace_size */
+  LYCHEE_ERR_CUDA = 4,        /* a CUDA runtime call or launch failed               */
+  LYCHEE_ERR_BAD_INDEX = 5,   /* device-side: bad incoming index / length / budget  */
+  LYCHEE_ERR_TIMEOUT = 6      /* device-side: a pipeline wait gave up (never expected) */
+} lychee_status;
+
+typedef enum { LYCHEE_BF16 = 0, LYCHEE_FP32 = 1 } lychee_dtype;
+
+enum { LYCHEE_ROLE_SPARSE = 0, LYCHEE_ROLE_RETRIEVAL = 1 };
+
+/* Problem shape.  Supported: Hq % Hkv == 0 with G = Hq / Hkv in {1, 2, 4, 8},
+ * Hq <= 128, d in {64, 128}, 1 <= k <= N_max <= 2^24, B >= 1. */
+typedef struct {
+  int32_t B;      /* batch (sequences)                         */
+  int32_t Hq;     /* query heads                               */
+  int32_t Hkv;    /* key/value heads                           */
+  int32_t d;      /* head dimension                            */
+  int32_t N_max;  /* cache capacity in positions               */
+  int32_t dtype;  /* lychee_dtype of q, caches and out         */
+  int32_t k;      /* capacity of an index-set row              */
+} lychee_shape;
+
+/* Bytes of device workspace that lychee_hybrid_decode_attn and
+ * lychee_decode_stack need for shape *s (the same figure for both, any L).
+ * Returns 0 if *s is invalid.  The workspace holds fp32 logits of retrieval
+ * heads ([B, Hq, N_max], the raw dot products q.k, not divided by sqrt(d)),
+ * split partials, one membership bitmap per head position ([B, Hq,
+ * ceil(N_max/32)] uint32, bit j of word w = position 32w+j is in S), a work
+ * counter and the device error word. */
+LYCHEE_API size_t lychee_workspace_size(const lychee_shape* s);
+
+/* Byte offsets, inside a workspace for shape *s, of the fp32 logits region
+ * [B, Hq, N_max] (raw q.k of the retrieval heads of the most recent layer,
+ * positions j < n_b) and of the membership-bitmap region [B, Hq, nwords]
+ * (nwords = ceil(N_max / 32)); *nwords receives nwords.  For inspection and
+ * tests.  Returns LYCHEE_ERR_INVALID_ARG for an invalid shape or NULL output. */
+LYCHEE_API lychee_status lychee_workspace_offsets(const lychee_shape* s, size_t* logits_off,
+                                                  size_t* bitmaps_off, int32_t* nwords);
+
+/* One hybrid-head layer (method steps (3) and (4)).
+ *   q         device [B, Hq, d]          dtype
+ *   k_cache   device [B, Hkv, N_max, d]  dtype, rows j < n_b hold the cache
+ *   v_cache   device [B, Hkv, N_max, d]  dtype
+ *   seqlens   device [B] int32, 1 <= n_b <= N_max (the current token is included)
+ *   k_per_seq device [B] int32 or NULL (then k_b = min(k, n_b))
+ *   head_role HOST   [Hq] uint8, LYCHEE_ROLE_RETRIEVAL or LYCHEE_ROLE_SPARSE
+ *   idx_in    device [B, Hq, k] int32; rows of sparse heads are read (their first
+ *             k_b entries, strictly ascending, in [0, n_b)); may be NULL only
+ *             when every head is a retrieval head
+ *   out       device [B, Hq, d] dtype
+ *   idx_out   device [B, Hq, k] int32: retrieval heads get argsTopK of their
+ *             logits (ascending, -1 padded); sparse heads get their idx_in row
+ *             copied bit for bit
+ *   workspace device, >= lychee_workspace_size(s) bytes, 256-byte aligned
+ *   stream    cudaStream_t
+ * The call overwrites the whole workspace header, so device errors reported by
+ * lychee_check_device_error() refer to the most recent call on that workspace. */
+LYCHEE_API lychee_status lychee_hybrid_decode_attn(const lychee_shape* s, const void* q,
+                                        const void* k_cache, const void* v_cache,
+                                        const int32_t* seqlens, const int32_t* k_per_seq,
+                                        const uint8_t* head_role, const int32_t* idx_in,
+                                        void* out, int32_t* idx_out, void* workspace,
+                                        size_t workspace_bytes, void* stream);
+
+/* L chained layers of one decode step (method steps (1), (3), (4)): the set
+ * leaving head position h of layer l is the incoming set of head position h of
+ * layer l+1; it is carried between layers as the per-head bitmap in the
+ * workspace.
+ *   q          device [L, B, Hq, d] dtype (one query per layer)
+ *   k_caches   HOST array of L device pointers, each [B, Hkv, N_max, d]
+ *   v_caches   HOST array of L device pointers, each [B, Hkv, N_max, d]
+ *   seqlens    device [B]; k_per_seq device [B] or NULL (as above)
+ *   head_role  HOST [L, Hq] uint8; row 0 must be all retrieval
+ *   out        device [L, B, Hq, d] dtype
+ *   idx_final  device [B, Hq, k] int32: the sets leaving layer L-1
+ *   idx_layers device [L, B, Hq, k] int32 or NULL: the sets leaving every layer
+ *   workspace, stream as above. */
+LYCHEE_API lychee_status lychee_decode_stack(const lychee_shape* s, int32_t L, const void* q,
+                                  const void* const* k_caches, const void* const* v_caches,
+                                  const int32_t* seqlens, const int32_t* k_per_seq,
+                                  const uint8_t* head_role, void* out, int32_t* idx_final,
+                                  int32_t* idx_layers, void* workspace, size_t workspace_bytes,
+                                  void* stream);
+
+/* Synchronises `stream`, reads the device error word of `workspace` and clears
+ * it.  Returns LYCHEE_OK, LYCHEE_ERR_BAD_INDEX, LYCHEE_ERR_TIMEOUT or
+ * LYCHEE_ERR_CUDA.  If detail is not NULL it receives the raw flag bits
+ * (1 = bad index, 2 = bad sequence length, 4 = bad budget, 8 = wait timeout). */
+LYCHEE_API lychee_status lychee_check_device_error(void* workspace, void* stream, uint32_t* detail);
+
+/* Static, NUL-terminated description of a status code. */
+LYCHEE_API const char* lychee_status_string(lychee_status st);
+
+/* Library version as 10000*major + 100*minor + patch. */
+LYCHEE_API int32_t lychee_version(void);
+
+/* Launch profiler (measurement aid, off by default).  Between begin and end,
+ * every kernel launch of the library on any stream is bracketed by two CUDA
+ * events recorded on its launch stream, up to max_launches launches (later
+ * launches run unrecorded).  lychee_profile_end synchronises on the recorded
+ * events and writes, for the first min(n, capacity) launches, the kind
+ * (0 attention, 1 top-k, 2 combine, 3 set->bitmap, 4 bitmap->set) and the
+ * elapsed milliseconds; *n_out receives n.  Process-global state: one profiling
+ * session at a time.  Events are created on the current device on first use
+ * and kept for reuse. */
+LYCHEE_API lychee_status lychee_profile_begin(int32_t max_launches);
+LYCHEE_API lychee_status lychee_profile_end(int32_t capacity, int32_t* kinds, float* ms, int32_t* n_out);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* LYCHEE_H */

@@ -1,0 +1,127 @@
+"""The C ABI on the host: the library loads, exports every entry point that
+include/lychee.h declares, and rejects bad arguments before launching anything
+(these calls never reach the GPU, so they run without one)."""
+import ctypes
+import os
+import re
+
+import pytest
+import torch
+
+from hybrid_head_sparse_decode_b200 import build, ops
+from hybrid_head_sparse_decode_b200 import _native as N
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    build.build()
+    return N.load()
+
+
+def declared_symbols():
+    text = open(os.path.join(ROOT, "include", "lychee.h")).read()
+    return sorted(set(re.findall(r"LYCHEE_API\s+[\w\s\*]*?\b(lychee_\w+)\s*\(", text)))
+
+
+def test_header_declares_the_binding_symbols():
+    assert declared_symbols() == sorted(N.EXPORTED)
+
+
+def test_library_exports_every_declared_symbol(lib):
+    for name in declared_symbols():
+        assert hasattr(lib, name), name
+    assert lib.lychee_version() >= 100
+
+
+def shape(B=1, Hq=4, Hkv=2, d=128, N_max=1024, dtype=N.BF16, k=307):
+    return N.Shape(B, Hq, Hkv, d, N_max, dtype, k)
+
+
+def test_workspace_size_valid_and_invalid(lib):
+    s = shape()
+    n = lib.lychee_workspace_size(ctypes.byref(s))
+    # header + logits + partials + bitmaps, each 256-byte aligned
+    assert n >= 256 + 1 * 4 * 1024 * 4 + 4 * 1 * (2 + 128) * 4 + 4 * 32 * 4
+    assert n % 256 == 0
+    bad = [shape(Hq=6, Hkv=4), shape(d=96), shape(k=0), shape(k=2000), shape(Hq=48, Hkv=3),
+           shape(dtype=7), shape(B=0), shape(N_max=(1 << 24) + 1)]
+    for b in bad:
+        assert lib.lychee_workspace_size(ctypes.byref(b)) == 0
+    assert lib.lychee_workspace_size(None) == 0
+
+
+def test_workspace_offsets(lib):
+    s = shape(B=2, Hq=8, Hkv=2, N_max=5000, k=100)
+    lo, bo, nw = ctypes.c_size_t(), ctypes.c_size_t(), ctypes.c_int32()
+    assert lib.lychee_workspace_offsets(ctypes.byref(s), ctypes.byref(lo), ctypes.byref(bo),
+                                        ctypes.byref(nw)) == N.OK
+    assert lo.value == 256 and nw.value == (5000 + 31) // 32
+    total = lib.lychee_workspace_size(ctypes.byref(s))
+    assert lo.value + 2 * 8 * 5000 * 4 <= bo.value
+    assert bo.value + 2 * 8 * nw.value * 4 <= total
+
+
+FAKE = 0x10000   # 16-byte aligned, never dereferenced: every call below fails on the host
+
+
+def call_layer(lib, s, roles, ws_bytes=1 << 40, q=FAKE, idx_in=FAKE, ws=FAKE, out=FAKE):
+    r = (ctypes.c_uint8 * len(roles))(*roles)
+    return lib.lychee_hybrid_decode_attn(
+        ctypes.byref(s) if s is not None else None, q, FAKE, FAKE, FAKE, None,
+        ctypes.cast(r, ctypes.c_void_p), idx_in, out, FAKE, ws, ctypes.c_size_t(ws_bytes), None)
+
+
+def test_layer_rejects_bad_arguments_on_host(lib):
+    s = shape()
+    assert call_layer(lib, None, [1, 1, 1, 1]) == N.ERR_INVALID_ARG
+    assert call_layer(lib, shape(Hq=6, Hkv=4), [1] * 6) == N.ERR_INVALID_ARG
+    assert call_layer(lib, shape(d=96), [1] * 4) == N.ERR_UNSUPPORTED
+    assert call_layer(lib, s, [1, 2, 1, 1]) == N.ERR_INVALID_ARG          # bad role value
+    assert call_layer(lib, s, [1, 0, 1, 1], idx_in=None) == N.ERR_INVALID_ARG  # sparse needs sets
+    assert call_layer(lib, s, [1, 1, 1, 1], q=None) == N.ERR_INVALID_ARG
+    assert call_layer(lib, s, [1, 1, 1, 1], q=FAKE + 4) == N.ERR_INVALID_ARG   # misaligned
+    assert call_layer(lib, s, [1, 1, 1, 1], ws_bytes=100) == N.ERR_WORKSPACE
+    assert call_layer(lib, s, [1, 1, 1, 1], ws=None) == N.ERR_WORKSPACE
+    assert call_layer(lib, s, [1, 1, 1, 1], ws=FAKE + 16) == N.ERR_WORKSPACE   # not 256-aligned
+
+
+def call_stack(lib, s, L, roles, kc=None, ws_bytes=1 << 40):
+    r = (ctypes.c_uint8 * len(roles))(*roles)
+    kc = kc if kc is not None else [FAKE] * L
+    kp = (ctypes.c_void_p * L)(*kc)
+    vp = (ctypes.c_void_p * L)(*([FAKE] * L))
+    return lib.lychee_decode_stack(ctypes.byref(s), L, FAKE, ctypes.cast(kp, ctypes.c_void_p),
+                                   ctypes.cast(vp, ctypes.c_void_p), FAKE, None,
+                                   ctypes.cast(r, ctypes.c_void_p), FAKE, FAKE, None, FAKE,
+                                   ctypes.c_size_t(ws_bytes), None)
+
+
+def test_stack_rejects_bad_arguments_on_host(lib):
+    s = shape()
+    # step (1): layer 0 must be all retrieval
+    assert call_stack(lib, s, 2, [1, 1, 0, 1] + [0, 0, 0, 0]) == N.ERR_INVALID_ARG
+    assert call_stack(lib, s, 0, []) == N.ERR_INVALID_ARG
+    assert call_stack(lib, s, 2, [1] * 4 + [0, 3, 0, 0]) == N.ERR_INVALID_ARG
+    assert call_stack(lib, s, 2, [1] * 4 + [0] * 4, kc=[FAKE, 0]) == N.ERR_INVALID_ARG
+    assert call_stack(lib, s, 2, [1] * 4 + [0] * 4, ws_bytes=256) == N.ERR_WORKSPACE
+
+
+def test_status_strings(lib):
+    for st in range(7):
+        assert lib.lychee_status_string(st)
+    assert b"unknown" in lib.lychee_status_string(99)
+
+
+def test_binding_refuses_cpu_tensors(lib):
+    q = torch.zeros(1, 4, 128, dtype=torch.bfloat16)
+    kv = torch.zeros(1, 2, 64, 128, dtype=torch.bfloat16)
+    sl = torch.tensor([64], dtype=torch.int32)
+    with pytest.raises(ValueError, match="CUDA"):
+        ops.hybrid_decode_attn(q, kv, kv, sl, [1, 1, 1, 1], None, 8)
+
+
+def test_missing_library_fails_loudly(tmp_path):
+    with pytest.raises(RuntimeError, match="not found"):
+        N.load(str(tmp_path / "liblychee.so"))
