@@ -29,7 +29,7 @@ struct WsHeader {
 };
 static_assert(sizeof(WsHeader) == 256, "header is 256 bytes");
 
-constexpr int kChunk = 1024;          // positions per attention work item
+constexpr int kChunk = 960;           // positions per attention work item (30 words)
 constexpr int kMaxHq = 128;           // query heads supported
 constexpr uint64_t kWaitLimitNs = 2000000000ull;   // 2 s: a wait this long is a fault
 
@@ -70,14 +70,17 @@ __device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
                : "memory");
 }
 
-__device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
+// One bounded wait: the thread may be suspended until the phase completes or
+// about `hint_ns` elapse (a hint to the hardware), so waiting warps do not spin.
+__device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity,
+                                              uint32_t hint_ns = 1000000u) {
   uint32_t ok;
   asm volatile(
       "{\n\t.reg .pred p;\n\t"
-      "mbarrier.try_wait.parity.acquire.cta.shared::cta.b64 p, [%1], %2;\n\t"
+      "mbarrier.try_wait.parity.acquire.cta.shared::cta.b64 p, [%1], %2, %3;\n\t"
       "selp.u32 %0, 1, 0, p;\n\t}"
       : "=r"(ok)
-      : "r"(smem_u32(bar)), "r"(parity)
+      : "r"(smem_u32(bar)), "r"(parity), "r"(hint_ns)
       : "memory");
   return ok != 0;
 }
@@ -87,14 +90,38 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, uint32_t* err) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = globaltimer();
-  uint32_t spins = 0;
   while (!mbar_try_wait(bar, parity)) {
-    if ((++spins & 255u) == 0u && globaltimer() - t0 > kWaitLimitNs) {
+    if (globaltimer() - t0 > kWaitLimitNs) {
       flag_error(err, kErrTimeout);
       return false;
     }
   }
   return true;
+}
+
+// ---- 16-byte asynchronous copies global -> shared (cp.async, L2 only) -------
+// The plain three-operand form: a fourth operand would be read as the source
+// size of a zero-filling copy.
+__device__ __forceinline__ void cp_async16(void* dst, const void* src) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(dst)), "l"(src)
+               : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() {
+  asm volatile("cp.async.commit_group;" ::: "memory");
+}
+template <int N>
+__device__ __forceinline__ void cp_async_wait() {
+  asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
+}
+// The mbarrier's pending count is raised by one now and lowered again when all
+// of this thread's earlier cp.async copies have landed.
+__device__ __forceinline__ void cp_async_mbar_arrive(uint64_t* bar) {
+  asm volatile("cp.async.mbarrier.arrive.shared::cta.b64 [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+// Orders this thread's earlier generic-proxy shared-memory accesses before its
+// later async-proxy (TMA) accesses.
+__device__ __forceinline__ void fence_proxy_async_smem() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
 
 // ---- 1-D bulk copy global -> shared (TMA, no tensor map, no multicast) ------
@@ -149,8 +176,8 @@ __device__ __forceinline__ uint32_t dsmem_ld_u32(uint32_t addr) {
 }
 
 // ---- numeric helpers --------------------------------------------------------------
-// 2^x on the special-function unit (PTX ex2.approx; max relative error about
-// 2^-22 over the range used here).
+// 2^x on the special-function unit (PTX ex2.approx.ftz; its error is orders of
+// magnitude below the output tolerances; inputs here are <= 0).
 __device__ __forceinline__ float fast_exp2(float x) {
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
