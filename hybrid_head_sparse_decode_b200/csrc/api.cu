@@ -156,6 +156,7 @@ lychee_status run_layer(const Ctx& c, const void* q, const void* kc, const void*
   if (build_bits && ns > 0) {
     BuildBitsParams bp{};
     bp.idx_in = idx_in;
+    bp.idx_out = idx_out;
     bp.seqlens = seqlens;
     bp.k_per_seq = k_per_seq;
     bp.bitmaps = bitmaps;
@@ -173,8 +174,10 @@ lychee_status run_layer(const Ctx& c, const void* q, const void* kc, const void*
   ap.logits = logits;
   ap.part_ml = part_ml;
   ap.part_acc = part_acc;
+  ap.k_per_seq = k_per_seq;
   ap.err = err;
   ap.counter = counter;
+  ap.exits = &c.hdr()->counters[1];
   ap.B = s->B; ap.Hq = Hq; ap.Hkv = s->Hkv; ap.N_max = s->N_max;
   ap.nwords = c.L.nwords; ap.nchunk = c.L.nchunk;
   ap.n_items = s->B * s->Hkv * c.L.nchunk;
@@ -200,15 +203,9 @@ lychee_status run_layer(const Ctx& c, const void* q, const void* kc, const void*
   cp.part_ml = part_ml;
   cp.part_acc = part_acc;
   cp.seqlens = seqlens;
-  cp.k_per_seq = k_per_seq;
   cp.out = out;
-  cp.idx_in = idx_in;
-  cp.idx_out = idx_in ? idx_out : nullptr;
-  cp.err = err;
-  cp.counter = counter;
-  cp.B = s->B; cp.Hq = Hq; cp.N_max = s->N_max; cp.nchunk = c.L.nchunk; cp.k = s->k;
+  cp.B = s->B; cp.Hq = Hq; cp.N_max = s->N_max; cp.nchunk = c.L.nchunk;
   cp.scale_log2 = ap.scale_log2;
-  std::memcpy(cp.role, ap.role, sizeof(cp.role));
   e = timed(kKindCombine, c.st, [&] { return launch_combine(cp, s->dtype, s->d, c.st); });
   if (e != cudaSuccess) return LYCHEE_ERR_CUDA;
   return LYCHEE_OK;
@@ -263,7 +260,7 @@ lychee_status lychee_hybrid_decode_attn(const lychee_shape* s, const void* q,
     return LYCHEE_ERR_WORKSPACE;
   Ctx c{s, L, static_cast<unsigned char*>(workspace), static_cast<cudaStream_t>(stream), 0};
   if ((c.sms = num_sms_current()) <= 0) return LYCHEE_ERR_CUDA;
-  if (cudaMemsetAsync(workspace, 0, sizeof(WsHeader), c.st) != cudaSuccess) return LYCHEE_ERR_CUDA;
+  if (cudaMemsetAsync(workspace, 0, L.logits, c.st) != cudaSuccess) return LYCHEE_ERR_CUDA;
   return run_layer(c, q, k_cache, v_cache, seqlens, k_per_seq, head_role, ns > 0 ? idx_in : nullptr,
                    out, idx_out, /*build_bits=*/true, /*write_bits=*/false);
 }
@@ -291,7 +288,7 @@ lychee_status lychee_decode_stack(const lychee_shape* s, int32_t L, const void* 
     return LYCHEE_ERR_WORKSPACE;
   Ctx c{s, lay, static_cast<unsigned char*>(workspace), static_cast<cudaStream_t>(stream), 0};
   if ((c.sms = num_sms_current()) <= 0) return LYCHEE_ERR_CUDA;
-  if (cudaMemsetAsync(workspace, 0, sizeof(WsHeader), c.st) != cudaSuccess) return LYCHEE_ERR_CUDA;
+  if (cudaMemsetAsync(workspace, 0, lay.logits, c.st) != cudaSuccess) return LYCHEE_ERR_CUDA;
   const size_t layer_elems = (size_t)s->B * s->Hq * s->d;
   const size_t esz = elem_size(s);
   for (int l = 0; l < L; ++l) {

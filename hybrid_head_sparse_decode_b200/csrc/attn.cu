@@ -146,7 +146,8 @@ struct AttnCfg {
   static constexpr int OFF_POS = OFF_INFO + STAGES * 16;
   static constexpr int OFF_MASK = OFF_POS + STAGES * TT * 4;
   static constexpr int OFF_PS = (OFF_MASK + STAGES * TT + 15) / 16 * 16;
-  static constexpr int OFF_MERGE = OFF_PS + NW * RW * G * 8;   // [NW][G][MS] per-warp states
+  // per-warp states at an item's end ([NW][G][MS])
+  static constexpr int OFF_MERGE = OFF_PS + NW * RW * G * 8;
   static constexpr int OFF_ITEM = OFF_MERGE + NW * G * MS * 4;
   static constexpr int OFF_LPOS = OFF_ITEM + 32;
   static constexpr int OFF_LMASK = OFF_LPOS + kChunk * 4;
@@ -178,6 +179,10 @@ __device__ __forceinline__ void decode_item(int item, bool compact, const int* c
     c = cg % nchunk;
   }
 }
+
+template <typename T, int D, int G, int RQ, int NW, int NP, int STAGES>
+__device__ __forceinline__ void consumer_loop(const AttnParams& p, unsigned char* smem,
+                                              uint64_t* full, uint64_t* empty);
 
 template <typename T, int D, int G, int RQ, int NW, int NP, int STAGES>
 __global__ void __launch_bounds__((NW + NP) * 32, 1)
@@ -256,6 +261,13 @@ __global__ void __launch_bounds__((NW + NP) * 32, 1)
         for (int t = 0; t < G; ++t) w[t] = __ldg(&p.bitmaps[wbase + (size_t)t * p.nwords]);
       }
     };
+    if (pw == 0 && blockIdx.x == 0) {
+      for (int bb = lane; bb < B; bb += 32) {
+        const int n_raw = __ldg(&p.seqlens[bb]);
+        if (n_raw < 1 || n_raw > N_max) flag_error(p.err, kErrBadSeqlen);
+        if (p.k_per_seq && __ldg(&p.k_per_seq[bb]) < 1) flag_error(p.err, kErrBadBudget);
+      }
+    }
     int cur = 0, cur_n = 1, claimed = 0;
     uint32_t cur_w[G];
     if (pw == 0) {
@@ -322,18 +334,12 @@ __global__ void __launch_bounds__((NW + NP) * 32, 1)
               lmask[o] = (uint8_t)m;
               ++o;
             }
-            if (total == 0 && lane < G) {
-              // no row of this chunk is used by any head of the group: empty partials
-              float* ml = p.part_ml + ((size_t)(b * Hq + h0 + lane) * p.nchunk + c) * 2;
-              ml[0] = -INFINITY;
-              ml[1] = 0.f;
-            }
           }
           cur = nxt;
           cur_n = nxt_n;
 #pragma unroll
           for (int t = 0; t < G; ++t) cur_w[t] = nxt_w[t];
-          if (total > 0) break;
+          if (p0 < n) break;   // chunks beyond n_b exist only without the compact space
         }
         if (lane == 0) {
           item_desc[0] = total;
@@ -355,7 +361,8 @@ __global__ void __launch_bounds__((NW + NP) * 32, 1)
       const int unit = b * Hkv + g;
       const T* kbase = reinterpret_cast<const T*>(p.k) + (size_t)unit * N_max * D;
       const T* vbase = reinterpret_cast<const T*>(p.v) + (size_t)unit * N_max * D;
-      const int ntile = total < 0 ? 1 : (total + TT - 1) / TT;   // the end is one entry
+      // the end is one entry; a chunk no head of the group uses is one empty tile
+      const int ntile = total <= 0 ? 1 : (total + TT - 1) / TT;
       for (int tt = 0; tt < ntile; ++tt) {
         const int t0 = tt * TT;
         if (!mbar_wait(&empty[s], ph ^ 1u, p.err)) {
@@ -423,10 +430,36 @@ __global__ void __launch_bounds__((NW + NP) * 32, 1)
       if (!ok || total < 0) break;
       named_bar_sync(2, NP * 32);            // every gather of this item was issued
     }
-    return;
+  } else {
+    consumer_loop<T, D, G, RQ, NW, NP, STAGES>(p, smem, full, empty);
   }
+  // ---- the last CTA to leave resets the launch counters for the next launch
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    __threadfence();
+    if (atomicAdd(p.exits, 1u) == gridDim.x - 1) {
+      *p.counter = 0u;
+      *p.exits = 0u;
+      __threadfence();
+    }
+  }
+}
 
-  // -------------------------------------------------------------- consumers
+// Consumer warps of attn_kernel (see the file comment).
+template <typename T, int D, int G, int RQ, int NW, int NP, int STAGES>
+__device__ __forceinline__ void consumer_loop(const AttnParams& p, unsigned char* smem,
+                                              uint64_t* full, uint64_t* empty) {
+  using C = AttnCfg<T, D, G, RQ, NW, NP, STAGES>;
+  constexpr int TPR = C::TPR, E = C::E, CPT = C::CPT, RSL = C::RSL, RW = C::RW, TT = C::TT;
+  constexpr int ROWB = C::ROWB, PVC = C::PVC, RGV = C::RGV, PVR = C::PVR, PVB = C::PVB;
+  constexpr int LPH = C::LPH, MS = C::MS;
+  const int4* info = reinterpret_cast<const int4*>(smem + C::OFF_INFO);
+  const int32_t* mpos = reinterpret_cast<const int32_t*>(smem + C::OFF_POS);
+  const uint8_t* mmask = reinterpret_cast<const uint8_t*>(smem + C::OFF_MASK);
+  float* merge = reinterpret_cast<float*>(smem + C::OFF_MERGE);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int Hq = p.Hq, N_max = p.N_max;
+
   const int r = lane / TPR, pp = lane % TPR;     // q.K: row slot, part
   const int rot = r % CPT;                       // same for every row of the lane
   const int hb = pp / LPH;                       // the head this lane reduces to
@@ -454,7 +487,7 @@ __global__ void __launch_bounds__((NW + NP) * 32, 1)
 
   uint32_t s = 0, ph = 0;
   for (;;) {
-    if (!mbar_wait(&full[s], ph, p.err)) return;
+    if (!mbar_wait(&full[s], ph, p.err)) break;
     const int4 inf = info[s];
     if (inf.w & kTerm) break;
     const int nrows = inf.z & 255, flags = inf.w;

@@ -16,8 +16,10 @@ struct AttnParams {
   float* logits;            // [B, Hq, N_max]: raw q.k of retrieval heads
   float* part_ml;           // [B, Hq, nchunk, 2]: (max raw dot, sum of weights)
   float* part_acc;          // [B, Hq, nchunk, D]: unnormalised weighted values
+  const int32_t* k_per_seq; // [B] or null (validated here)
   uint32_t* err;
-  uint32_t* counter;        // work-item counter, 0 at launch
+  uint32_t* counter;        // work-item counter, 0 at launch, 0 again at exit
+  uint32_t* exits;          // CTAs that finished, 0 at launch, 0 again at exit
   int B, Hq, Hkv, N_max, nwords, nchunk, n_items;
   float scale_log2;         // log2(e) / sqrt(D)
   uint32_t role[4];         // bit h set: head h is a retrieval head
@@ -38,26 +40,22 @@ struct TopkParams {
 };
 cudaError_t launch_topk(const TopkParams& p, cudaStream_t st);
 
-// Merge of split partials, output rounding, set pass-through (combine.cu).
+// Merge of split partials into the attention output (combine.cu).
 struct CombineParams {
-  const float* part_ml;
-  const float* part_acc;
-  const int32_t* seqlens;
-  const int32_t* k_per_seq;  // [B] or null (validated here)
+  const float* part_ml;      // [B, Hq, nchunk, 2]
+  const float* part_acc;     // [B, Hq, nchunk, D]
+  const int32_t* seqlens;    // [B]
   void* out;                 // [B, Hq, D]
-  const int32_t* idx_in;     // [B, Hq, k] or null
-  int32_t* idx_out;          // [B, Hq, k] or null: rows of sparse heads copied from idx_in
-  uint32_t* err;
-  uint32_t* counter;         // reset to 0 for the next attention launch
-  int B, Hq, N_max, nchunk, k;
+  int B, Hq, N_max, nchunk;
   float scale_log2;
-  uint32_t role[4];
 };
 cudaError_t launch_combine(const CombineParams& p, int dtype, int D, cudaStream_t st);
 
-// Incoming index sets -> membership bitmaps, with validation (sets.cu).
+// Incoming index sets -> membership bitmaps, with validation; the rows are also
+// copied to idx_out (sparse heads pass their set on unchanged) (sets.cu).
 struct BuildBitsParams {
   const int32_t* idx_in;     // [B, Hq, k]
+  int32_t* idx_out;          // [B, Hq, k] or null
   const int32_t* seqlens;
   const int32_t* k_per_seq;
   uint32_t* bitmaps;         // [B, Hq, nwords]

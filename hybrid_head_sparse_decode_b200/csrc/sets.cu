@@ -11,28 +11,54 @@ namespace lychee {
 namespace {
 
 constexpr int kThreads = 256;
+constexpr int kEntriesPerCta = 4 * kThreads;   // set entries one build_bits CTA covers
 
-// Index rows of the listed sparse heads -> bitmaps.  An entry outside [0, n_b)
-// or not strictly above its predecessor sets kErrBadIndex and is skipped.
+// Index rows of the listed sparse heads -> bitmaps (and, when asked, a bit-exact
+// copy of the rows: a sparse head hands its set on unchanged).  One thread per
+// entry, loads coalesced along the row.  Every bitmap word has exactly one
+// writer, so the row needs no clearing pass and no atomics: the thread holding
+// the first entry of a word ORs that word's entries (at most 32, contiguous in
+// the ascending row) and also writes the empty words between the previous
+// entry's word and its own; the first and last entries cover the words before
+// and after the set.  An entry outside [0, n_b) or not strictly above its
+// predecessor sets kErrBadIndex; the row is then not a set and its bitmap is
+// unspecified, but every store still stays inside the row.
 __global__ void __launch_bounds__(kThreads) build_bits_kernel(const __grid_constant__ BuildBitsParams p) {
-  const int b = blockIdx.x / p.nheads, h = p.heads[blockIdx.x % p.nheads];
+  const int b = blockIdx.y / p.nheads, h = p.heads[blockIdx.y % p.nheads];
   const int n = min(max(p.seqlens[b], 1), p.N_max);
   int kb = p.k_per_seq ? p.k_per_seq[b] : p.k;
   kb = min(min(max(kb, 1), p.k), n);
   const size_t bh = (size_t)b * p.Hq + h;
   uint32_t* row = p.bitmaps + bh * p.nwords;
   const int words = (n + 31) >> 5;
-  for (int w = threadIdx.x; w < words; w += kThreads) row[w] = 0u;
-  __syncthreads();
   const int32_t* idx = p.idx_in + bh * p.k;
-  for (int t = threadIdx.x; t < kb; t += kThreads) {
+  const int base = blockIdx.x * kEntriesPerCta;
+#pragma unroll
+  for (int r = 0; r < kEntriesPerCta / kThreads; ++r) {
+    const int t = base + r * kThreads + threadIdx.x;
+    if (t >= p.k) break;
     const int j = idx[t];
+    if (p.idx_out) p.idx_out[bh * p.k + t] = j;
+    if (t >= kb) continue;
     const int prev = t > 0 ? idx[t - 1] : -1;
     if (j < 0 || j >= n || j <= prev) {
       flag_error(p.err, kErrBadIndex);
       continue;
     }
-    atomicOr(&row[j >> 5], 1u << (j & 31));
+    const int w = j >> 5;
+    const int pw = prev >> 5;   // -1 for the first entry (arithmetic shift)
+    if (w != pw) {
+      uint32_t bits = 1u << (j & 31);
+      for (int u = t + 1; u < kb; ++u) {
+        const int ju = idx[u];
+        if ((ju >> 5) != w || ju <= j) break;
+        bits |= 1u << (ju & 31);
+      }
+      row[w] = bits;
+      for (int g = max(pw + 1, 0); g < w; ++g) row[g] = 0u;
+    }
+    if (t == kb - 1)
+      for (int g = w + 1; g < words; ++g) row[g] = 0u;
   }
 }
 
@@ -80,7 +106,8 @@ __global__ void __launch_bounds__(kThreads) export_kernel(const __grid_constant_
 
 cudaError_t launch_build_bits(const BuildBitsParams& p, cudaStream_t st) {
   if (p.nheads <= 0) return cudaSuccess;
-  build_bits_kernel<<<(unsigned)(p.B * p.nheads), kThreads, 0, st>>>(p);
+  const dim3 grid((unsigned)((p.k + kEntriesPerCta - 1) / kEntriesPerCta), (unsigned)(p.B * p.nheads));
+  build_bits_kernel<<<grid, kThreads, 0, st>>>(p);
   return cudaGetLastError();
 }
 

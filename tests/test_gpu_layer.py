@@ -111,6 +111,29 @@ def test_deterministic_bitwise():
     assert torch.equal(a[0], b[0]) and torch.equal(a[1], b[1])
 
 
+def test_topk_repeated_on_vector_aligned_rows():
+    """Every retrieval head, rows starting on 16-byte boundaries (N_max a multiple
+    of 4, so the top-k takes its vector-load path), several calls in a row: each
+    call's sets are exactly the top-k of that call's own logits (a race between the
+    threads that stage the keys and those that count them shows up here)."""
+    B, Hq, Hkv, d, N_max = 2, 16, 4, 64, 12288
+    prob = inputs.make_layer(B, Hq, Hkv, d, N_max, roles=[1] * Hq, seed=21,
+                             seqlens=[N_max, 7000], k_fixed=3686)
+    for _ in range(4):
+        _, idx_out, logits, st, _ = run_gpu(prob)
+        assert st == N.OK
+        gi = idx_out.cpu().numpy()
+        lg = logits.cpu().numpy()
+        for b in range(B):
+            n = int(prob.seqlens[b])
+            kb = int(prob.meta["kb"][b])
+            for h in range(Hq):
+                rep = SetReport()
+                check_set(rep, (b, h), gi[b, h], kb, prob.k, lg[b, h, :n].astype(np.float64),
+                          gpu_raw=lg[b, h, :n], d=d)
+                assert not rep.failures, rep.failures
+
+
 def test_bad_index_is_reported_not_trapped():
     prob = inputs.make_layer(1, 4, 2, 128, 500, roles=[1, 0, 1, 0], seed=11, k_fixed=100)
     bad = prob.idx_in.clone()
