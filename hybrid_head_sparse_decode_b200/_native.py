@@ -29,7 +29,11 @@ FP32 = 1
 ROLE_SPARSE = 0
 ROLE_RETRIEVAL = 1
 
-EXPORTED = ("lychee_workspace_size", "lychee_workspace_offsets", "lychee_hybrid_decode_attn", "lychee_decode_stack",
+# LYCHEE_NOALLOC_SCRATCH_BYTES of include/lychee.h
+NOALLOC_SCRATCH_BYTES = 32 << 20
+
+EXPORTED = ("lychee_workspace_size", "lychee_workspace_offsets", "lychee_hybrid_decode_attn",
+            "lychee_hybrid_decode_attn_noalloc", "lychee_decode_stack",
             "lychee_check_device_error", "lychee_status_string", "lychee_version",
             "lychee_profile_begin", "lychee_profile_end")
 
@@ -71,6 +75,8 @@ def load(path: str | None = None):
         lib.lychee_workspace_offsets.restype = ctypes.c_int
         lib.lychee_hybrid_decode_attn.argtypes = [sp] + [vp] * 10 + [ctypes.c_size_t, vp]
         lib.lychee_hybrid_decode_attn.restype = ctypes.c_int
+        lib.lychee_hybrid_decode_attn_noalloc.argtypes = [sp] + [vp] * 11
+        lib.lychee_hybrid_decode_attn_noalloc.restype = ctypes.c_int
         lib.lychee_decode_stack.argtypes = [sp, i32] + [vp] * 10 + [ctypes.c_size_t, vp]
         lib.lychee_decode_stack.restype = ctypes.c_int
         lib.lychee_check_device_error.argtypes = [vp, vp, u32p]

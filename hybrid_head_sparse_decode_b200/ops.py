@@ -109,6 +109,48 @@ def hybrid_decode_attn(q, k_cache, v_cache, seqlens, head_role, idx_in, k, *, k_
     return out, idx_out
 
 
+def hybrid_decode_attn_noalloc(q, k_cache, v_cache, seqlens, head_role, idx_in, k, *,
+                               k_per_seq=None, out=None, idx_out=None, device_error=None,
+                               stream=None):
+    """hybrid_decode_attn served from the library's static device scratch: no
+    workspace argument and no device allocation by the library (out / idx_out
+    are allocated here only when not given).  device_error: optional device
+    int32 tensor [1] that receives the call's device error bits.  Calls on one device
+    share the scratch, so they must not overlap; the first call on a device must
+    precede any stream capture."""
+    B, Hq, d = q.shape
+    _, Hkv, N_max, _ = k_cache.shape
+    _need_cuda("q", q)
+    dt = q.dtype
+    _need_cuda("k_cache", k_cache, dt, (B, Hkv, N_max, d))
+    _need_cuda("v_cache", v_cache, dt, (B, Hkv, N_max, d))
+    _need_cuda("seqlens", seqlens, torch.int32, (B,))
+    if k_per_seq is not None:
+        _need_cuda("k_per_seq", k_per_seq, torch.int32, (B,))
+    if idx_in is not None:
+        _need_cuda("idx_in", idx_in, torch.int32, (B, Hq, k))
+    need = workspace_size(B, Hq, Hkv, d, N_max, k, dt)
+    if need > N.NOALLOC_SCRATCH_BYTES:
+        raise ValueError(f"this layer needs {need} bytes of scratch; the static scratch holds "
+                         f"{N.NOALLOC_SCRATCH_BYTES} (use hybrid_decode_attn with a workspace)")
+    role = _roles_host(head_role, Hq)
+    if out is None:
+        out = torch.empty((B, Hq, d), dtype=dt, device=q.device)
+    _need_cuda("out", out, dt, (B, Hq, d))
+    if idx_out is None:
+        idx_out = torch.empty((B, Hq, k), dtype=torch.int32, device=q.device)
+    _need_cuda("idx_out", idx_out, torch.int32, (B, Hq, k))
+    if device_error is not None:
+        _need_cuda("device_error", device_error, torch.int32, (1,))
+    sh = make_shape(B, Hq, Hkv, d, N_max, k, dt)
+    st = N.load().lychee_hybrid_decode_attn_noalloc(
+        ctypes.byref(sh), _ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(seqlens), _ptr(k_per_seq),
+        ctypes.c_void_p(role.data_ptr()), _ptr(idx_in), _ptr(out), _ptr(idx_out),
+        _ptr(device_error), _stream_handle(stream))
+    _check(st, "lychee_hybrid_decode_attn_noalloc")
+    return out, idx_out
+
+
 def decode_stack(q, k_caches, v_caches, seqlens, head_roles, k, *, k_per_seq=None, out=None,
                  idx_final=None, idx_layers=None, want_layers=False, workspace=None, stream=None):
     """L chained layers of one decode step.  q [L,B,Hq,d]; k_caches / v_caches:

@@ -123,6 +123,36 @@ LYCHEE_API lychee_status lychee_hybrid_decode_attn(const lychee_shape* s, const 
                                         void* out, int32_t* idx_out, void* workspace,
                                         size_t workspace_bytes, void* stream);
 
+/* Size of the static device scratch behind lychee_hybrid_decode_attn_noalloc:
+ * 32 MiB per device, enough for a layer whose lychee_workspace_size() is at
+ * most that (e.g. B = 1, Hq = 32, d = 128, N_max = 131072 needs about 19 MiB). */
+#define LYCHEE_NOALLOC_SCRATCH_BYTES (32u << 20)
+
+/* lychee_hybrid_decode_attn without a caller-owned workspace and without any
+ * device allocation.  The method has no counterpart to this call: it is a
+ * convenience of the library boundary for callers that may not allocate.
+ * Arguments q .. idx_out and stream are those of lychee_hybrid_decode_attn and
+ * the results are the same, bit for bit.  The workspace is a file-scope
+ * __device__ array of LYCHEE_NOALLOC_SCRATCH_BYTES (one per device, part of the
+ * library's device code); the call allocates nothing, and clears the part of the
+ * scratch that must start at zero (error word, work counters) itself.
+ *   device_error device uint32 or NULL: receives, in stream order, the device
+ *                error bits of this call (as lychee_check_device_error's detail)
+ * Returns LYCHEE_ERR_WORKSPACE, before touching the GPU, when
+ * lychee_workspace_size(s) exceeds LYCHEE_NOALLOC_SCRATCH_BYTES; the shape and
+ * argument errors of lychee_hybrid_decode_attn otherwise; LYCHEE_ERR_CUDA if the
+ * scratch address cannot be looked up.
+ * All calls on one device share the scratch: calls whose executions overlap
+ * (other streams, host threads) race on it, so serialise them.  The first call
+ * on each device looks the scratch address up (cudaGetSymbolAddress); make it
+ * before any stream capture. */
+LYCHEE_API lychee_status lychee_hybrid_decode_attn_noalloc(const lychee_shape* s, const void* q,
+                                        const void* k_cache, const void* v_cache,
+                                        const int32_t* seqlens, const int32_t* k_per_seq,
+                                        const uint8_t* head_role, const int32_t* idx_in,
+                                        void* out, int32_t* idx_out, uint32_t* device_error,
+                                        void* stream);
+
 /* L chained layers of one decode step (method steps (1), (3), (4)): the set
  * leaving head position h of layer l is the incoming set of head position h of
  * layer l+1; it is carried between layers as the per-head bitmap in the
