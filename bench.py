@@ -46,6 +46,27 @@ def measured_peak():
         return FALLBACK_HBM_GBS, "fallback"
 
 
+def attn_traffic_per_launch(alg_bytes_per_launch):
+    """DRAM bytes (read + write) of one attention launch: the ncu capture of a
+    small case with the same per-layer shape (profiles/attn_kernel.traffic.json)
+    gives DRAM bytes per algorithmic byte; a full launch's traffic is that ratio
+    times its algorithmic bytes.  None when the kernel sources have changed since
+    the capture (the counters no longer describe this kernel)."""
+    import hashlib
+    try:
+        with open(os.path.join(ROOT, "profiles", "attn_kernel.traffic.json")) as f:
+            prof = json.load(f)
+        h = hashlib.sha256()
+        for src in prof["sources"]:
+            with open(os.path.join(ROOT, src), "rb") as f:
+                h.update(f.read())
+        if h.hexdigest() != prof["source_sha256"]:
+            return None
+        return int(round(prof["traffic_per_algorithmic_byte"] * alg_bytes_per_launch))
+    except (OSError, KeyError, ValueError):
+        return None
+
+
 class ClockSampler:
     """Samples SM clock, max clock, power and throttle reasons through NVML while
     running (reads only; changes no setting)."""
@@ -128,10 +149,12 @@ def make_workload(name, device, seed_offset=0):
     if name == "llama3_ragged_stack":
         return inputs.llama3_ragged_stack(device=device, seed=inputs.BASE_SEED + 3 + seed_offset)
     if name.startswith("qwen3_stack_"):      # qwen3_stack_<N>x<L>, for small profiling cases
-        n, l = name[len("qwen3_stack_"):].split("x")
-        return inputs.make_stack(int(l), 1, 32, 8, 128, int(n), seed=inputs.BASE_SEED + 2,
+        # the 36-layer stack's head mix scaled to L layers: layer 0 all retrieval,
+        # 32 retrieval heads spread over the other 35 layers (about one per layer)
+        n, l = (int(x) for x in name[len("qwen3_stack_"):].split("x"))
+        return inputs.make_stack(l, 1, 32, 8, 128, n, seed=inputs.BASE_SEED + 2 + seed_offset,
                                  device=device, k_frac=0.3, n_planted=64,
-                                 n_extra_retrieval=min(32, (int(l) - 1) * 32))
+                                 n_extra_retrieval=max(1, round(32 * (l - 1) / 35)) if l > 1 else 0)
     raise SystemExit(f"unknown workload {name}")
 
 
@@ -335,7 +358,9 @@ def run_lychee(args, rank, world, device):
         "bytes_per_step": {"union": sum(union_bytes), "literal": sum(literal_bytes),
                            "dense": sum(dense_bytes)},
         "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak,
-                     "unit": "GB/s", "frac": round(achieved / peak, 4), "traffic": None,
+                     "unit": "GB/s", "frac": round(achieved / peak, 4),
+                     "traffic": attn_traffic_per_launch(attn_bytes_per_step / L),
+                     "algorithmic_bytes_per_launch": int(attn_bytes_per_step / L),
                      "kernel": "attn_kernel (hybrid attention, all layers)",
                      "peak_source": peak_kind, "frac_of_nominal_8tbs": round(achieved / NOMINAL_HBM_GBS, 4),
                      "bytes_rule": "union rows x 512 B per launch"},
