@@ -46,6 +46,22 @@ def measured_peak():
         return FALLBACK_HBM_GBS, "fallback"
 
 
+def max_over_ranks(x, world, device):
+    """The largest of the ranks' values (every rank passes its own and gets the
+    maximum back); the value itself when there is one rank."""
+    if world <= 1:
+        return float(x)
+    t = torch.tensor([float(x)], device=device, dtype=torch.float64)
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_us_per_step(ms_per_step_slowest, world):
+    """µs per decode step of the whole job: the N replicas each complete one step
+    within the slowest rank's step time."""
+    return ms_per_step_slowest * 1e3 / world
+
+
 def attn_traffic_per_launch(alg_bytes_per_launch):
     """DRAM bytes (read + write) of one attention launch: the ncu capture of a
     small case with the same per-layer shape (profiles/attn_kernel.traffic.json)
@@ -272,10 +288,7 @@ def run_lychee(args, rank, world, device):
         for _ in range(args.steps):
             step()
         torch.cuda.synchronize()
-    if world > 1:
-        t = torch.tensor([ms_total], device=device, dtype=torch.float64)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        ms_total = float(t.item())
+    ms_total = max_over_ranks(ms_total, world, device)
     ms_step = ms_total / args.steps
     recs = prof.records
     attn = [ms for k, ms in recs if k == "attn"]
@@ -338,14 +351,11 @@ def run_lychee(args, rank, world, device):
     torch.cuda.synchronize()
     barrier()
     e_ms = e0.elapsed_time(e1)
-    if world > 1:
-        t = torch.tensor([e_ms], device=device, dtype=torch.float64)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        e_ms = float(t.item())
+    e_ms = max_over_ranks(e_ms, world, device)
     h2d = (q_h.numel() * q_h.element_size() + sl_h.numel() * 4 + kb_h.numel() * 4)
     d2h = out_h.numel() * out_h.element_size() + fin_h.numel() * 4
 
-    us_step_job = ms_step * 1e3 / world
+    us_step_job = job_us_per_step(ms_step, world)
     result = {
         "metric": METRIC, "value": round(us_step_job, 3), "unit": UNIT, "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_step, 5),
@@ -368,7 +378,7 @@ def run_lychee(args, rank, world, device):
         "dense_comparator": {"ms_per_step": round(dense_ms, 4),
                              "hbm_gbs": round(sum(dense_bytes) / (dense_ms * 1e-3) / 1e9, 1),
                              "speedup_hybrid_vs_dense": round(dense_ms / ms_step, 3)},
-        "e2e": {"value": round(e_ms * 1e3 / args.steps / world, 3), "unit": UNIT,
+        "e2e": {"value": round(job_us_per_step(e_ms / args.steps, world), 3), "unit": UNIT,
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
         "gpu_launches": sum(v[0] for v in kinds.values()),
         "clocks": sampler.summary(),

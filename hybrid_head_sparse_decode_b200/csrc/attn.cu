@@ -15,11 +15,13 @@
 // head masks the rows that are not its own.
 //
 // CTA layout (persistent, one CTA per SM, items taken from an atomic counter):
-//   * producer warp: claims the next item and loads its bitmap words while the
-//     current item streams; builds the row list; for each tile of TT rows waits
-//     for a free ring stage and issues 1-D bulk copies (cp.async.bulk, no tensor
-//     map, no multicast) of the K rows and V rows into shared memory, one copy
-//     per run of consecutive positions;
+//   * NP producer warps: the lead warp claims the next item and loads its
+//     bitmap words while the current item streams, and builds the row list;
+//     for each tile of TT rows the producers wait for a free ring stage, then a
+//     dense tile (consecutive positions) arrives as two 1-D bulk copies
+//     (cp.async.bulk, no tensor map, no multicast) of its K rows and V rows,
+//     while a sparse tile is gathered row by row with 16-byte cp.async by all
+//     producer warps (whole 32-byte sectors, each union row read once);
 //   * NW consumer warps: each owns RW rows of every tile.  q.K: TPR lanes per row,
 //     q held in registers (fp32), K widened from bf16 in registers, packed
 //     fp32x2 FMA; a reduce-scatter leaves each lane with whole dot products of

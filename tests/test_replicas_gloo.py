@@ -1,0 +1,71 @@
+"""The multi-process (replica) plumbing of bench.py on CPU: two ranks over gloo.
+
+The decode step has no exchange between GPUs, so N GPUs run N independent
+replicas; what crosses ranks is only the timing (the slowest rank's time is the
+job's).  These tests run that host logic with world size 2 on the gloo backend."""
+import argparse
+import os
+import socket
+import sys
+
+import pytest
+import torch
+import torch.distributed as dist
+import torch.multiprocessing as mp
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _free_port():
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def _rank_main(rank, world, port, out_path):
+    sys.path.insert(0, ROOT)
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    import datetime
+    dist.init_process_group("gloo", rank=rank, world_size=world,
+                            timeout=datetime.timedelta(seconds=60))
+    try:
+        import bench
+        cpu = torch.device("cpu")
+        # each rank brings its own time; all get the slowest
+        slowest = bench.max_over_ranks(1.5 + rank, world, cpu)
+        job = bench.job_us_per_step(slowest, world)
+        # replicas draw different inputs (seeded by rank)
+        prob = bench.make_workload("qwen3_stack_64x2", cpu, seed_offset=rank)
+        qsum = float(prob.q.float().sum())
+        sums = [None] * world
+        dist.all_gather_object(sums, qsum)
+        # the reference arm runs on rank 0 only; other ranks return at once
+        args = argparse.Namespace(workload="qwen3_stack_64x2", steps=1, warmup=0)
+        ref = bench.run_reference(args, rank, world) if rank != 0 else None
+        with open(f"{out_path}.{rank}", "w") as f:
+            f.write(repr((slowest, job, sums, ref)))
+        dist.barrier()
+    finally:
+        dist.destroy_process_group()
+
+
+def test_two_gloo_ranks_take_the_slowest_time_and_distinct_inputs(tmp_path):
+    world = 2
+    out = str(tmp_path / "res")
+    mp.start_processes(_rank_main, args=(world, _free_port(), out), nprocs=world,
+                       start_method="spawn", join=True)
+    res = [eval(open(f"{out}.{r}").read()) for r in range(world)]
+    for slowest, job, sums, ref in res:
+        assert slowest == 2.5                       # max over ranks
+        assert job == pytest.approx(2.5e3 / world)  # µs per decode step of the job
+        assert sums[0] != sums[1]                   # each replica has its own inputs
+        assert ref is None
+    assert res[0][2] == res[1][2]
+
+
+def test_single_rank_needs_no_process_group():
+    sys.path.insert(0, ROOT)
+    import bench
+    assert bench.max_over_ranks(3.25, 1, torch.device("cpu")) == 3.25
+    assert bench.job_us_per_step(3.25, 1) == pytest.approx(3250.0)
