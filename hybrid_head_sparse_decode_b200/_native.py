@@ -30,7 +30,7 @@ ROLE_SPARSE = 0
 ROLE_RETRIEVAL = 1
 
 # LYCHEE_NOALLOC_SCRATCH_BYTES of include/lychee.h
-NOALLOC_SCRATCH_BYTES = 32 << 20
+NOALLOC_SCRATCH_BYTES = 64 << 20
 
 EXPORTED = ("lychee_workspace_size", "lychee_workspace_offsets", "lychee_hybrid_decode_attn",
             "lychee_hybrid_decode_attn_noalloc", "lychee_decode_stack",

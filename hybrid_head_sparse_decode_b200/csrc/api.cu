@@ -1,6 +1,8 @@
 // api.cu -- the C ABI of libychee (declared in include/lychee.h): argument
 // validation, workspace layout and the launch sequence of one layer and of an
 // L-layer decode step.  Host code only; no memory is allocated here.
+#include <cudaTypedefs.h>
+
 #include <cmath>
 #include <cstdint>
 #include <cstring>
@@ -18,7 +20,7 @@ namespace {
 constexpr int kVersion = 100;   // 0.1.0
 
 struct Layout {
-  size_t logits, part_ml, part_acc, bitmaps, total;
+  size_t logits, part_ml, part_acc, part_n, part2, ccnt, bitmaps, total;
   int nchunk, nwords;
 };
 
@@ -51,9 +53,15 @@ Layout layout_of(const lychee_shape* s) {
   L.logits = off;
   off += align256(bh * s->N_max * 4);
   L.part_ml = off;
-  off += align256(bh * L.nchunk * 2 * 4);
+  off += align256(bh * L.nchunk * kPartSlots * 2 * 4);
   L.part_acc = off;
-  off += align256(bh * L.nchunk * s->d * 4);
+  off += align256(bh * L.nchunk * kPartSlots * s->d * 4);
+  L.part_n = off;
+  off += align256(bh * L.nchunk * 4);
+  L.part2 = off;
+  off += align256(bh * kCombineSplit * (s->d + 4) * 4);
+  L.ccnt = off;
+  off += align256(bh * 4);
   L.bitmaps = off;
   off += align256(bh * L.nwords * 4);
   L.total = off;
@@ -90,6 +98,44 @@ int num_sms_current() {
     cache[dev] = n;
   }
   return cache[dev];
+}
+
+// ---- tensor maps for the attention kernel's row gathers -----------------------------
+// cuTensorMapEncodeTiled comes from the driver through the runtime's entry-point
+// query, so the library needs no link against libcuda.
+PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
+  static std::once_flag once;
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  std::call_once(once, [] {
+    void* f = nullptr;
+    cudaDriverEntryPointQueryResult q{};
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(f);
+    cudaGetLastError();
+  });
+  return fn;
+}
+
+// The cache [B, Hkv, N_max, d] as rows of d elements, box one row high and one
+// row wide (the form tile::gather4 needs).  False when it cannot be described
+// (no encoder, or more rows than a 32-bit coordinate reaches); the kernel then
+// gathers with 16-byte copies instead.
+bool encode_row_map(CUtensorMap* m, const void* base, const lychee_shape* s) {
+  PFN_cuTensorMapEncodeTiled_v12000 enc = tensor_map_encoder();
+  const unsigned long long rows = (unsigned long long)s->B * s->Hkv * s->N_max;
+  if (!enc || rows > 0x7fffffffull) return false;
+  const size_t es = s->dtype == LYCHEE_BF16 ? 2 : 4;
+  const cuuint64_t dims[2] = {(cuuint64_t)s->d, (cuuint64_t)rows};
+  const cuuint64_t strides[1] = {(cuuint64_t)s->d * es};
+  const cuuint32_t box[2] = {(cuuint32_t)s->d, 1u};
+  const cuuint32_t estr[2] = {1u, 1u};
+  const CUtensorMapDataType dt =
+      s->dtype == LYCHEE_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32;
+  return enc(m, dt, 2, const_cast<void*>(base), dims, strides, box, estr,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
 // ---- optional launch profiler ----------------------------------------------------
@@ -145,6 +191,9 @@ lychee_status run_layer(const Ctx& c, const void* q, const void* kc, const void*
   float* logits = reinterpret_cast<float*>(c.ws + c.L.logits);
   float* part_ml = reinterpret_cast<float*>(c.ws + c.L.part_ml);
   float* part_acc = reinterpret_cast<float*>(c.ws + c.L.part_acc);
+  int32_t* part_n = reinterpret_cast<int32_t*>(c.ws + c.L.part_n);
+  float* part2 = reinterpret_cast<float*>(c.ws + c.L.part2);
+  uint32_t* ccnt = reinterpret_cast<uint32_t*>(c.ws + c.L.ccnt);
   uint32_t* bitmaps = reinterpret_cast<uint32_t*>(c.ws + c.L.bitmaps);
   uint8_t rheads[kMaxHq], sheads[kMaxHq];
   int nr = 0, ns = 0;
@@ -174,6 +223,8 @@ lychee_status run_layer(const Ctx& c, const void* q, const void* kc, const void*
   ap.logits = logits;
   ap.part_ml = part_ml;
   ap.part_acc = part_acc;
+  ap.part_n = part_n;
+  ap.ccnt = ccnt;
   ap.k_per_seq = k_per_seq;
   ap.err = err;
   ap.counter = counter;
@@ -183,6 +234,7 @@ lychee_status run_layer(const Ctx& c, const void* q, const void* kc, const void*
   ap.n_items = s->B * s->Hkv * c.L.nchunk;
   ap.scale_log2 = (float)(1.4426950408889634 / std::sqrt((double)s->d));
   fill_roles(ap.role, role, Hq);
+  ap.gather_tma = (encode_row_map(&ap.tmk, kc, s) && encode_row_map(&ap.tmv, vc, s)) ? 1 : 0;
   e = timed(kKindAttn, c.st, [&] { return launch_attn(ap, s->dtype, s->d, G, c.sms, c.st); });
   if (e != cudaSuccess) return LYCHEE_ERR_CUDA;
   if (nr > 0) {
@@ -202,6 +254,9 @@ lychee_status run_layer(const Ctx& c, const void* q, const void* kc, const void*
   CombineParams cp{};
   cp.part_ml = part_ml;
   cp.part_acc = part_acc;
+  cp.part_n = part_n;
+  cp.part2 = part2;
+  cp.ccnt = ccnt;
   cp.seqlens = seqlens;
   cp.out = out;
   cp.B = s->B; cp.Hq = Hq; cp.N_max = s->N_max; cp.nchunk = c.L.nchunk;

@@ -11,27 +11,37 @@
 // the item needs the rows  R = {j in chunk : some head of the group uses j}:
 // every row when the group holds a retrieval head ("dense" group), otherwise
 // the union of the heads' sets (read from their membership bitmaps).  Each row
-// of R is read from HBM once and serves all G heads (GQA deduplication); each
-// head masks the rows that are not its own.
+// of R is read from HBM once into shared memory and serves every head of the
+// group that uses it (GQA deduplication).
 //
 // CTA layout (persistent, one CTA per SM, items taken from an atomic counter):
-//   * NP producer warps: the lead warp claims the next item and loads its
-//     bitmap words while the current item streams, and builds the row list;
-//     for each tile of TT rows the producers wait for a free ring stage, then a
-//     dense tile (consecutive positions) arrives as two 1-D bulk copies
-//     (cp.async.bulk, no tensor map, no multicast) of its K rows and V rows,
-//     while a sparse tile is gathered row by row with 16-byte cp.async by all
-//     producer warps (whole 32-byte sectors, each union row read once);
-//   * NW consumer warps: each owns RW rows of every tile.  q.K: TPR lanes per row,
-//     q held in registers (fp32), K widened from bf16 in registers, packed
-//     fp32x2 FMA; a reduce-scatter leaves each lane with whole dot products of
-//     its heads.  The online-softmax state (running max, running sum,
-//     accumulator) is kept per warp, so tiles need no CTA-wide barrier, and the
-//     accumulator is rescaled only when a running max grows.  P.V: four
-//     elements of a V row per lane, probabilities read as pre-duplicated fp32
-//     pairs.  At the end of an item the warps' states are merged once and one
-//     partial (m, l, acc[d]) per head is written for the combine kernel.
-// Tensor cores are not used: per KV row a group does at most 4 * 2d FMAs
+//   * a builder warp claims items and turns each into its row list R, each
+//     sparse head's list of the rows of R it uses (with per-tile offsets), and
+//     a share of the consumer warps for every head proportional to its rows.
+//     It fills two alternating item buffers, so the next item is built while
+//     the current one streams and is consumed.
+//   * streaming warps move each built item through a ring of shared-memory
+//     stages in tiles of TT rows of R.  A dense tile (consecutive positions)
+//     arrives as two 1-D bulk copies (cp.async.bulk) of its K rows and V rows,
+//     issued by the first streaming warp; a sparse tile is gathered row by row
+//     over two paths at once: part of its rows as TMA tile::gather4 copies
+//     (four rows each, through a tensor map over the cache rows) issued by the
+//     first streaming warp, the rest as 16-byte cp.async by the other streaming
+//     warps (whole 32-byte sectors either way).  No copy uses multicast.
+//   * NW consumer warps: during an item each warp serves one head and only
+//     that head's rows (pairs (row, head)), so a sparse head costs work in
+//     proportion to its own set, not to the group's union.  Four lanes share a
+//     pair, each holding a quarter of q (fp32 registers) and of the output
+//     accumulator; eight pairs are in flight per warp.  q.K: K widened from
+//     bf16 in registers, packed fp32x2 FMA, two shuffles to finish the dot
+//     product.  Online softmax per pair slot with a lazy maximum: the running
+//     maximum moves only when a score exceeds it by 2^8 in probability, so the
+//     accumulator is rarely rescaled.  P.V on the same lanes and rows.  At the
+//     end of an item a warp merges its eight slots with shuffles and writes one
+//     partial state (m, l, acc[d]) to its own slot of the workspace; the
+//     combine kernel merges the warps and chunks in a fixed order, so the
+//     result does not depend on scheduling and no warp waits for another.
+// Tensor cores are not used: per K/V row a group does at most 4 * 2d FMAs
 // against 2d * sizeof(T) bytes -- a batched GEMV that HBM, not math, bounds.
 //
 // Logits of retrieval heads (raw q.k in fp32, not divided by sqrt(d)) are
@@ -48,6 +58,18 @@ namespace {
 constexpr uint32_t kFull = 0xffffffffu;
 constexpr int kFirst = 1, kLast = 2, kTerm = 4, kDense = 8;
 constexpr int kMaxBatchCompact = 1024;  // sequences whose chunk counts are kept in smem
+constexpr int kLanesPerPair = 4;        // lanes sharing one (row, head) pair
+constexpr int kPairsPerBatch = 32 / kLanesPerPair;
+constexpr float kLazyLog2 = 8.f;        // rescale when a probability would exceed 2^8
+constexpr uint8_t kNoHead = 0xff;
+
+// Sparse tiles take two copy paths at once: the first LYCHEE_ATTN_TMA_ROWS/16 of
+// a tile's rows as TMA tile::gather4 copies issued by the first streaming warp,
+// the rest as 16-byte cp.async by the other streaming warps (each path alone
+// caps below HBM bandwidth).  0: cp.async only.
+#ifndef LYCHEE_ATTN_TMA_ROWS
+#define LYCHEE_ATTN_TMA_ROWS 8
+#endif
 
 template <typename T>
 struct Vec;
@@ -61,12 +83,6 @@ struct Vec<__nv_bfloat16> {
     o[2] = bf16x2_to_float2(w.z);
     o[3] = bf16x2_to_float2(w.w);
   }
-  // four consecutive elements
-  __device__ __forceinline__ static void load4(const void* p, float2 (&o)[2]) {
-    const uint2 w = *reinterpret_cast<const uint2*>(p);
-    o[0] = bf16x2_to_float2(w.x);
-    o[1] = bf16x2_to_float2(w.y);
-  }
 };
 template <>
 struct Vec<float> {
@@ -76,93 +92,59 @@ struct Vec<float> {
     o[0] = make_float2(w.x, w.y);
     o[1] = make_float2(w.z, w.w);
   }
-  __device__ __forceinline__ static void load4(const void* p, float2 (&o)[2]) {
-    const float4 w = *reinterpret_cast<const float4*>(p);
-    o[0] = make_float2(w.x, w.y);
-    o[1] = make_float2(w.z, w.w);
-  }
 };
 
-// Reduce-scatter of per-lane partial dot products over the TPR lanes of a row.
-// cur[0..NCUR) holds one partial per head; each halving level keeps half of the
-// heads (upper half when the lane bit M is set) and adds the partner's copy of
-// them; once one head is left the remaining levels are plain butterflies.
-template <int NCUR, int M>
-struct ReduceScatter {
-  __device__ __forceinline__ static void run(float* cur, int pp) {
-    if constexpr (M >= 1) {
-      if constexpr (NCUR > 1) {
-        constexpr int HALF = NCUR / 2;
-        const bool upper = (pp & M) != 0;
-        float keep[HALF];
-#pragma unroll
-        for (int i = 0; i < HALF; ++i) {
-          const float mine = upper ? cur[HALF + i] : cur[i];
-          const float send = upper ? cur[i] : cur[HALF + i];
-          keep[i] = mine + __shfl_xor_sync(kFull, send, M);
-        }
-#pragma unroll
-        for (int i = 0; i < HALF; ++i) cur[i] = keep[i];
-        ReduceScatter<HALF, M / 2>::run(cur, pp);
-      } else {
-        cur[0] += __shfl_xor_sync(kFull, cur[0], M);
-        ReduceScatter<1, M / 2>::run(cur, pp);
-      }
-    }
-  }
-};
-
-template <typename T, int D, int G, int RQ, int NW, int NP, int STAGES>
+template <typename T, int D, int G, int NW, int NP, int TT, int STAGES>
 struct AttnCfg {
-  static constexpr int TPR = 8;                   // q.K lanes per row
-  static constexpr int E = Vec<T>::E;             // elements per 16-byte q.K chunk
-  static constexpr int CPR = D / E;               // q.K chunks per row
-  static constexpr int CPT = CPR / TPR;           // q.K chunks per lane
-  static constexpr int RSL = 32 / TPR;            // q.K row slots per warp
-  static constexpr int RW = RSL * RQ;             // rows per warp per tile
-  static constexpr int TT = NW * RW;              // rows per tile
+  static constexpr int E = Vec<T>::E;             // elements per 16-byte chunk
+  static constexpr int DL = D / kLanesPerPair;    // dimensions per lane
+  static constexpr int CPL = DL / E;              // 16-byte chunks per lane
   static constexpr int ROWB = D * (int)sizeof(T); // bytes per K (or V) row
-  static constexpr int PVC = D / 4;               // P.V lanes per row (4 elements each)
-  static constexpr int RGV = 32 / PVC;            // rows a warp covers at once in P.V
-  static constexpr int PVR = RW / RGV;            // rows per P.V lane per tile
-  static constexpr int PVB = 4 * (int)sizeof(T);  // bytes of V per P.V lane and row
-  static constexpr int LPH = TPR / G;             // q.K lanes per head
   static constexpr int PPR = ROWB / 16;           // 16-byte pieces per row (gathers)
   static constexpr int RPI = PPR >= 32 ? 1 : 32 / PPR;  // rows per gather instruction
   static constexpr int NT = (NW + NP) * 32;
-  static constexpr int MS = D + 4;                // merge row: acc[D], l, m, pad (16-B rows)
-  static_assert(CPR % TPR == 0 && CPT >= 1 && (4 % CPT == 0), "q.K mapping");
-  static_assert(G <= TPR && TPR % G == 0, "one head per q.K lane");
-  static_assert(PVC <= 32 && RW % RGV == 0, "P.V mapping");
-  static_assert(TT <= 255, "row count is packed in 8 bits");
-  static_assert(kChunk % 32 == 0 && kChunk <= 1024, "producer builds one word per lane");
+  static constexpr int NS = NP - 1;               // streaming warps (all producers but the builder)
+  static constexpr int MAXT = (kChunk + TT - 1) / TT;   // tiles per item at most
+  static_assert(CPL >= 2 && DL % E == 0 && CPL % 2 == 0, "lane mapping");
+  static_assert(TT % kPairsPerBatch == 0 && TT % 4 == 0 && TT <= 255, "tile rows");
+  static_assert(G <= NW && NW <= kPartSlots && NW < 16, "warps per head fit the partial slots");
+  static_assert(NP >= 2, "a builder and at least one streaming warp");
+  static_assert(kChunk % 32 == 0 && kChunk <= 1024, "builder holds one word per lane");
+  static_assert(MAXT < 32, "one lane per tile start");
 
-  // shared memory layout (byte offsets)
+  // item buffer (two of them): descriptor, warp assignment, the chunk's union
+  // bitmap words, each head's bitmap words, the union index of each word's
+  // first row, the gather positions
+  static constexpr int NWD = kChunk / 32;         // bitmap words per chunk
+  static constexpr int ASGB = NW + G;             // warp -> (head, slot), warps per head
+  static constexpr int IB_ASG = 32;
+  static constexpr int IB_UW = IB_ASG + (ASGB + 15) / 16 * 16;          // [32] u32
+  static constexpr int IB_HW = IB_UW + 32 * 4;                           // [G][32] u32
+  static constexpr int IB_UB = IB_HW + G * 32 * 4;                       // [32] i32
+  static constexpr int IB_LPOS = IB_UB + 32 * 4;                         // [kChunk] i32
+  static constexpr int IBUF = IB_LPOS + kChunk * 4;
+
+  // shared memory layout (byte offsets from a 128-byte aligned base)
   static constexpr int kStageKV = TT * ROWB;
   static constexpr int kQBytes = G * D * (int)sizeof(T);
   static constexpr int QSTRIDE = (kQBytes + 127) / 128 * 128;
   static constexpr int OFF_K = 0;
   static constexpr int OFF_V = OFF_K + STAGES * kStageKV;
   static constexpr int OFF_Q = OFF_V + STAGES * kStageKV;
-  static constexpr int OFF_INFO = OFF_Q + STAGES * QSTRIDE;
-  static constexpr int OFF_POS = OFF_INFO + STAGES * 16;
-  static constexpr int OFF_MASK = OFF_POS + STAGES * TT * 4;
-  static constexpr int OFF_PS = (OFF_MASK + STAGES * TT + 15) / 16 * 16;
-  // per-warp states at an item's end ([NW][G][MS])
-  static constexpr int OFF_MERGE = OFF_PS + NW * RW * G * 8;
-  static constexpr int OFF_ITEM = OFF_MERGE + NW * G * MS * 4;
-  static constexpr int OFF_LPOS = OFF_ITEM + 32;
-  static constexpr int OFF_LMASK = OFF_LPOS + kChunk * 4;
-  static constexpr int OFF_CUM = (OFF_LMASK + kChunk + 15) / 16 * 16;
+  static constexpr int OFF_INFO = OFF_Q + STAGES * QSTRIDE;             // [STAGES][2] int4
+  static constexpr int OFF_ITEM = OFF_INFO + STAGES * 32;               // [2][IBUF]
+  static constexpr int OFF_HL = OFF_ITEM + 2 * IBUF;                    // [NW][kChunk] u16
+  static constexpr int OFF_CUM = OFF_HL + NW * kChunk * 2;
   static constexpr int OFF_BAR = (OFF_CUM + (kMaxBatchCompact + 1) * 4 + 15) / 16 * 16;
-  static constexpr int SMEM = OFF_BAR + 2 * STAGES * 8;
+  static constexpr int NBAR = 2 * STAGES + 4;     // full, empty, ready[2], freeb[2]
+  static constexpr int SMEM = OFF_BAR + NBAR * 8 + 128;   // + alignment slack
 };
 
-// Item decode shared by the producer: item -> (b, c, g).  With a compact item
+// Item decode shared by the builder: item -> (b, c, g).  With a compact item
 // space (B <= kMaxBatchCompact) items enumerate only chunks below n_b, chunk
 // major over the concatenated sequences, KV group fastest; cum[b] holds the
 // number of chunks of sequences before b.  Otherwise every (b, c < nchunk, g)
-// is an item and chunks beyond n_b are skipped by the producer.
+// is an item and chunks beyond n_b are skipped.
 __device__ __forceinline__ void decode_item(int item, bool compact, const int* cum, int B,
                                             int Hkv, int nchunk, int& b, int& c, int& g) {
   g = item % Hkv;
@@ -182,39 +164,95 @@ __device__ __forceinline__ void decode_item(int item, bool compact, const int* c
   }
 }
 
-template <typename T, int D, int G, int RQ, int NW, int NP, int STAGES>
-__device__ __forceinline__ void consumer_loop(const AttnParams& p, unsigned char* smem,
-                                              uint64_t* full, uint64_t* empty);
+// Consumer warps for the G heads of an item, in proportion to each head's rows:
+// every head with rows gets one warp, then each further warp goes to the head
+// with the most rows per warp (lowest head on ties).  Warps are numbered head
+// by head: asg[w] = head | slot << 4 (kNoHead when the item has no rows at all),
+// nh[h] = warps of head h.  Run by one thread.
+template <int G, int NW>
+__device__ __forceinline__ void assign_warps(const int (&work)[G], uint8_t* asg, uint8_t* nhs) {
+  int nh[G];
+  int used = 0;
+#pragma unroll
+  for (int t = 0; t < G; ++t) {
+    nh[t] = work[t] > 0 ? 1 : 0;
+    used += nh[t];
+  }
+  if (used > 0) {
+    for (; used < NW; ++used) {
+      int best = -1, bw = 0, bn = 1;
+#pragma unroll
+      for (int t = 0; t < G; ++t) {
+        if (nh[t] > 0 && (best < 0 || (long long)work[t] * bn > (long long)bw * nh[t])) {
+          best = t;
+          bw = work[t];
+          bn = nh[t];
+        }
+      }
+#pragma unroll
+      for (int t = 0; t < G; ++t) nh[t] += (t == best) ? 1 : 0;
+    }
+  }
+  int w = 0;
+#pragma unroll
+  for (int t = 0; t < G; ++t) {
+    nhs[t] = (uint8_t)nh[t];
+    for (int j = 0; j < nh[t]; ++j) asg[w++] = (uint8_t)(t | (j << 4));
+  }
+  for (; w < NW; ++w) asg[w] = kNoHead;
+}
 
-template <typename T, int D, int G, int RQ, int NW, int NP, int STAGES>
+// Merge of two online-softmax states (m: running max of raw dots, l: sum of
+// weights) into the first; returns the weights of the two accumulators.
+struct MergeW {
+  float a, b;
+};
+__device__ __forceinline__ MergeW merge_weights(float& m, float& l, float m2, float l2, float sl) {
+  const float M = fmaxf(m, m2);
+  MergeW w;
+  w.a = (m == -INFINITY) ? 0.f : fast_exp2((m - M) * sl);
+  w.b = (m2 == -INFINITY) ? 0.f : fast_exp2((m2 - M) * sl);
+  l = l * w.a + l2 * w.b;
+  m = M;
+  return w;
+}
+
+template <typename T, int D, int G, int NW, int NP, int TT, int STAGES>
+__device__ __forceinline__ void consumer_loop(const AttnParams& p, unsigned char* smem,
+                                              uint64_t* full, uint64_t* empty, uint64_t* freeb);
+
+template <typename T, int D, int G, int NW, int NP, int TT, int STAGES>
 __global__ void __launch_bounds__((NW + NP) * 32, 1)
     attn_kernel(const __grid_constant__ AttnParams p) {
-  using C = AttnCfg<T, D, G, RQ, NW, NP, STAGES>;
-  constexpr int TPR = C::TPR, E = C::E, CPT = C::CPT, RSL = C::RSL, RW = C::RW, TT = C::TT;
-  constexpr int ROWB = C::ROWB, PVC = C::PVC, RGV = C::RGV, PVR = C::PVR, PVB = C::PVB;
-  constexpr int LPH = C::LPH, PPR = C::PPR, RPI = C::RPI, MS = C::MS;
+  using C = AttnCfg<T, D, G, NW, NP, TT, STAGES>;
+  constexpr int ROWB = C::ROWB, PPR = C::PPR, RPI = C::RPI, E = C::E, NS = C::NS;
 
-  extern __shared__ __align__(128) unsigned char smem[];
+  extern __shared__ __align__(128) unsigned char smem_raw[];
+  unsigned char* smem = smem_raw + ((128u - (smem_u32(smem_raw) & 127u)) & 127u);
   int4* info = reinterpret_cast<int4*>(smem + C::OFF_INFO);
-  int32_t* mpos = reinterpret_cast<int32_t*>(smem + C::OFF_POS);
-  uint8_t* mmask = reinterpret_cast<uint8_t*>(smem + C::OFF_MASK);
-  float* merge = reinterpret_cast<float*>(smem + C::OFF_MERGE);
-  int* item_desc = reinterpret_cast<int*>(smem + C::OFF_ITEM);
-  int32_t* lpos = reinterpret_cast<int32_t*>(smem + C::OFF_LPOS);
-  uint8_t* lmask = reinterpret_cast<uint8_t*>(smem + C::OFF_LMASK);
   int* cum = reinterpret_cast<int*>(smem + C::OFF_CUM);
-  // per stage: full (row list, q and K/V rows landed; one arrival per producer
-  // warp), empty (every consumer warp is done with the stage)
+  // per stage: full (q and K/V rows landed; one arrival per streaming warp),
+  // empty (every consumer warp is done with the stage); per item buffer: ready
+  // (built), freeb (streamed and consumed: every streaming and consumer warp)
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + C::OFF_BAR);
   uint64_t* empty = full + STAGES;
+  uint64_t* ready = empty + STAGES;
+  uint64_t* freeb = ready + 2;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int Hq = p.Hq, Hkv = p.Hkv, N_max = p.N_max, B = p.B;
   const bool compact = B <= kMaxBatchCompact;
+  // the combine kernel that follows counts its finished CTAs from zero
+  for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < B * Hq; i += gridDim.x * blockDim.x)
+    p.ccnt[i] = 0u;
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
-      mbar_init(&full[s], NP);
+      mbar_init(&full[s], NS);
       mbar_init(&empty[s], NW);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&ready[i], 1);
+      mbar_init(&freeb[i], NS + NW);
     }
     fence_mbar_init();
   }
@@ -238,15 +276,10 @@ __global__ void __launch_bounds__((NW + NP) * 32, 1)
   }
   __syncthreads();
 
-  if (warp >= NW) {
-    // ------------------------------------------------------- producer group
-    const int pw = warp - NW;              // 0 leads: claims, row lists, TMA
+  if (warp == NW + 1) {
+    // ------------------------------------------------------------ builder
     const int n_items = compact ? cum[B] * Hkv : p.n_items;
-    const uint64_t pol = l2_evict_first_policy();
-    uint32_t s = 0, ph = 0;                // ring stage and its phase parity
-    bool ok = true;
-
-    // lead only: claim an item (lane 0) and load what building its row list needs
+    // claim an item (lane 0) and load what building its row list needs
     auto claim = [&]() -> int { return lane == 0 ? (int)atomicAdd(p.counter, 1u) : 0; };
     auto prefetch = [&](int item, int& nraw, uint32_t (&w)[G]) {
       nraw = 1;
@@ -263,106 +296,135 @@ __global__ void __launch_bounds__((NW + NP) * 32, 1)
         for (int t = 0; t < G; ++t) w[t] = __ldg(&p.bitmaps[wbase + (size_t)t * p.nwords]);
       }
     };
-    if (pw == 0 && blockIdx.x == 0) {
+    if (blockIdx.x == 0) {
       for (int bb = lane; bb < B; bb += 32) {
         const int n_raw = __ldg(&p.seqlens[bb]);
         if (n_raw < 1 || n_raw > N_max) flag_error(p.err, kErrBadSeqlen);
         if (p.k_per_seq && __ldg(&p.k_per_seq[bb]) < 1) flag_error(p.err, kErrBadBudget);
       }
     }
-    int cur = 0, cur_n = 1, claimed = 0;
+    int cur = __shfl_sync(kFull, claim(), 0), cur_n = 1;
     uint32_t cur_w[G];
-    if (pw == 0) {
-      cur = __shfl_sync(kFull, claim(), 0);
-      prefetch(cur, cur_n, cur_w);
-      claimed = claim();
-    }
-
-    for (;;) {
-      // -- the lead builds the next item's row list; the group then streams it
+    prefetch(cur, cur_n, cur_w);
+    int claimed = claim();
+    for (uint32_t it = 0;; ++it) {
+      const int buf = it & 1;
+      if (!mbar_wait(&freeb[buf], ((it >> 1) & 1u) ^ 1u, p.err)) break;
+      unsigned char* ib = smem + C::OFF_ITEM + buf * C::IBUF;
+      int* desc = reinterpret_cast<int*>(ib);
+      uint8_t* asg = ib + C::IB_ASG;
+      int32_t* lpos = reinterpret_cast<int32_t*>(ib + C::IB_LPOS);
       int total = 0, b = 0, c = 0, g = 0, p0 = 0;
-      bool dense = false;
-      if (pw == 0) {
-        int nxt_n = 1, nxt = 0;
+      uint32_t rmask = 0;
+      for (;;) {   // skip chunks beyond n_b (only without the compact space)
+        if (cur >= n_items) {
+          total = -1;
+          break;
+        }
+        decode_item(cur, compact, cum, B, Hkv, p.nchunk, b, c, g);
+        const int n = min(max(cur_n, 1), N_max);
+        p0 = c * kChunk;
+        const int h0 = g * G;
+        // claim and load the item after this one while this one is built
+        int nxt_n = 1;
         uint32_t nxt_w[G];
-        for (;;) {   // skip items without rows
-          if (cur >= n_items) {
-            total = -1;
-            break;
+        const int nxt = __shfl_sync(kFull, claimed, 0);
+        prefetch(nxt, nxt_n, nxt_w);
+        claimed = claim();
+        if (p0 < n) {
+          const int p1 = min(p0 + kChunk, n);
+          rmask = 0;
+#pragma unroll
+          for (int t = 0; t < G; ++t) rmask |= ((p.role[(h0 + t) >> 5] >> ((h0 + t) & 31)) & 1u) << t;
+          const int nwords = (p1 - p0 + 31) >> 5;
+          const int nbits = lane < nwords ? min(32, p1 - p0 - 32 * lane) : 0;
+          const uint32_t valid = nbits >= 32 ? kFull : ((1u << nbits) - 1u);
+          uint32_t bits[G];
+          uint32_t uni = 0;
+#pragma unroll
+          for (int t = 0; t < G; ++t) {
+            bits[t] = ((rmask >> t) & 1u) ? valid : (cur_w[t] & valid);
+            uni |= bits[t];
           }
-          decode_item(cur, compact, cum, B, Hkv, p.nchunk, b, c, g);
-          const int n = min(max(cur_n, 1), N_max);
-          p0 = c * kChunk;
-          const int h0 = g * G;
-          // claim and load the item after this one while this one streams
-          nxt = __shfl_sync(kFull, claimed, 0);
-          prefetch(nxt, nxt_n, nxt_w);
-          claimed = claim();
-          if (p0 < n) {
-            const int p1 = min(p0 + kChunk, n);
-            uint32_t rmask = 0;
+          const int cnt = __popc(uni);
+          int incl = cnt;
 #pragma unroll
-            for (int t = 0; t < G; ++t)
-              rmask |= ((p.role[(h0 + t) >> 5] >> ((h0 + t) & 31)) & 1u) << t;
-            dense = rmask != 0;
-            const int nwords = (p1 - p0 + 31) >> 5;
-            uint32_t bits[G];
-            uint32_t uni = 0;
-            const int nb = lane < nwords ? min(32, p1 - p0 - 32 * lane) : 0;
-            const uint32_t valid = nb >= 32 ? kFull : ((1u << nb) - 1u);
-#pragma unroll
-            for (int t = 0; t < G; ++t) {
-              bits[t] = ((rmask >> t) & 1u) ? valid : (cur_w[t] & valid);
-              uni |= bits[t];
-            }
-            if (dense) uni = valid;
-            const int cnt = __popc(uni);
-            int incl = cnt;
-#pragma unroll
-            for (int o = 1; o < 32; o <<= 1) {
-              const int y = __shfl_up_sync(kFull, incl, o);
-              if (lane >= o) incl += y;
-            }
-            total = __shfl_sync(kFull, incl, 31);
-            int o = incl - cnt;
+          for (int o = 1; o < 32; o <<= 1) {
+            const int y = __shfl_up_sync(kFull, incl, o);
+            if (lane >= o) incl += y;
+          }
+          total = __shfl_sync(kFull, incl, 31);
+          const int ubase = incl - cnt;      // union index of this word's first row
+          if (rmask == 0) {
+            // sparse item: positions of the union rows, in order
+            int o = ubase;
             uint32_t u = uni;
             while (u) {
               const int j = __ffs(u) - 1;
               u &= u - 1;
-              uint32_t m = 0;
-#pragma unroll
-              for (int t = 0; t < G; ++t) m |= ((bits[t] >> j) & 1u) << t;
-              lpos[o] = p0 + 32 * lane + j;
-              lmask[o] = (uint8_t)m;
-              ++o;
+              lpos[o++] = p0 + 32 * lane + j;
             }
           }
-          cur = nxt;
-          cur_n = nxt_n;
+          // the words the consumer warps build their heads' row lists from
+          uint32_t* uw = reinterpret_cast<uint32_t*>(ib + C::IB_UW);
+          uint32_t* hw = reinterpret_cast<uint32_t*>(ib + C::IB_HW);
+          int32_t* ub = reinterpret_cast<int32_t*>(ib + C::IB_UB);
+          uw[lane] = uni;
+          ub[lane] = ubase;
+          int work[G];
 #pragma unroll
-          for (int t = 0; t < G; ++t) cur_w[t] = nxt_w[t];
-          if (p0 < n) break;   // chunks beyond n_b exist only without the compact space
+          for (int t = 0; t < G; ++t) {
+            hw[t * 32 + lane] = bits[t];
+            int ct = __popc(bits[t]);
+#pragma unroll
+            for (int o = 16; o >= 1; o >>= 1) ct += __shfl_xor_sync(kFull, ct, o);
+            work[t] = ct;
+          }
+          if (lane == 0) assign_warps<G, NW>(work, asg, asg + NW);
+          __syncwarp();
+          // partial states each head's warps will write for this chunk
+          if (lane < G)
+            p.part_n[(size_t)(b * Hq + h0 + lane) * p.nchunk + c] = (int)asg[NW + lane];
         }
-        if (lane == 0) {
-          item_desc[0] = total;
-          item_desc[1] = b;
-          item_desc[2] = c;
-          item_desc[3] = g;
-          item_desc[4] = p0;
-          item_desc[5] = dense ? 1 : 0;
-        }
+        cur = nxt;
+        cur_n = nxt_n;
+#pragma unroll
+        for (int t = 0; t < G; ++t) cur_w[t] = nxt_w[t];
+        if (p0 < n) break;
       }
-      named_bar_sync(2, NP * 32);            // row list and descriptor ready
-      total = item_desc[0];
-      b = item_desc[1];
-      c = item_desc[2];
-      g = item_desc[3];
-      p0 = item_desc[4];
-      dense = item_desc[5] != 0;
+      if (lane == 0) {
+        desc[0] = total;
+        desc[1] = b;
+        desc[2] = c;
+        desc[3] = g;
+        desc[4] = p0;
+        desc[5] = (int)rmask;
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&ready[buf]);
+      if (total < 0) break;
+    }
+  } else if (warp >= NW) {
+    // ------------------------------------------------------ streaming warps
+    const int sw = warp == NW ? 0 : warp - NW - 1;   // 0: publishes tiles, bulk copies
+    const uint64_t pol = l2_evict_first_policy();
+    const bool tma_rows = LYCHEE_ATTN_TMA_ROWS > 0 && NS > 1 && p.gather_tma != 0;
+    uint32_t s = 0, ph = 0;                // ring stage and its phase parity
+    bool ok = true;
+    for (uint32_t it = 0;; ++it) {
+      const int buf = it & 1;
+      if (!mbar_wait(&ready[buf], (it >> 1) & 1u, p.err)) break;
+      const unsigned char* ib = smem + C::OFF_ITEM + buf * C::IBUF;
+      const int* desc = reinterpret_cast<const int*>(ib);
+      const int32_t* lpos = reinterpret_cast<const int32_t*>(ib + C::IB_LPOS);
+      const int total = desc[0], b = desc[1], c = desc[2], g = desc[3], p0 = desc[4];
+      const uint32_t rmask = (uint32_t)desc[5];
+      const bool dense = rmask != 0;
       const int h0 = g * G;
       const int unit = b * Hkv + g;
       const T* kbase = reinterpret_cast<const T*>(p.k) + (size_t)unit * N_max * D;
       const T* vbase = reinterpret_cast<const T*>(p.v) + (size_t)unit * N_max * D;
+      const int row0 = unit * N_max;        // this group's first row in the tensor maps
       // the end is one entry; a chunk no head of the group uses is one empty tile
       const int ntile = total <= 0 ? 1 : (total + TT - 1) / TT;
       for (int tt = 0; tt < ntile; ++tt) {
@@ -375,26 +437,31 @@ __global__ void __launch_bounds__((NW + NP) * 32, 1)
         const int flags = total < 0 ? kTerm
                                     : ((t0 == 0 ? kFirst : 0) | (t0 + TT >= total ? kLast : 0) |
                                        (dense ? kDense : 0));
-        T* kd = reinterpret_cast<T*>(smem + C::OFF_K + s * C::kStageKV);
-        T* vd = reinterpret_cast<T*>(smem + C::OFF_V + s * C::kStageKV);
-        if (pw == 0) {
-          if (lane == 0) info[s] = make_int4(b, h0, (c << 8) | nrows, flags);
-          for (int i = lane; i < nrows; i += 32) {
-            mpos[s * TT + i] = lpos[t0 + i];
-            mmask[s * TT + i] = lmask[t0 + i];
-          }
+        unsigned char* kd = smem + C::OFF_K + s * C::kStageKV;
+        unsigned char* vd = smem + C::OFF_V + s * C::kStageKV;
+        const bool gather = !(flags & (kDense | kTerm));
+        if (sw == 0 && lane == 0) {
+          info[2 * s] = make_int4(b, h0, c, nrows);
+          info[2 * s + 1] = make_int4(flags, (int)rmask, t0, buf | (tt << 8));
         }
-        if (!(flags & (kDense | kTerm))) {
-          // gather the listed rows with 16-byte copies, split over the group;
-          // each lane's copies are tracked by the stage's full barrier
-          for (int r0 = pw * RPI; r0 < nrows; r0 += NP * RPI) {
+        // rows [0, nt) by TMA (whole groups of four, the last one padded only
+        // when it ends the tile), rows [nt, nrows) by 16-byte copies
+        const int nt = !gather || !tma_rows
+                           ? 0
+                           : (nrows <= 4 ? nrows : ((nrows * LYCHEE_ATTN_TMA_ROWS) >> 4) & ~3);
+        const int ngrp = (nt + 3) >> 2;
+        const int csw = tma_rows ? sw - 1 : sw, ncs = tma_rows ? NS - 1 : NS;
+        if (gather && csw >= 0) {
+          // 16-byte copies shared by the copying warps, each lane's copies
+          // tracked by the stage's full barrier
+          for (int r0 = nt + csw * RPI; r0 < nrows; r0 += ncs * RPI) {
 #pragma unroll
             for (int pc2 = 0; pc2 < (PPR + 31) / 32; ++pc2) {
               const int row = r0 + (PPR >= 32 ? 0 : lane / PPR);
               const int piece = PPR >= 32 ? pc2 * 32 + lane : lane % PPR;
               if (row < nrows && piece < PPR) {
                 const size_t src = (size_t)lpos[t0 + row] * D + piece * E;
-                const int dst = row * D + piece * E;
+                const int dst = row * ROWB + piece * 16;
                 cp_async16(kd + dst, kbase + src);
                 cp_async16(vd + dst, vbase + src);
               }
@@ -403,25 +470,36 @@ __global__ void __launch_bounds__((NW + NP) * 32, 1)
           cp_async_mbar_arrive(&full[s]);
         }
         __syncwarp();
-        if (lane == 0) {
-          if (pw == 0) {
-            const uint32_t bytes = ((flags & kDense) ? 2u * (uint32_t)nrows * ROWB : 0u) +
-                                   ((flags & kFirst) ? (uint32_t)C::kQBytes : 0u);
-            fence_proxy_async_smem();
-            if (bytes) mbar_arrive_expect_tx(&full[s], bytes);
-            else mbar_arrive(&full[s]);
-            if (flags & kFirst) {
-              T* qd = reinterpret_cast<T*>(smem + C::OFF_Q + s * C::QSTRIDE);
-              bulk_g2s(qd, reinterpret_cast<const T*>(p.q) + (size_t)(b * Hq + h0) * D,
-                       (uint32_t)C::kQBytes, &full[s], pol);
-            }
-            if (flags & kDense) {
-              const size_t off = (size_t)(p0 + t0) * D;
-              bulk_g2s(kd, kbase + off, (uint32_t)nrows * ROWB, &full[s], pol);
-              bulk_g2s(vd, vbase + off, (uint32_t)nrows * ROWB, &full[s], pol);
-            }
-          } else {
-            mbar_arrive(&full[s]);
+        if (lane == 0 && sw != 0) mbar_arrive(&full[s]);
+        if (lane == 0 && sw == 0) {
+          const uint32_t bytes = ((flags & kDense) ? 2u * (uint32_t)nrows * ROWB : 0u) +
+                                 ((flags & kFirst) ? (uint32_t)C::kQBytes : 0u) +
+                                 2u * (uint32_t)ngrp * 4u * ROWB;
+          fence_proxy_async_smem();
+          if (bytes) mbar_arrive_expect_tx(&full[s], bytes);
+          else mbar_arrive(&full[s]);
+          if (flags & kFirst) {
+            T* qd = reinterpret_cast<T*>(smem + C::OFF_Q + s * C::QSTRIDE);
+            bulk_g2s(qd, reinterpret_cast<const T*>(p.q) + (size_t)(b * Hq + h0) * D,
+                     (uint32_t)C::kQBytes, &full[s], pol);
+          }
+          if (flags & kDense) {
+            const size_t off = (size_t)(p0 + t0) * D;
+            bulk_g2s(kd, kbase + off, (uint32_t)nrows * ROWB, &full[s], pol);
+            bulk_g2s(vd, vbase + off, (uint32_t)nrows * ROWB, &full[s], pol);
+          }
+        }
+        if (ngrp > 0 && sw == 0) {
+          // four rows per copy; a padded group repeats the range's last row
+          const int last = lpos[t0 + nt - 1];
+          for (int gi = lane; gi < ngrp; gi += 32) {
+            const int4 q4 = *reinterpret_cast<const int4*>(lpos + t0 + 4 * gi);
+            const int y0 = row0 + q4.x;
+            const int y1 = row0 + (4 * gi + 1 < nt ? q4.y : last);
+            const int y2 = row0 + (4 * gi + 2 < nt ? q4.z : last);
+            const int y3 = row0 + (4 * gi + 3 < nt ? q4.w : last);
+            tma_gather4(kd + gi * 4 * ROWB, &p.tmk, 0, y0, y1, y2, y3, &full[s], pol);
+            tma_gather4(vd + gi * 4 * ROWB, &p.tmv, 0, y0, y1, y2, y3, &full[s], pol);
           }
         }
         if (++s == STAGES) {
@@ -430,10 +508,11 @@ __global__ void __launch_bounds__((NW + NP) * 32, 1)
         }
       }
       if (!ok || total < 0) break;
-      named_bar_sync(2, NP * 32);            // every gather of this item was issued
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&freeb[buf]);   // done reading this item's positions
     }
-  } else {
-    consumer_loop<T, D, G, RQ, NW, NP, STAGES>(p, smem, full, empty);
+  } else if (warp < NW) {
+    consumer_loop<T, D, G, NW, NP, TT, STAGES>(p, smem, full, empty, freeb);
   }
   // ---- the last CTA to leave resets the launch counters for the next launch
   __syncthreads();
@@ -448,178 +527,177 @@ __global__ void __launch_bounds__((NW + NP) * 32, 1)
 }
 
 // Consumer warps of attn_kernel (see the file comment).
-template <typename T, int D, int G, int RQ, int NW, int NP, int STAGES>
+template <typename T, int D, int G, int NW, int NP, int TT, int STAGES>
 __device__ __forceinline__ void consumer_loop(const AttnParams& p, unsigned char* smem,
-                                              uint64_t* full, uint64_t* empty) {
-  using C = AttnCfg<T, D, G, RQ, NW, NP, STAGES>;
-  constexpr int TPR = C::TPR, E = C::E, CPT = C::CPT, RSL = C::RSL, RW = C::RW, TT = C::TT;
-  constexpr int ROWB = C::ROWB, PVC = C::PVC, RGV = C::RGV, PVR = C::PVR, PVB = C::PVB;
-  constexpr int LPH = C::LPH, MS = C::MS;
+                                              uint64_t* full, uint64_t* empty, uint64_t* freeb) {
+  using C = AttnCfg<T, D, G, NW, NP, TT, STAGES>;
+  constexpr int E = C::E, DL = C::DL, CPL = C::CPL, ROWB = C::ROWB;
   const int4* info = reinterpret_cast<const int4*>(smem + C::OFF_INFO);
-  const int32_t* mpos = reinterpret_cast<const int32_t*>(smem + C::OFF_POS);
-  const uint8_t* mmask = reinterpret_cast<const uint8_t*>(smem + C::OFF_MASK);
-  float* merge = reinterpret_cast<float*>(smem + C::OFF_MERGE);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int Hq = p.Hq, N_max = p.N_max;
-
-  const int r = lane / TPR, pp = lane % TPR;     // q.K: row slot, part
-  const int rot = r % CPT;                       // same for every row of the lane
-  const int hb = pp / LPH;                       // the head this lane reduces to
-  const bool writer = (pp % LPH) == 0;           // one lane per (row, head) writes
-  const int pc = lane % PVC, rg = lane / PVC;    // P.V: 4-element chunk, row group
+  const int r = lane / kLanesPerPair, pp = lane % kLanesPerPair;   // pair slot, quarter
+  // Chunk order rotated per lane: a 16-byte shared load is served per group of
+  // 8 consecutive lanes (slots r, r+1 with r even, all four quarters), which
+  // must touch 8 different 16-byte bank slots of a 128-byte line.  The rotation
+  // depends on r only through r & 1 (slots r, r^2, r^4 share it), and slot r^1
+  // is rotated by exactly CPL/2 chunks against slot r.
+  const int rot = CPL == 2 ? (r & 1)
+                : CPL == 4 ? ((pp >> 1) + 2 * (r & 1)) % 4
+                           : (pp + 4 * (r & 1)) % CPL;
   const float sl = p.scale_log2;
+  const float lazy = kLazyLog2 / sl;      // raw-dot growth that moves the maximum
 
-  // lane-constant shared-memory byte offsets (stage 0)
-  int koff[CPT];
+  int coff[CPL];                           // byte offsets of the lane's chunks in a row
 #pragma unroll
-  for (int cc = 0; cc < CPT; ++cc)
-    koff[cc] = C::OFF_K + (warp * RW + r) * ROWB + (pp + TPR * ((cc + rot) % CPT)) * 16;
-  const int voff = C::OFF_V + (warp * RW + rg) * ROWB + pc * PVB;
-  const int pw_off = C::OFF_PS + ((warp * RW + r) * G + hb) * 8;   // p writes (slot r)
-  const int pr_off = C::OFF_PS + (warp * RW + rg) * G * 8;         // p reads (row rg)
-  const int row0 = warp * RW + r;                                  // first q.K row
+  for (int cc = 0; cc < CPL; ++cc) coff[cc] = pp * DL * (int)sizeof(T) + ((cc + rot) % CPL) * 16;
 
-  float2 qr[G][CPT][E / 2];
-  float m_run[G];
-  float m_own = -INFINITY, msl = 0.f, l_own = 0.f;
-  float2 acc[G][2];
-  float* lg = nullptr;        // logits row of the lane's head (retrieval heads only)
-  bool lg_on = false;
+  float2 qr[CPL][E / 2];
+  float2 acc[CPL][E / 2];
+  float m = -INFINITY, mth = -INFINITY, msl = 0.f, l = 0.f;
+  int myh = -1, slot = 0, nh = 1, buf = 0;
+  int tstart = 0;                          // lane t: start of tile t in the head's row list
+  uint16_t* hl = reinterpret_cast<uint16_t*>(smem + C::OFF_HL) + warp * kChunk;
+  bool ident = false, lg_on = false;
+  float* lg = nullptr;
   int b = 0, h0 = 0, c = 0;
 
   uint32_t s = 0, ph = 0;
   for (;;) {
     if (!mbar_wait(&full[s], ph, p.err)) break;
-    const int4 inf = info[s];
-    if (inf.w & kTerm) break;
-    const int nrows = inf.z & 255, flags = inf.w;
-    const int kst = s * C::kStageKV;           // stage offset in the K and V rings
+    const int4 i0 = info[2 * s], i1 = info[2 * s + 1];
+    const int flags = i1.x;
+    if (flags & kTerm) break;
+    const int nrows = i0.w, t0 = i1.z, tt = i1.w >> 8;
+    const unsigned char* ib = smem + C::OFF_ITEM + (i1.w & 1) * C::IBUF;
 
     if (flags & kFirst) {
-      b = inf.x;
-      h0 = inf.y;
-      c = inf.z >> 8;
-      const int hq = h0 + hb;
-      lg_on = writer && ((p.role[hq >> 5] >> (hq & 31)) & 1u);
-      lg = p.logits + (size_t)(b * Hq + hq) * N_max;
-      const T* qs = reinterpret_cast<const T*>(smem + C::OFF_Q + s * C::QSTRIDE);
+      b = i0.x;
+      h0 = i0.y;
+      c = i0.z;
+      buf = i1.w & 1;
+      const uint8_t a = ib[C::IB_ASG + warp];
+      myh = a == kNoHead ? -1 : (a & 15);
+      slot = a >> 4;
+      if (myh >= 0) {
+        nh = ib[C::IB_ASG + NW + myh];
+        ident = (i1.y >> myh) & 1;
+        lg_on = ident && pp == 0;
+        lg = p.logits + (size_t)(b * p.Hq + h0 + myh) * p.N_max + (size_t)c * kChunk;
+        const unsigned char* qs = smem + C::OFF_Q + s * C::QSTRIDE + myh * ROWB;
 #pragma unroll
-      for (int h = 0; h < G; ++h)
+        for (int cc = 0; cc < CPL; ++cc) {
+          Vec<T>::load16(qs + coff[cc], qr[cc]);
 #pragma unroll
-        for (int cc = 0; cc < CPT; ++cc) {
-          const int j = pp + TPR * ((cc + rot) % CPT);
-          Vec<T>::load16(qs + h * D + j * E, qr[h][cc]);
+          for (int e = 0; e < E / 2; ++e) acc[cc][e] = make_float2(0.f, 0.f);
         }
+        if (!ident) {
+          // the head's rows as union indices of the item, in order, and where
+          // each tile starts in that list
+          const uint32_t bt = reinterpret_cast<const uint32_t*>(ib + C::IB_HW)[myh * 32 + lane];
+          const uint32_t uu = reinterpret_cast<const uint32_t*>(ib + C::IB_UW)[lane];
+          const int base = reinterpret_cast<const int32_t*>(ib + C::IB_UB)[lane];
+          const int ct = __popc(bt);
+          int ic = ct;
 #pragma unroll
-      for (int h = 0; h < G; ++h) {
-        m_run[h] = -INFINITY;
-        acc[h][0] = acc[h][1] = make_float2(0.f, 0.f);
+          for (int o = 1; o < 32; o <<= 1) {
+            const int y = __shfl_up_sync(kFull, ic, o);
+            if (lane >= o) ic += y;
+          }
+          const int nh_rows = __shfl_sync(kFull, ic, 31);
+          int kk = ic - ct;
+          uint32_t u = bt;
+          while (u) {
+            const int j = __ffs(u) - 1;
+            u &= u - 1;
+            hl[kk++] = (uint16_t)(base + __popc(uu & ((1u << j) - 1u)));
+          }
+          __syncwarp();
+          const int bound = lane * TT;
+          int lo = 0, hi = nh_rows;
+          while (lo < hi) {
+            const int mid = (lo + hi) >> 1;
+            if ((int)hl[mid] < bound) lo = mid + 1;
+            else hi = mid;
+          }
+          tstart = lo;
+        }
       }
-      m_own = -INFINITY;
+      m = -INFINITY;
+      mth = -INFINITY;
       msl = 0.f;
-      l_own = 0.f;
+      l = 0.f;
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&freeb[buf]);   // done reading this item's buffer
     }
 
-    // one tile; WHOLE: every row of the tile exists (no per-row tests)
-    auto tile = [&](auto whole_tag) {
-      constexpr bool WHOLE = decltype(whole_tag)::value;
-      // ---- q.K for the lane's RQ rows
-      float sv[RQ];
-      const int mrow = s * TT + row0;
+    if (myh >= 0) {
+      // this tile's rows of the warp's head: all of them for a retrieval head,
+      // else a slice of the head's row list (union indices of the item)
+      int cnt = nrows, st0 = 0;
+      if (!ident) {
+        st0 = __shfl_sync(kFull, tstart, tt);
+        cnt = __shfl_sync(kFull, tstart, tt + 1) - st0;
+      }
+      const int nb = (cnt + kPairsPerBatch - 1) / kPairsPerBatch;
+      const unsigned char* kt = smem + C::OFF_K + s * C::kStageKV;
+      const unsigned char* vt = smem + C::OFF_V + s * C::kStageKV;
+      // batch k is served by slot (k + tt) % nh: the first batch of a tile
+      // moves from slot to slot so that no warp of the head always gets the most
+      int k = slot - tt % nh;
+      if (k < 0) k += nh;
+      for (; k < nb; k += nh) {
+        const int idx = k * kPairsPerBatch + r;
+        const bool valid = idx < cnt;
+        const int row = valid ? (ident ? idx : (int)hl[st0 + idx] - t0) : 0;
+        // ---- q.K over the lane's quarter: CPL independent partial sums
+        const unsigned char* kr = kt + row * ROWB;
+        float2 part[CPL];
 #pragma unroll
-      for (int i = 0; i < RQ; ++i) {
-        const bool rv = WHOLE || (row0 + RSL * i) < nrows;
-        float2 a2[G];
+        for (int cc = 0; cc < CPL; ++cc) {
+          float2 kx[E / 2];
+          Vec<T>::load16(kr + coff[cc], kx);
+          part[cc] = __fmul2_rn(qr[cc][0], kx[0]);
 #pragma unroll
-        for (int h = 0; h < G; ++h) a2[h] = make_float2(0.f, 0.f);
-        if (rv) {
-#pragma unroll
-          for (int cc = 0; cc < CPT; ++cc) {
-            float2 k2[E / 2];
-            Vec<T>::load16(smem + kst + koff[cc] + i * RSL * ROWB, k2);
-#pragma unroll
-            for (int h = 0; h < G; ++h)
-#pragma unroll
-              for (int e = 0; e < E / 2; ++e) a2[h] = __ffma2_rn(qr[h][cc][e], k2[e], a2[h]);
-          }
+          for (int e = 1; e < E / 2; ++e) part[cc] = __ffma2_rn(qr[cc][e], kx[e], part[cc]);
         }
-        float dots[G];
 #pragma unroll
-        for (int h = 0; h < G; ++h) dots[h] = a2[h].x + a2[h].y;
-        ReduceScatter<G, TPR / 2>::run(dots, pp);
-        const uint32_t rmask = rv ? (uint32_t)mmask[mrow + RSL * i] : 0u;
-        const bool on = (rmask >> hb) & 1u;
-        if (on && lg_on) lg[mpos[mrow + RSL * i]] = dots[0];
-        sv[i] = on ? dots[0] : -INFINITY;
-      }
-      // ---- running maximum of every head over the warp's rows
-      float mx = sv[0];
+        for (int w2 = 1; w2 < CPL; w2 <<= 1)
 #pragma unroll
-      for (int i = 1; i < RQ; ++i) mx = fmaxf(mx, sv[i]);
-#pragma unroll
-      for (int o = TPR; o < 32; o <<= 1) mx = fmaxf(mx, __shfl_xor_sync(kFull, mx, o));
-      float tmax[G];
-      bool grow = false;
-#pragma unroll
-      for (int h = 0; h < G; ++h) {
-        tmax[h] = __shfl_sync(kFull, mx, h * LPH);
-        grow |= tmax[h] > m_run[h];
-      }
-      if (grow) {  // warp-uniform: every lane holds the same maxima
-        float a_own = 1.f;
-#pragma unroll
-        for (int h = 0; h < G; ++h) {
-          const float mn = fmaxf(m_run[h], tmax[h]);
-          const float al = (mn == m_run[h]) ? 1.f : fast_exp2((m_run[h] - mn) * sl);
-          m_run[h] = mn;
+          for (int cc = 0; cc + w2 < CPL; cc += 2 * w2) part[cc] = __fadd2_rn(part[cc], part[cc + w2]);
+        float dot = part[0].x + part[0].y;
+        dot += __shfl_xor_sync(kFull, dot, 1);
+        dot += __shfl_xor_sync(kFull, dot, 2);
+        if (lg_on && valid) lg[t0 + row] = dot;
+        const float sv = valid ? dot : -INFINITY;
+        // ---- online softmax with a lazy maximum (warp-uniform branch)
+        if (__any_sync(kFull, sv > mth)) {
+          const float mn = sv > mth ? sv : m;
+          const float al = (mn == m) ? 1.f : fast_exp2((m - mn) * sl);   // 0 while m is -inf
           const float2 a2 = make_float2(al, al);
-          acc[h][0] = __fmul2_rn(acc[h][0], a2);
-          acc[h][1] = __fmul2_rn(acc[h][1], a2);
-          if (h == hb) {
-            m_own = mn;
-            a_own = al;
-          }
+#pragma unroll
+          for (int cc = 0; cc < CPL; ++cc)
+#pragma unroll
+            for (int e = 0; e < E / 2; ++e) acc[cc][e] = __fmul2_rn(acc[cc][e], a2);
+          l *= al;
+          m = mn;
+          mth = (m == -INFINITY) ? -INFINITY : m + lazy;
+          msl = (m == -INFINITY) ? 0.f : m * sl;
         }
-        l_own *= a_own;
-        msl = (m_own == -INFINITY) ? 0.f : m_own * sl;
-      }
-      // ---- probabilities of the lane's rows, shared as (p, p) pairs
+        const float pr = fast_exp2(fmaf(sv, sl, -msl));   // 0 for rows not taken
+        l += pr;
+        // ---- P.V on the same row and quarter
+        if (valid) {
+          const unsigned char* vr = vt + row * ROWB;
+          const float2 p2 = make_float2(pr, pr);
 #pragma unroll
-      for (int i = 0; i < RQ; ++i) {
-        const float pr = fast_exp2(fmaf(sv[i], sl, -msl));
-        l_own += pr;
-        if (writer)
-          *reinterpret_cast<float2*>(smem + pw_off + i * RSL * G * 8) = make_float2(pr, pr);
-      }
-      __syncwarp();
-      // ---- P.V: lane (pc, rg) accumulates elements [4pc, 4pc+4) of rows rg + RGV*i
+          for (int cc = 0; cc < CPL; ++cc) {
+            float2 vx[E / 2];
+            Vec<T>::load16(vr + coff[cc], vx);
 #pragma unroll
-      for (int i = 0; i < PVR; ++i) {
-        if (WHOLE || (warp * RW + rg + RGV * i) < nrows) {
-          const unsigned char* pb = smem + pr_off + i * RGV * G * 8;
-          float2 pr2[G];
-          if constexpr (G == 1) {
-            pr2[0] = *reinterpret_cast<const float2*>(pb);
-          } else {
-#pragma unroll
-            for (int h = 0; h < G; h += 2) {
-              const float4 t = *reinterpret_cast<const float4*>(pb + h * 8);
-              pr2[h] = make_float2(t.x, t.y);
-              pr2[h + 1] = make_float2(t.z, t.w);
-            }
-          }
-          float2 v2[2];
-          Vec<T>::load4(smem + kst + voff + i * RGV * ROWB, v2);
-#pragma unroll
-          for (int h = 0; h < G; ++h) {
-            acc[h][0] = __ffma2_rn(pr2[h], v2[0], acc[h][0]);
-            acc[h][1] = __ffma2_rn(pr2[h], v2[1], acc[h][1]);
+            for (int e = 0; e < E / 2; ++e) acc[cc][e] = __ffma2_rn(p2, vx[e], acc[cc][e]);
           }
         }
       }
-    };
-    if (nrows == TT) tile(std::true_type{});
-    else tile(std::false_type{});
+    }
     __syncwarp();
     if (lane == 0) mbar_arrive(&empty[s]);
     if (++s == STAGES) {
@@ -628,62 +706,64 @@ __device__ __forceinline__ void consumer_loop(const AttnParams& p, unsigned char
     }
 
     if (flags & kLast) {
-      // ---- merge the warps' states in a fixed order and write one partial per head
-      float l_w = l_own;
+      if (myh >= 0) {
+        // ---- merge the warp's eight slots in registers: r^2, r^4 (same
+        // rotation), then r^1 (rotated by CPL/2 chunks)
 #pragma unroll
-      for (int o = TPR; o < 32; o <<= 1) l_w += __shfl_xor_sync(kFull, l_w, o);
+        for (int o = 2 * kLanesPerPair; o <= 4 * kLanesPerPair; o <<= 1) {
+          const MergeW w = merge_weights(m, l, __shfl_xor_sync(kFull, m, o),
+                                         __shfl_xor_sync(kFull, l, o), sl);
+          const float2 wa = make_float2(w.a, w.a), wb = make_float2(w.b, w.b);
 #pragma unroll
-      for (int o = PVC; o < 32; o <<= 1)
+          for (int cc = 0; cc < CPL; ++cc)
 #pragma unroll
-        for (int h = 0; h < G; ++h)
-#pragma unroll
-          for (int e = 0; e < 2; ++e) {
-            acc[h][e].x += __shfl_xor_sync(kFull, acc[h][e].x, o);
-            acc[h][e].y += __shfl_xor_sync(kFull, acc[h][e].y, o);
-          }
-      float* mg = merge + warp * G * MS;
-      if (rg == 0) {
-#pragma unroll
-        for (int h = 0; h < G; ++h)
-          *reinterpret_cast<float4*>(mg + h * MS + pc * 4) =
-              make_float4(acc[h][0].x, acc[h][0].y, acc[h][1].x, acc[h][1].y);
-      }
-      if (r == 0 && writer) {
-        mg[hb * MS + D] = l_w;
-        mg[hb * MS + D + 1] = m_own;
-      }
-      named_bar_sync(1, NW * 32);
-      for (int idx = threadIdx.x; idx < G * D; idx += NW * 32) {
-        const int h = idx / D, dim = idx % D;
-        float M = -INFINITY;
-#pragma unroll 4
-        for (int w = 0; w < NW; ++w) M = fmaxf(M, merge[(w * G + h) * MS + D + 1]);
-        float A = 0.f, L = 0.f;
-        if (M != -INFINITY) {
-#pragma unroll 4
-          for (int w = 0; w < NW; ++w) {
-            const float* e = merge + (w * G + h) * MS;
-            const float wt = (e[D + 1] == -INFINITY) ? 0.f : fast_exp2((e[D + 1] - M) * sl);
-            A = fmaf(e[dim], wt, A);
-            L = fmaf(e[D], wt, L);
-          }
+            for (int e = 0; e < E / 2; ++e) {
+              float2 x;
+              x.x = __shfl_xor_sync(kFull, acc[cc][e].x, o);
+              x.y = __shfl_xor_sync(kFull, acc[cc][e].y, o);
+              acc[cc][e] = __ffma2_rn(acc[cc][e], wa, __fmul2_rn(x, wb));
+            }
         }
-        const size_t slot = (size_t)(b * Hq + h0 + h) * p.nchunk + c;
-        p.part_acc[slot * D + dim] = A;
-        if (dim == 0) {
-          p.part_ml[slot * 2] = M;
-          p.part_ml[slot * 2 + 1] = L;
+        {
+          constexpr int o = kLanesPerPair;
+          const MergeW w = merge_weights(m, l, __shfl_xor_sync(kFull, m, o),
+                                         __shfl_xor_sync(kFull, l, o), sl);
+          const float2 wa = make_float2(w.a, w.a), wb = make_float2(w.b, w.b);
+          float2 x[CPL][E / 2];
+#pragma unroll
+          for (int cc = 0; cc < CPL; ++cc)
+#pragma unroll
+            for (int e = 0; e < E / 2; ++e) {
+              x[cc][e].x = __shfl_xor_sync(kFull, acc[(cc + CPL / 2) % CPL][e].x, o);
+              x[cc][e].y = __shfl_xor_sync(kFull, acc[(cc + CPL / 2) % CPL][e].y, o);
+            }
+#pragma unroll
+          for (int cc = 0; cc < CPL; ++cc)
+#pragma unroll
+            for (int e = 0; e < E / 2; ++e)
+              acc[cc][e] = __ffma2_rn(acc[cc][e], wa, __fmul2_rn(x[cc][e], wb));
+        }
+        // ---- slot 0 (lanes 0..3) writes the warp's state to its partial slot
+        if (r == 0) {
+          const size_t ps = ((size_t)(b * p.Hq + h0 + myh) * p.nchunk + c) * kPartSlots + slot;
+          float* dst = p.part_acc + ps * D + pp * DL;
+#pragma unroll
+          for (int cc = 0; cc < CPL; ++cc)
+#pragma unroll
+            for (int e = 0; e < E / 2; e += 2)
+              *reinterpret_cast<float4*>(dst + ((cc + rot) % CPL) * E + 2 * e) =
+                  make_float4(acc[cc][e].x, acc[cc][e].y, acc[cc][e + 1].x, acc[cc][e + 1].y);
+          if (pp == 0) *reinterpret_cast<float2*>(p.part_ml + ps * 2) = make_float2(m, l);
         }
       }
-      named_bar_sync(1, NW * 32);   // the slots are rewritten at the next item's end
     }
   }
 }
 
-template <typename T, int D, int G, int RQ, int NW, int NP, int STAGES>
+template <typename T, int D, int G, int NW, int NP, int TT, int STAGES>
 cudaError_t launch_attn_t(const AttnParams& p, int num_sms, cudaStream_t st) {
-  using C = AttnCfg<T, D, G, RQ, NW, NP, STAGES>;
-  auto kfn = attn_kernel<T, D, G, RQ, NW, NP, STAGES>;
+  using C = AttnCfg<T, D, G, NW, NP, TT, STAGES>;
+  auto kfn = attn_kernel<T, D, G, NW, NP, TT, STAGES>;
   static bool attr_set = false;  // per instantiation; set once per process
   if (!attr_set) {
     cudaError_t e =
@@ -696,11 +776,8 @@ cudaError_t launch_attn_t(const AttnParams& p, int num_sms, cudaStream_t st) {
   return cudaGetLastError();
 }
 
-// 16 warps per CTA: NW consumers and NP producers, 4 warps on each SM
-// sub-partition with up to 128 registers per thread.  q.K uses 8 lanes per row
-// (64 q values in registers for G <= 4) and RQ rows per lane; the producers
-// gather sparse rows with 16-byte copies and stream dense rows with TMA.
-// G = 8 keeps 128 q values per lane and runs 8 warps (up to 255 registers).
+// 16 warps per CTA: NW consumers and NP producers (builder, streaming warps), 4
+// warps on each SM sub-partition with up to 128 registers per thread.
 #ifndef LYCHEE_ATTN_NW
 #define LYCHEE_ATTN_NW 12
 #endif
@@ -711,31 +788,36 @@ cudaError_t launch_attn_t(const AttnParams& p, int num_sms, cudaStream_t st) {
 #define LYCHEE_ATTN_RING_KB 150
 #endif
 
-// Ring depth: about LYCHEE_ATTN_RING_KB of K/V tiles per SM, 2..8 stages.
-template <typename T, int D, int G, int RQ, int NW>
+// Tile rows: 96 rows of up to 256 bytes, 48 rows of 512 bytes (fp32, d = 128).
+template <typename T, int D>
+constexpr int tile_rows() {
+  return D * (int)sizeof(T) > 256 ? 48 : 96;
+}
+
+// Ring depth: about LYCHEE_ATTN_RING_KB of K/V tiles (and q) per SM, 2..8 stages.
+template <typename T, int D, int G, int TT>
 constexpr int ring_stages() {
-  constexpr int bytes = 2 * NW * 4 * RQ * D * (int)sizeof(T) +
-                        (G * D * (int)sizeof(T) + 127) / 128 * 128;   // K, V tiles and q
+  constexpr int bytes = 2 * TT * D * (int)sizeof(T) + (G * D * (int)sizeof(T) + 127) / 128 * 128;
   constexpr int s = (LYCHEE_ATTN_RING_KB * 1024) / bytes;
   return s < 2 ? 2 : (s > 8 ? 8 : s);
 }
 
-template <typename T, int D, int G, int RQ, int NW, int NP>
+template <typename T, int D, int G>
 cudaError_t launch_attn_g(const AttnParams& p, int num_sms, cudaStream_t st) {
-  constexpr int STAGES = ring_stages<T, D, G, RQ, NW>();
-  static_assert(AttnCfg<T, D, G, RQ, NW, NP, STAGES>::SMEM <= 227 * 1024, "shared memory");
-  return launch_attn_t<T, D, G, RQ, NW, NP, STAGES>(p, num_sms, st);
+  constexpr int NW = LYCHEE_ATTN_NW, NP = LYCHEE_ATTN_NP;
+  constexpr int TT = tile_rows<T, D>();
+  constexpr int STAGES = ring_stages<T, D, G, TT>();
+  static_assert(AttnCfg<T, D, G, NW, NP, TT, STAGES>::SMEM <= 227 * 1024, "shared memory");
+  return launch_attn_t<T, D, G, NW, NP, TT, STAGES>(p, num_sms, st);
 }
 
 template <typename T, int D>
 cudaError_t launch_attn_d(const AttnParams& p, int G, int num_sms, cudaStream_t st) {
-  constexpr int NW = LYCHEE_ATTN_NW, NP = LYCHEE_ATTN_NP;
-  constexpr int RQ = (sizeof(T) * D > 256) ? 1 : 2;   // fp32 rows of 512 bytes: one per lane
   switch (G) {
-    case 1: return launch_attn_g<T, D, 1, RQ, NW, NP>(p, num_sms, st);
-    case 2: return launch_attn_g<T, D, 2, RQ, NW, NP>(p, num_sms, st);
-    case 4: return launch_attn_g<T, D, 4, RQ, NW, NP>(p, num_sms, st);
-    case 8: return launch_attn_g<T, D, 8, 1, 6, 2>(p, num_sms, st);
+    case 1: return launch_attn_g<T, D, 1>(p, num_sms, st);
+    case 2: return launch_attn_g<T, D, 2>(p, num_sms, st);
+    case 4: return launch_attn_g<T, D, 4>(p, num_sms, st);
+    case 8: return launch_attn_g<T, D, 8>(p, num_sms, st);
     default: return cudaErrorInvalidValue;
   }
 }

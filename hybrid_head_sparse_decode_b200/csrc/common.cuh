@@ -30,6 +30,8 @@ struct WsHeader {
 static_assert(sizeof(WsHeader) == 256, "header is 256 bytes");
 
 constexpr int kChunk = 960;           // positions per attention work item (30 words)
+constexpr int kPartSlots = 12;        // partial states per (sequence, head, chunk): one per warp
+constexpr int kCombineSplit = 4;      // combine CTAs per (sequence, head)
 constexpr int kMaxHq = 128;           // query heads supported
 constexpr uint64_t kWaitLimitNs = 2000000000ull;   // 2 s: a wait this long is a fault
 
@@ -140,6 +142,22 @@ __device__ __forceinline__ void bulk_g2s(void* dst, const void* src, uint32_t by
       "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint"
       " [%0], [%1], %2, [%3], %4;" ::"r"(smem_u32(dst)),
       "l"(src), "r"(bytes), "r"(smem_u32(bar)), "l"(policy)
+      : "memory");
+}
+
+// ---- row gather through a tensor map (TMA tile::gather4, no multicast) ----------
+// The tensor map describes a 2-D array of rows (inner dimension: the row's
+// elements) with a box one row high and one full row wide.  One instruction
+// copies rows y0..y3 (any order, repeats allowed), columns from x (a multiple
+// of 16 bytes; 0 here), into four consecutive box-sized slots at dst (128-byte
+// aligned).  Completion is signalled as transaction bytes on `bar`.
+__device__ __forceinline__ void tma_gather4(void* dst, const void* tmap, int x, int y0, int y1,
+                                            int y2, int y3, uint64_t* bar, uint64_t policy) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.tile::gather4.mbarrier::complete_tx::bytes"
+      ".L2::cache_hint [%0], [%1, {%2, %3, %4, %5, %6}], [%7], %8;" ::"r"(smem_u32(dst)),
+      "l"(reinterpret_cast<uint64_t>(tmap)), "r"(x), "r"(y0), "r"(y1), "r"(y2), "r"(y3),
+      "r"(smem_u32(bar)), "l"(policy)
       : "memory");
 }
 

@@ -1,6 +1,7 @@
 // kernels.h -- parameter blocks and launchers of the libychee kernels (internal).
 #pragma once
 
+#include <cuda.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
 
@@ -14,8 +15,10 @@ struct AttnParams {
   const int32_t* seqlens;   // [B]
   const uint32_t* bitmaps;  // [B, Hq, nwords]: incoming sets of sparse heads
   float* logits;            // [B, Hq, N_max]: raw q.k of retrieval heads
-  float* part_ml;           // [B, Hq, nchunk, 2]: (max raw dot, sum of weights)
-  float* part_acc;          // [B, Hq, nchunk, D]: unnormalised weighted values
+  float* part_ml;           // [B, Hq, nchunk, kPartSlots, 2]: (max raw dot, sum of weights)
+  float* part_acc;          // [B, Hq, nchunk, kPartSlots, D]: unnormalised weighted values
+  int32_t* part_n;          // [B, Hq, nchunk]: partial states written for the chunk
+  uint32_t* ccnt;           // [B, Hq]: combine counters, zeroed here for the combine kernel
   const int32_t* k_per_seq; // [B] or null (validated here)
   uint32_t* err;
   uint32_t* counter;        // work-item counter, 0 at launch, 0 again at exit
@@ -23,6 +26,11 @@ struct AttnParams {
   int B, Hq, Hkv, N_max, nwords, nchunk, n_items;
   float scale_log2;         // log2(e) / sqrt(D)
   uint32_t role[4];         // bit h set: head h is a retrieval head
+  int gather_tma;           // 1: sparse rows are gathered through tmk / tmv
+  // K and V caches viewed as [B * Hkv * N_max] rows of D elements, box one row
+  // (TMA tile::gather4); valid when gather_tma is 1
+  alignas(64) CUtensorMap tmk;
+  alignas(64) CUtensorMap tmv;
 };
 cudaError_t launch_attn(const AttnParams& p, int dtype, int D, int G, int num_sms,
                         cudaStream_t st);
@@ -42,8 +50,11 @@ cudaError_t launch_topk(const TopkParams& p, cudaStream_t st);
 
 // Merge of split partials into the attention output (combine.cu).
 struct CombineParams {
-  const float* part_ml;      // [B, Hq, nchunk, 2]
-  const float* part_acc;     // [B, Hq, nchunk, D]
+  const float* part_ml;      // [B, Hq, nchunk, kPartSlots, 2]
+  const float* part_acc;     // [B, Hq, nchunk, kPartSlots, D]
+  const int32_t* part_n;     // [B, Hq, nchunk]: states used per chunk
+  float* part2;              // [B, Hq, kCombineSplit, D + 4]: one state per combine CTA
+  uint32_t* ccnt;            // [B, Hq]: finished combine CTAs (0 at launch, 0 again at exit)
   const int32_t* seqlens;    // [B]
   void* out;                 // [B, Hq, D]
   int B, Hq, N_max, nchunk;

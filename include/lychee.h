@@ -124,9 +124,9 @@ LYCHEE_API lychee_status lychee_hybrid_decode_attn(const lychee_shape* s, const 
                                         size_t workspace_bytes, void* stream);
 
 /* Size of the static device scratch behind lychee_hybrid_decode_attn_noalloc:
- * 32 MiB per device, enough for a layer whose lychee_workspace_size() is at
- * most that (e.g. B = 1, Hq = 32, d = 128, N_max = 131072 needs about 19 MiB). */
-#define LYCHEE_NOALLOC_SCRATCH_BYTES (32u << 20)
+ * 64 MiB per device, enough for a layer whose lychee_workspace_size() is at
+ * most that (e.g. B = 1, Hq = 32, d = 128, N_max = 131072 needs about 43 MiB). */
+#define LYCHEE_NOALLOC_SCRATCH_BYTES (64u << 20)
 
 /* lychee_hybrid_decode_attn without a caller-owned workspace and without any
  * device allocation.  The method has no counterpart to this call: it is a

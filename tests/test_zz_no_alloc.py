@@ -31,7 +31,7 @@ def test_scratch_size_matches_header():
 
 
 def test_oversize_layer_refused_on_host(lib):
-    # B = 2, Hq = 32, N_max = 131072: ~38 MiB of scratch > 32 MiB
+    # B = 2, Hq = 32, N_max = 131072: ~86 MiB of scratch > 64 MiB
     s = N.Shape(2, 32, 8, 128, 131072, N.BF16, 39321)
     assert lib.lychee_workspace_size(ctypes.byref(s)) > N.NOALLOC_SCRATCH_BYTES
     roles = (ctypes.c_uint8 * 32)(*([1] * 32))
