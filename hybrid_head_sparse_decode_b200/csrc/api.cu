@@ -148,7 +148,14 @@ struct Profiler {
 };
 Profiler g_prof;
 
-enum { kKindAttn = 0, kKindTopk = 1, kKindCombine = 2, kKindBuildBits = 3, kKindExport = 4 };
+enum {
+  kKindAttn = 0,
+  kKindTopk = 1,
+  kKindCombine = 2,
+  kKindBuildBits = 3,
+  kKindExport = 4,
+  kKindTopkCombine = 5
+};
 
 template <typename F>
 cudaError_t timed(int kind, cudaStream_t st, F&& launch) {
@@ -237,20 +244,18 @@ lychee_status run_layer(const Ctx& c, const void* q, const void* kc, const void*
   ap.gather_tma = (encode_row_map(&ap.tmk, kc, s) && encode_row_map(&ap.tmv, vc, s)) ? 1 : 0;
   e = timed(kKindAttn, c.st, [&] { return launch_attn(ap, s->dtype, s->d, G, c.sms, c.st); });
   if (e != cudaSuccess) return LYCHEE_ERR_CUDA;
-  if (nr > 0) {
-    TopkParams tp{};
-    tp.logits = logits;
-    tp.seqlens = seqlens;
-    tp.k_per_seq = k_per_seq;
-    tp.bitmaps = write_bits ? bitmaps : nullptr;
-    tp.idx_out = idx_out;
-    tp.err = err;
-    tp.B = s->B; tp.Hq = Hq; tp.N_max = s->N_max; tp.nwords = c.L.nwords; tp.k = s->k;
-    tp.nheads = nr;
-    std::memcpy(tp.heads, rheads, nr);
-    e = timed(kKindTopk, c.st, [&] { return launch_topk(tp, c.st); });
-    if (e != cudaSuccess) return LYCHEE_ERR_CUDA;
-  }
+  // top-k of the retrieval heads and the combine of every head: independent
+  // (logits vs partial states), so one launch does both
+  TopkParams tp{};
+  tp.logits = logits;
+  tp.seqlens = seqlens;
+  tp.k_per_seq = k_per_seq;
+  tp.bitmaps = write_bits ? bitmaps : nullptr;
+  tp.idx_out = idx_out;
+  tp.err = err;
+  tp.B = s->B; tp.Hq = Hq; tp.N_max = s->N_max; tp.nwords = c.L.nwords; tp.k = s->k;
+  tp.nheads = nr;
+  std::memcpy(tp.heads, rheads, nr);
   CombineParams cp{};
   cp.part_ml = part_ml;
   cp.part_acc = part_acc;
@@ -261,7 +266,8 @@ lychee_status run_layer(const Ctx& c, const void* q, const void* kc, const void*
   cp.out = out;
   cp.B = s->B; cp.Hq = Hq; cp.N_max = s->N_max; cp.nchunk = c.L.nchunk;
   cp.scale_log2 = ap.scale_log2;
-  e = timed(kKindCombine, c.st, [&] { return launch_combine(cp, s->dtype, s->d, c.st); });
+  e = timed(nr > 0 ? kKindTopkCombine : kKindCombine, c.st,
+            [&] { return launch_topk_combine(tp, cp, s->dtype, s->d, c.st); });
   if (e != cudaSuccess) return LYCHEE_ERR_CUDA;
   return LYCHEE_OK;
 }

@@ -76,21 +76,25 @@ struct Vec;
 template <>
 struct Vec<__nv_bfloat16> {
   static constexpr int E = 8;  // elements per 16-byte chunk
-  __device__ __forceinline__ static void load16(const void* p, float2 (&o)[4]) {
-    const uint4 w = *reinterpret_cast<const uint4*>(p);
+  __device__ __forceinline__ static void widen(uint4 w, float2 (&o)[4]) {
     o[0] = bf16x2_to_float2(w.x);
     o[1] = bf16x2_to_float2(w.y);
     o[2] = bf16x2_to_float2(w.z);
     o[3] = bf16x2_to_float2(w.w);
   }
+  __device__ __forceinline__ static void load16(const void* p, float2 (&o)[4]) {
+    widen(*reinterpret_cast<const uint4*>(p), o);
+  }
 };
 template <>
 struct Vec<float> {
   static constexpr int E = 4;
+  __device__ __forceinline__ static void widen(uint4 w, float2 (&o)[2]) {
+    o[0] = make_float2(__uint_as_float(w.x), __uint_as_float(w.y));
+    o[1] = make_float2(__uint_as_float(w.z), __uint_as_float(w.w));
+  }
   __device__ __forceinline__ static void load16(const void* p, float2 (&o)[2]) {
-    const float4 w = *reinterpret_cast<const float4*>(p);
-    o[0] = make_float2(w.x, w.y);
-    o[1] = make_float2(w.z, w.w);
+    widen(*reinterpret_cast<const uint4*>(p), o);
   }
 };
 
@@ -107,21 +111,19 @@ struct AttnCfg {
   static constexpr int MAXT = (kChunk + TT - 1) / TT;   // tiles per item at most
   static_assert(CPL >= 2 && DL % E == 0 && CPL % 2 == 0, "lane mapping");
   static_assert(TT % kPairsPerBatch == 0 && TT % 4 == 0 && TT <= 255, "tile rows");
-  static_assert(G <= NW && NW <= kPartSlots && NW < 16, "warps per head fit the partial slots");
+  static_assert(G <= NW && NW <= kPartSlots && NW <= 16, "warps per head fit the partial slots");
   static_assert(NP >= 2, "a builder and at least one streaming warp");
   static_assert(kChunk % 32 == 0 && kChunk <= 1024, "builder holds one word per lane");
   static_assert(MAXT < 32, "one lane per tile start");
 
-  // item buffer (two of them): descriptor, warp assignment, the chunk's union
-  // bitmap words, each head's bitmap words, the union index of each word's
-  // first row, the gather positions
-  static constexpr int NWD = kChunk / 32;         // bitmap words per chunk
+  // item buffer (two of them): descriptor, warp assignment, where each tile
+  // starts in each sparse head's row list, the row lists (union indices of the
+  // head's rows, in order), the gather positions
   static constexpr int ASGB = NW + G;             // warp -> (head, slot), warps per head
   static constexpr int IB_ASG = 32;
-  static constexpr int IB_UW = IB_ASG + (ASGB + 15) / 16 * 16;          // [32] u32
-  static constexpr int IB_HW = IB_UW + 32 * 4;                           // [G][32] u32
-  static constexpr int IB_UB = IB_HW + G * 32 * 4;                       // [32] i32
-  static constexpr int IB_LPOS = IB_UB + 32 * 4;                         // [kChunk] i32
+  static constexpr int IB_TST = IB_ASG + (ASGB + 15) / 16 * 16;          // [G][32] u16
+  static constexpr int IB_HROW = IB_TST + G * 32 * 2;                    // [G][kChunk] u16
+  static constexpr int IB_LPOS = IB_HROW + G * kChunk * 2;               // [kChunk] i32
   static constexpr int IBUF = IB_LPOS + kChunk * 4;
 
   // shared memory layout (byte offsets from a 128-byte aligned base)
@@ -133,8 +135,7 @@ struct AttnCfg {
   static constexpr int OFF_Q = OFF_V + STAGES * kStageKV;
   static constexpr int OFF_INFO = OFF_Q + STAGES * QSTRIDE;             // [STAGES][2] int4
   static constexpr int OFF_ITEM = OFF_INFO + STAGES * 32;               // [2][IBUF]
-  static constexpr int OFF_HL = OFF_ITEM + 2 * IBUF;                    // [NW][kChunk] u16
-  static constexpr int OFF_CUM = OFF_HL + NW * kChunk * 2;
+  static constexpr int OFF_CUM = OFF_ITEM + 2 * IBUF;
   static constexpr int OFF_BAR = (OFF_CUM + (kMaxBatchCompact + 1) * 4 + 15) / 16 * 16;
   static constexpr int NBAR = 2 * STAGES + 4;     // full, empty, ready[2], freeb[2]
   static constexpr int SMEM = OFF_BAR + NBAR * 8 + 128;   // + alignment slack
@@ -365,20 +366,44 @@ __global__ void __launch_bounds__((NW + NP) * 32, 1)
               lpos[o++] = p0 + 32 * lane + j;
             }
           }
-          // the words the consumer warps build their heads' row lists from
-          uint32_t* uw = reinterpret_cast<uint32_t*>(ib + C::IB_UW);
-          uint32_t* hw = reinterpret_cast<uint32_t*>(ib + C::IB_HW);
-          int32_t* ub = reinterpret_cast<int32_t*>(ib + C::IB_UB);
-          uw[lane] = uni;
-          ub[lane] = ubase;
+          // each sparse head's rows as union indices, in order: one word at a
+          // time, lane j placing bit j of the word; then, per tile, where the
+          // tile starts in the list (a retrieval head takes every row: no list)
+          uint16_t* hrow = reinterpret_cast<uint16_t*>(ib + C::IB_HROW);
+          uint16_t* tst = reinterpret_cast<uint16_t*>(ib + C::IB_TST);
+          const uint32_t lt = (1u << lane) - 1u;
+          const int ntile = (total + TT - 1) / TT;
           int work[G];
 #pragma unroll
           for (int t = 0; t < G; ++t) {
-            hw[t * 32 + lane] = bits[t];
-            int ct = __popc(bits[t]);
+            const int ct = __popc(bits[t]);
+            int ic = ct;
 #pragma unroll
-            for (int o = 16; o >= 1; o >>= 1) ct += __shfl_xor_sync(kFull, ct, o);
-            work[t] = ct;
+            for (int o = 1; o < 32; o <<= 1) {
+              const int y = __shfl_up_sync(kFull, ic, o);
+              if (lane >= o) ic += y;
+            }
+            work[t] = __shfl_sync(kFull, ic, 31);
+            if ((rmask >> t) & 1u) continue;
+            uint16_t* hl = hrow + t * kChunk;
+            const int hpre = ic - ct;
+#pragma unroll 6
+            for (int w = 0; w < nwords; ++w) {
+              const uint32_t bw = __shfl_sync(kFull, bits[t], w);
+              const uint32_t uw = __shfl_sync(kFull, uni, w);
+              const int hp = __shfl_sync(kFull, hpre, w);
+              const int ubw = __shfl_sync(kFull, ubase, w);
+              if ((bw >> lane) & 1u) hl[hp + __popc(bw & lt)] = (uint16_t)(ubw + __popc(uw & lt));
+            }
+            __syncwarp();
+            const int bound = lane * TT;
+            int lo = 0, hi = work[t];
+            while (lo < hi) {
+              const int mid = (lo + hi) >> 1;
+              if ((int)hl[mid] < bound) lo = mid + 1;
+              else hi = mid;
+            }
+            if (lane <= ntile) tst[t * 32 + lane] = (uint16_t)lo;
           }
           if (lane == 0) assign_warps<G, NW>(work, asg, asg + NW);
           __syncwarp();
@@ -554,8 +579,7 @@ __device__ __forceinline__ void consumer_loop(const AttnParams& p, unsigned char
   float2 acc[CPL][E / 2];
   float m = -INFINITY, mth = -INFINITY, msl = 0.f, l = 0.f;
   int myh = -1, slot = 0, nh = 1, buf = 0;
-  int tstart = 0;                          // lane t: start of tile t in the head's row list
-  uint16_t* hl = reinterpret_cast<uint16_t*>(smem + C::OFF_HL) + warp * kChunk;
+
   bool ident = false, lg_on = false;
   float* lg = nullptr;
   int b = 0, h0 = 0, c = 0;
@@ -589,53 +613,22 @@ __device__ __forceinline__ void consumer_loop(const AttnParams& p, unsigned char
 #pragma unroll
           for (int e = 0; e < E / 2; ++e) acc[cc][e] = make_float2(0.f, 0.f);
         }
-        if (!ident) {
-          // the head's rows as union indices of the item, in order, and where
-          // each tile starts in that list
-          const uint32_t bt = reinterpret_cast<const uint32_t*>(ib + C::IB_HW)[myh * 32 + lane];
-          const uint32_t uu = reinterpret_cast<const uint32_t*>(ib + C::IB_UW)[lane];
-          const int base = reinterpret_cast<const int32_t*>(ib + C::IB_UB)[lane];
-          const int ct = __popc(bt);
-          int ic = ct;
-#pragma unroll
-          for (int o = 1; o < 32; o <<= 1) {
-            const int y = __shfl_up_sync(kFull, ic, o);
-            if (lane >= o) ic += y;
-          }
-          const int nh_rows = __shfl_sync(kFull, ic, 31);
-          int kk = ic - ct;
-          uint32_t u = bt;
-          while (u) {
-            const int j = __ffs(u) - 1;
-            u &= u - 1;
-            hl[kk++] = (uint16_t)(base + __popc(uu & ((1u << j) - 1u)));
-          }
-          __syncwarp();
-          const int bound = lane * TT;
-          int lo = 0, hi = nh_rows;
-          while (lo < hi) {
-            const int mid = (lo + hi) >> 1;
-            if ((int)hl[mid] < bound) lo = mid + 1;
-            else hi = mid;
-          }
-          tstart = lo;
-        }
       }
       m = -INFINITY;
       mth = -INFINITY;
       msl = 0.f;
       l = 0.f;
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&freeb[buf]);   // done reading this item's buffer
     }
 
     if (myh >= 0) {
       // this tile's rows of the warp's head: all of them for a retrieval head,
       // else a slice of the head's row list (union indices of the item)
       int cnt = nrows, st0 = 0;
+      const uint16_t* hl = reinterpret_cast<const uint16_t*>(ib + C::IB_HROW) + myh * kChunk;
       if (!ident) {
-        st0 = __shfl_sync(kFull, tstart, tt);
-        cnt = __shfl_sync(kFull, tstart, tt + 1) - st0;
+        const uint16_t* ts = reinterpret_cast<const uint16_t*>(ib + C::IB_TST) + myh * 32;
+        st0 = ts[tt];
+        cnt = (int)ts[tt + 1] - st0;
       }
       const int nb = (cnt + kPairsPerBatch - 1) / kPairsPerBatch;
       const unsigned char* kt = smem + C::OFF_K + s * C::kStageKV;
@@ -648,13 +641,23 @@ __device__ __forceinline__ void consumer_loop(const AttnParams& p, unsigned char
         const int idx = k * kPairsPerBatch + r;
         const bool valid = idx < cnt;
         const int row = valid ? (ident ? idx : (int)hl[st0 + idx] - t0) : 0;
-        // ---- q.K over the lane's quarter: CPL independent partial sums
+        // ---- the pair's K and V chunks (V is fetched now so that its load is
+        // off the softmax's critical path; row 0 always holds real data, and
+        // a pair that is not taken gets weight 0)
         const unsigned char* kr = kt + row * ROWB;
+        const unsigned char* vr = vt + row * ROWB;
+        uint4 kraw[CPL], vraw[CPL];
+#pragma unroll
+        for (int cc = 0; cc < CPL; ++cc) {
+          kraw[cc] = *reinterpret_cast<const uint4*>(kr + coff[cc]);
+          vraw[cc] = *reinterpret_cast<const uint4*>(vr + coff[cc]);
+        }
+        // ---- q.K over the lane's quarter: CPL independent partial sums
         float2 part[CPL];
 #pragma unroll
         for (int cc = 0; cc < CPL; ++cc) {
           float2 kx[E / 2];
-          Vec<T>::load16(kr + coff[cc], kx);
+          Vec<T>::widen(kraw[cc], kx);
           part[cc] = __fmul2_rn(qr[cc][0], kx[0]);
 #pragma unroll
           for (int e = 1; e < E / 2; ++e) part[cc] = __ffma2_rn(qr[cc][e], kx[e], part[cc]);
@@ -685,16 +688,13 @@ __device__ __forceinline__ void consumer_loop(const AttnParams& p, unsigned char
         const float pr = fast_exp2(fmaf(sv, sl, -msl));   // 0 for rows not taken
         l += pr;
         // ---- P.V on the same row and quarter
-        if (valid) {
-          const unsigned char* vr = vt + row * ROWB;
-          const float2 p2 = make_float2(pr, pr);
+        const float2 p2 = make_float2(pr, pr);
 #pragma unroll
-          for (int cc = 0; cc < CPL; ++cc) {
-            float2 vx[E / 2];
-            Vec<T>::load16(vr + coff[cc], vx);
+        for (int cc = 0; cc < CPL; ++cc) {
+          float2 vx[E / 2];
+          Vec<T>::widen(vraw[cc], vx);
 #pragma unroll
-            for (int e = 0; e < E / 2; ++e) acc[cc][e] = __ffma2_rn(p2, vx[e], acc[cc][e]);
-          }
+          for (int e = 0; e < E / 2; ++e) acc[cc][e] = __ffma2_rn(p2, vx[e], acc[cc][e]);
         }
       }
     }
@@ -706,6 +706,7 @@ __device__ __forceinline__ void consumer_loop(const AttnParams& p, unsigned char
     }
 
     if (flags & kLast) {
+      if (lane == 0) mbar_arrive(&freeb[buf]);   // done with this item's buffer
       if (myh >= 0) {
         // ---- merge the warp's eight slots in registers: r^2, r^4 (same
         // rotation), then r^1 (rotated by CPL/2 chunks)
@@ -785,20 +786,29 @@ cudaError_t launch_attn_t(const AttnParams& p, int num_sms, cudaStream_t st) {
 #define LYCHEE_ATTN_NP 4
 #endif
 #ifndef LYCHEE_ATTN_RING_KB
-#define LYCHEE_ATTN_RING_KB 150
+#define LYCHEE_ATTN_RING_KB 200
 #endif
 
-// Tile rows: 96 rows of up to 256 bytes, 48 rows of 512 bytes (fp32, d = 128).
+#ifndef LYCHEE_ATTN_TT
+#define LYCHEE_ATTN_TT 96
+#endif
+
+// Tile rows: LYCHEE_ATTN_TT rows of up to 256 bytes, half as many of 512 bytes
+// (fp32, d = 128).
 template <typename T, int D>
 constexpr int tile_rows() {
-  return D * (int)sizeof(T) > 256 ? 48 : 96;
+  return D * (int)sizeof(T) > 256 ? LYCHEE_ATTN_TT / 2 : LYCHEE_ATTN_TT;
 }
 
-// Ring depth: about LYCHEE_ATTN_RING_KB of K/V tiles (and q) per SM, 2..8 stages.
-template <typename T, int D, int G, int TT>
+// Ring depth: as many stages (2..8) as the shared memory left by everything else
+// holds, within LYCHEE_ATTN_RING_KB of K/V tiles and q.
+template <typename T, int D, int G, int NW, int NP, int TT>
 constexpr int ring_stages() {
-  constexpr int bytes = 2 * TT * D * (int)sizeof(T) + (G * D * (int)sizeof(T) + 127) / 128 * 128;
-  constexpr int s = (LYCHEE_ATTN_RING_KB * 1024) / bytes;
+  constexpr int stage = 2 * TT * D * (int)sizeof(T) + (G * D * (int)sizeof(T) + 127) / 128 * 128;
+  constexpr int rest = AttnCfg<T, D, G, NW, NP, TT, 1>::SMEM - stage;   // per-stage extras are small
+  constexpr int fit = (227 * 1024 - rest) / (stage + 64);
+  constexpr int want = (LYCHEE_ATTN_RING_KB * 1024) / stage;
+  constexpr int s = fit < want ? fit : want;
   return s < 2 ? 2 : (s > 8 ? 8 : s);
 }
 
@@ -806,7 +816,7 @@ template <typename T, int D, int G>
 cudaError_t launch_attn_g(const AttnParams& p, int num_sms, cudaStream_t st) {
   constexpr int NW = LYCHEE_ATTN_NW, NP = LYCHEE_ATTN_NP;
   constexpr int TT = tile_rows<T, D>();
-  constexpr int STAGES = ring_stages<T, D, G, TT>();
+  constexpr int STAGES = ring_stages<T, D, G, NW, NP, TT>();
   static_assert(AttnCfg<T, D, G, NW, NP, TT, STAGES>::SMEM <= 227 * 1024, "shared memory");
   return launch_attn_t<T, D, G, NW, NP, TT, STAGES>(p, num_sms, st);
 }

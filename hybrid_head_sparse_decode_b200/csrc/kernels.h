@@ -62,6 +62,11 @@ struct CombineParams {
 };
 cudaError_t launch_combine(const CombineParams& p, int dtype, int D, cudaStream_t st);
 
+// The top-k of the retrieval heads and the combine of every head in one launch
+// (topk.cu); just the combine when p.nheads is 0.
+cudaError_t launch_topk_combine(const TopkParams& p, const CombineParams& cp, int dtype, int D,
+                                cudaStream_t st);
+
 // Incoming index sets -> membership bitmaps, with validation; the rows are also
 // copied to idx_out (sparse heads pass their set on unchanged) (sets.cu).
 struct BuildBitsParams {

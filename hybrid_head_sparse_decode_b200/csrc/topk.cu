@@ -18,6 +18,7 @@
 // selecting on attention weights.
 #include <algorithm>
 
+#include "combine_body.cuh"
 #include "common.cuh"
 #include "kernels.h"
 
@@ -57,10 +58,11 @@ __device__ __forceinline__ uint32_t block_exclusive_scan(uint32_t v, uint32_t* w
   return before + x - v;
 }
 
+// One CTA of the selection: CTA `cta` of cluster cta / C (its rank in the
+// cluster is the hardware rank), dynamic shared memory at dsm.
 template <int C>
-__global__ void __launch_bounds__(kThreads, 1)
-    topk_kernel(const __grid_constant__ TopkParams p, int keys_cap, int wpc_cap) {
-  extern __shared__ __align__(16) uint32_t dsm[];
+__device__ __forceinline__ void topk_body(const TopkParams& p, int keys_cap, int wpc_cap, int cta,
+                                          uint32_t* dsm) {
   uint32_t* keys = dsm;                    // [keys_cap]
   uint32_t* wa = keys + keys_cap;          // [wpc_cap] tie bits, then selected bits
   uint32_t* wb = wa + wpc_cap;             // [wpc_cap] greater bits, then output offsets
@@ -72,7 +74,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const uint32_t rank = cluster_ctarank();
-  const int pair = blockIdx.x / C;
+  const int pair = cta / C;
   const int b = pair / p.nheads, h = p.heads[pair % p.nheads];
   const int n = min(max(p.seqlens[b], 1), p.N_max);
   int kb = p.k_per_seq ? p.k_per_seq[b] : p.k;
@@ -225,6 +227,28 @@ __global__ void __launch_bounds__(kThreads, 1)
   cluster_sync();  // no CTA leaves while a peer may still read its shared memory
 }
 
+template <int C>
+__global__ void __launch_bounds__(kThreads, 1)
+    topk_kernel(const __grid_constant__ TopkParams p, int keys_cap, int wpc_cap) {
+  extern __shared__ __align__(16) uint32_t dsm[];
+  topk_body<C>(p, keys_cap, wpc_cap, blockIdx.x, dsm);
+}
+
+// Top-k of the retrieval heads and the combine of all heads in one launch: the
+// first ntopk CTAs (whole clusters) select, the next ncomb CTAs combine (their
+// clusters never synchronise), the rest of the last cluster has nothing to do.
+// The two read disjoint data (logits; partial states) and write disjoint
+// outputs (sets; the attention output).
+template <int C, typename T, int D>
+__global__ void __launch_bounds__(kThreads, 1)
+    topk_combine_kernel(const __grid_constant__ TopkParams p, const __grid_constant__ CombineParams cp,
+                        int keys_cap, int wpc_cap, int ntopk, int ncomb) {
+  extern __shared__ __align__(16) uint32_t dsm[];
+  const int cta = blockIdx.x;
+  if (cta < ntopk) topk_body<C>(p, keys_cap, wpc_cap, cta, dsm);
+  else if (cta - ntopk < ncomb) combine_body<T, D>(cp, cta - ntopk, reinterpret_cast<unsigned char*>(dsm));
+}
+
 // Launch geometry of a cluster size C for rows of up to N_max logits.
 template <int C>
 struct Geometry {
@@ -306,7 +330,47 @@ bool cluster16_ok(int N_max, cudaStream_t st) {
   return ok;
 }
 
+template <int C, typename T, int D>
+cudaError_t launch_tc(const TopkParams& p, const CombineParams& cp, cudaStream_t st) {
+  static_assert(kThreads == kCombThreads, "one block size for both roles");
+  const Geometry<C> g(p.N_max);
+  if (!g.ok) return cudaErrorInvalidValue;
+  static bool done = false;
+  auto kfn = topk_combine_kernel<C, T, D>;
+  if (!done) {
+    cudaError_t e = cudaFuncSetAttribute(kfn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemBudget);
+    if (e == cudaSuccess && C > 8) e = cudaFuncSetAttribute(kfn, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+    if (e != cudaSuccess) return e;
+    done = true;
+  }
+  const int ntopk = C * p.B * p.nheads;
+  const int ncomb = cp.B * cp.Hq * kCombineSplit;
+  const int grid = (ntopk + ncomb + C - 1) / C * C;
+  const size_t smem = std::max(g.smem, combine_smem_bytes<D>());
+  cudaLaunchConfig_t cfg;
+  cudaLaunchAttribute at[1];
+  fill_config<C>(cfg, at, (unsigned)grid, smem, st);
+  cudaError_t e = cudaLaunchKernelEx(&cfg, kfn, p, cp, g.keys_cap, g.wpc_cap, ntopk, ncomb);
+  if (e != cudaSuccess) return e;
+  return cudaGetLastError();
+}
+
+template <typename T, int D>
+cudaError_t launch_tc_d(const TopkParams& p, const CombineParams& cp, cudaStream_t st) {
+  return cluster16_ok(p.N_max, st) ? launch_tc<16, T, D>(p, cp, st) : launch_tc<8, T, D>(p, cp, st);
+}
+
 }  // namespace
+
+cudaError_t launch_topk_combine(const TopkParams& p, const CombineParams& cp, int dtype, int D,
+                                cudaStream_t st) {
+  if (p.nheads <= 0) return launch_combine(cp, dtype, D, st);
+  if (dtype == 0 && D == 128) return launch_tc_d<__nv_bfloat16, 128>(p, cp, st);
+  if (dtype == 0 && D == 64) return launch_tc_d<__nv_bfloat16, 64>(p, cp, st);
+  if (dtype == 1 && D == 128) return launch_tc_d<float, 128>(p, cp, st);
+  if (dtype == 1 && D == 64) return launch_tc_d<float, 64>(p, cp, st);
+  return cudaErrorInvalidValue;
+}
 
 cudaError_t launch_topk(const TopkParams& p, cudaStream_t st) {
   if (p.nheads <= 0) return cudaSuccess;

@@ -220,7 +220,8 @@ def workspace_views(workspace, B, Hq, Hkv, d, N_max, k, dtype):
 class Profile:
     """Context manager around lychee_profile_begin / lychee_profile_end.
     After exit, ``records`` is a list of (kind, ms) per library launch."""
-    KINDS = {0: "attn", 1: "topk", 2: "combine", 3: "build_bits", 4: "export"}
+    KINDS = {0: "attn", 1: "topk", 2: "combine", 3: "build_bits", 4: "export",
+             5: "topk+combine"}
 
     def __init__(self, max_launches=4096):
         self.max_launches = int(max_launches)
