@@ -63,12 +63,43 @@ constexpr int kPairsPerBatch = 32 / kLanesPerPair;
 constexpr float kLazyLog2 = 8.f;        // rescale when a probability would exceed 2^8
 constexpr uint8_t kNoHead = 0xff;
 
+#ifndef LYCHEE_ATTN_ILP
+#define LYCHEE_ATTN_ILP 2   // batches of pairs a consumer warp works on at once
+#endif
+// Batches in flight per consumer warp for element type T and head dim D: rows
+// of 512 bytes (fp32, d = 128) keep one (twice the registers per chunk).
+template <typename T, int D>
+constexpr int ilp_of() {
+  return D * (int)sizeof(T) > 256 ? 1 : LYCHEE_ATTN_ILP;
+}
+
+// Register split between the warpgroups (setmaxnreg): the producer warpgroup
+// gives registers back, the consumer warpgroups take them.  The block launches
+// with 128 registers per thread (checked on the host before the launch):
+// 4 * 32 * kProdRegs + NW * 32 * kConsRegs must not exceed 512 * 128.
+#ifndef LYCHEE_ATTN_REGSPLIT
+#define LYCHEE_ATTN_REGSPLIT 1
+#endif
+#ifndef LYCHEE_ATTN_PROD_REGS
+#define LYCHEE_ATTN_PROD_REGS 80
+#endif
+#ifndef LYCHEE_ATTN_CONS_REGS
+#define LYCHEE_ATTN_CONS_REGS 136
+#endif
+constexpr int kProdRegs = LYCHEE_ATTN_PROD_REGS;
+constexpr int kConsRegs = LYCHEE_ATTN_CONS_REGS;
+
 // Sparse tiles take two copy paths at once: the first LYCHEE_ATTN_TMA_ROWS/16 of
 // a tile's rows as TMA tile::gather4 copies issued by the first streaming warp,
 // the rest as 16-byte cp.async by the other streaming warps (each path alone
 // caps below HBM bandwidth).  0: cp.async only.
 #ifndef LYCHEE_ATTN_TMA_ROWS
 #define LYCHEE_ATTN_TMA_ROWS 8
+#endif
+// 1: the TMA part of a sparse tile goes as 1-D bulk copies of runs of
+// consecutive positions instead of tile::gather4 copies
+#ifndef LYCHEE_ATTN_RUNS
+#define LYCHEE_ATTN_RUNS 0
 #endif
 
 template <typename T>
@@ -277,6 +308,14 @@ __global__ void __launch_bounds__((NW + NP) * 32, 1)
   }
   __syncthreads();
 
+  constexpr int ILP = ilp_of<T, D>();
+  if constexpr (ILP > 1 && LYCHEE_ATTN_REGSPLIT) {
+    static_assert(NW % 4 == 0 && NP == 4, "whole warpgroups: NW consumers, 4 producers");
+    static_assert(4 * 32 * kProdRegs + NW * 32 * kConsRegs <= (NW + NP) * 32 * 128,
+                  "register split within the launch's registers");
+    if (warp >= NW) asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kProdRegs));
+    else asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kConsRegs));
+  }
   if (warp == NW + 1) {
     // ------------------------------------------------------------ builder
     const int n_items = compact ? cum[B] * Hkv : p.n_items;
@@ -366,13 +405,22 @@ __global__ void __launch_bounds__((NW + NP) * 32, 1)
               lpos[o++] = p0 + 32 * lane + j;
             }
           }
-          // each sparse head's rows as union indices, in order: one word at a
-          // time, lane j placing bit j of the word; then, per tile, where the
-          // tile starts in the list (a retrieval head takes every row: no list)
+          // each sparse head's rows as union indices, in order (lane w places
+          // the rows of word w), and where each tile starts in that list: a
+          // tile boundary (a multiple of TT > 32 union rows) falls inside at
+          // most one word, whose lane writes the start (a retrieval head takes
+          // every row: no list)
           uint16_t* hrow = reinterpret_cast<uint16_t*>(ib + C::IB_HROW);
           uint16_t* tst = reinterpret_cast<uint16_t*>(ib + C::IB_TST);
-          const uint32_t lt = (1u << lane) - 1u;
           const int ntile = (total + TT - 1) / TT;
+          const int tb = (ubase + TT - 1) / TT;         // first tile starting at or after ubase
+          const bool has_bound = tb * TT < ubase + cnt;  // ... and inside this word
+          int bpos = 0;                                  // position of that boundary row
+          if (has_bound) {
+            uint32_t u = uni;
+            for (int r2 = tb * TT - ubase; r2 > 0; --r2) u &= u - 1;
+            bpos = __ffs(u) - 1;
+          }
           int work[G];
 #pragma unroll
           for (int t = 0; t < G; ++t) {
@@ -386,24 +434,19 @@ __global__ void __launch_bounds__((NW + NP) * 32, 1)
             work[t] = __shfl_sync(kFull, ic, 31);
             if ((rmask >> t) & 1u) continue;
             uint16_t* hl = hrow + t * kChunk;
-            const int hpre = ic - ct;
-#pragma unroll 6
-            for (int w = 0; w < nwords; ++w) {
-              const uint32_t bw = __shfl_sync(kFull, bits[t], w);
-              const uint32_t uw = __shfl_sync(kFull, uni, w);
-              const int hp = __shfl_sync(kFull, hpre, w);
-              const int ubw = __shfl_sync(kFull, ubase, w);
-              if ((bw >> lane) & 1u) hl[hp + __popc(bw & lt)] = (uint16_t)(ubw + __popc(uw & lt));
+            int k = ic - ct;
+            uint32_t u = bits[t];
+            while (u) {
+              const int j = __ffs(u) - 1;
+              u &= u - 1;
+              hl[k++] = (uint16_t)(ubase + __popc(uni & ((1u << j) - 1u)));
             }
-            __syncwarp();
-            const int bound = lane * TT;
-            int lo = 0, hi = work[t];
-            while (lo < hi) {
-              const int mid = (lo + hi) >> 1;
-              if ((int)hl[mid] < bound) lo = mid + 1;
-              else hi = mid;
+            uint16_t* ts = tst + t * 32;
+            if (has_bound) ts[tb] = (uint16_t)(ic - ct + __popc(bits[t] & ((1u << bpos) - 1u)));
+            if (lane == 0) {
+              ts[0] = 0;
+              ts[ntile] = (uint16_t)work[t];
             }
-            if (lane <= ntile) tst[t * 32 + lane] = (uint16_t)lo;
           }
           if (lane == 0) assign_warps<G, NW>(work, asg, asg + NW);
           __syncwarp();
@@ -499,7 +542,8 @@ __global__ void __launch_bounds__((NW + NP) * 32, 1)
         if (lane == 0 && sw == 0) {
           const uint32_t bytes = ((flags & kDense) ? 2u * (uint32_t)nrows * ROWB : 0u) +
                                  ((flags & kFirst) ? (uint32_t)C::kQBytes : 0u) +
-                                 2u * (uint32_t)ngrp * 4u * ROWB;
+                                 (LYCHEE_ATTN_RUNS ? 2u * (uint32_t)nt * ROWB
+                                                   : 2u * (uint32_t)ngrp * 4u * ROWB);
           fence_proxy_async_smem();
           if (bytes) mbar_arrive_expect_tx(&full[s], bytes);
           else mbar_arrive(&full[s]);
@@ -514,7 +558,24 @@ __global__ void __launch_bounds__((NW + NP) * 32, 1)
             bulk_g2s(vd, vbase + off, (uint32_t)nrows * ROWB, &full[s], pol);
           }
         }
-        if (ngrp > 0 && sw == 0) {
+        if (LYCHEE_ATTN_RUNS && nt > 0 && sw == 0) {
+          // rows [0, nt) as runs of consecutive positions, one bulk copy of K
+          // and one of V per run (rows of a run are adjacent in the tile too)
+          for (int i0 = 0; i0 < nt; i0 += 32) {
+            const int i = i0 + lane;
+            if (i < nt) {
+              const int pos = lpos[t0 + i];
+              if (i == 0 || lpos[t0 + i - 1] != pos - 1) {
+                int len = 1;
+                while (i + len < nt && lpos[t0 + i + len] == pos + len) ++len;
+                const size_t off = (size_t)pos * D;
+                bulk_g2s(kd + i * ROWB, kbase + off, (uint32_t)len * ROWB, &full[s], pol);
+                bulk_g2s(vd + i * ROWB, vbase + off, (uint32_t)len * ROWB, &full[s], pol);
+              }
+            }
+          }
+        }
+        if (!LYCHEE_ATTN_RUNS && ngrp > 0 && sw == 0) {
           // four rows per copy; a padded group repeats the range's last row
           const int last = lpos[t0 + nt - 1];
           for (int gi = lane; gi < ngrp; gi += 32) {
@@ -557,6 +618,7 @@ __device__ __forceinline__ void consumer_loop(const AttnParams& p, unsigned char
                                               uint64_t* full, uint64_t* empty, uint64_t* freeb) {
   using C = AttnCfg<T, D, G, NW, NP, TT, STAGES>;
   constexpr int E = C::E, DL = C::DL, CPL = C::CPL, ROWB = C::ROWB;
+  constexpr int ILP = ilp_of<T, D>();
   const int4* info = reinterpret_cast<const int4*>(smem + C::OFF_INFO);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int r = lane / kLanesPerPair, pp = lane % kLanesPerPair;   // pair slot, quarter
@@ -637,43 +699,66 @@ __device__ __forceinline__ void consumer_loop(const AttnParams& p, unsigned char
       // moves from slot to slot so that no warp of the head always gets the most
       int k = slot - tt % nh;
       if (k < 0) k += nh;
-      for (; k < nb; k += nh) {
-        const int idx = k * kPairsPerBatch + r;
-        const bool valid = idx < cnt;
-        const int row = valid ? (ident ? idx : (int)hl[st0 + idx] - t0) : 0;
-        // ---- the pair's K and V chunks (V is fetched now so that its load is
-        // off the softmax's critical path; row 0 always holds real data, and
-        // a pair that is not taken gets weight 0)
-        const unsigned char* kr = kt + row * ROWB;
-        const unsigned char* vr = vt + row * ROWB;
-        uint4 kraw[CPL], vraw[CPL];
+      // NBAT batches per iteration (k, k + nh, ...) so that their dependency
+      // chains overlap; batches past the last are empty (no pair taken).  A
+      // retrieval head fills whole tiles, so its warps take ILP batches at
+      // once; a sparse head's warps get about two batches per tile, so one.
+      auto run = [&](auto nbat_tag) {
+      constexpr int NBAT = decltype(nbat_tag)::value;
+      for (; k < nb; k += NBAT * nh) {
+        int rowu[NBAT];
+        bool validu[NBAT];
+        uint4 raw[NBAT][CPL];
+        float svu[NBAT];
+        // ---- rows and K chunks
 #pragma unroll
-        for (int cc = 0; cc < CPL; ++cc) {
-          kraw[cc] = *reinterpret_cast<const uint4*>(kr + coff[cc]);
-          vraw[cc] = *reinterpret_cast<const uint4*>(vr + coff[cc]);
+        for (int u = 0; u < NBAT; ++u) {
+          const int idx = (k + u * nh) * kPairsPerBatch + r;
+          validu[u] = idx < cnt;
+          rowu[u] = validu[u] ? (ident ? idx : (int)hl[st0 + idx] - t0) : 0;
+#pragma unroll
+          for (int cc = 0; cc < CPL; ++cc)
+            raw[u][cc] = *reinterpret_cast<const uint4*>(kt + rowu[u] * ROWB + coff[cc]);
         }
         // ---- q.K over the lane's quarter: CPL independent partial sums
-        float2 part[CPL];
 #pragma unroll
-        for (int cc = 0; cc < CPL; ++cc) {
-          float2 kx[E / 2];
-          Vec<T>::widen(kraw[cc], kx);
-          part[cc] = __fmul2_rn(qr[cc][0], kx[0]);
+        for (int u = 0; u < NBAT; ++u) {
+          float2 part[CPL];
 #pragma unroll
-          for (int e = 1; e < E / 2; ++e) part[cc] = __ffma2_rn(qr[cc][e], kx[e], part[cc]);
+          for (int cc = 0; cc < CPL; ++cc) {
+            float2 kx[E / 2];
+            Vec<T>::widen(raw[u][cc], kx);
+            part[cc] = __fmul2_rn(qr[cc][0], kx[0]);
+#pragma unroll
+            for (int e = 1; e < E / 2; ++e) part[cc] = __ffma2_rn(qr[cc][e], kx[e], part[cc]);
+          }
+#pragma unroll
+          for (int w2 = 1; w2 < CPL; w2 <<= 1)
+#pragma unroll
+            for (int cc = 0; cc + w2 < CPL; cc += 2 * w2)
+              part[cc] = __fadd2_rn(part[cc], part[cc + w2]);
+          svu[u] = part[0].x + part[0].y;
         }
+        // ---- V chunks of the same rows (row 0 always holds real data; a pair
+        // that is not taken gets weight 0), loaded while the scores finish
 #pragma unroll
-        for (int w2 = 1; w2 < CPL; w2 <<= 1)
+        for (int u = 0; u < NBAT; ++u)
 #pragma unroll
-          for (int cc = 0; cc + w2 < CPL; cc += 2 * w2) part[cc] = __fadd2_rn(part[cc], part[cc + w2]);
-        float dot = part[0].x + part[0].y;
-        dot += __shfl_xor_sync(kFull, dot, 1);
-        dot += __shfl_xor_sync(kFull, dot, 2);
-        if (lg_on && valid) lg[t0 + row] = dot;
-        const float sv = valid ? dot : -INFINITY;
+          for (int cc = 0; cc < CPL; ++cc)
+            raw[u][cc] = *reinterpret_cast<const uint4*>(vt + rowu[u] * ROWB + coff[cc]);
+        float mx = -INFINITY;
+#pragma unroll
+        for (int u = 0; u < NBAT; ++u) {
+          float dot = svu[u];
+          dot += __shfl_xor_sync(kFull, dot, 1);
+          dot += __shfl_xor_sync(kFull, dot, 2);
+          if (lg_on && validu[u]) lg[t0 + rowu[u]] = dot;
+          svu[u] = validu[u] ? dot : -INFINITY;
+          mx = fmaxf(mx, svu[u]);
+        }
         // ---- online softmax with a lazy maximum (warp-uniform branch)
-        if (__any_sync(kFull, sv > mth)) {
-          const float mn = sv > mth ? sv : m;
+        if (__any_sync(kFull, mx > mth)) {
+          const float mn = mx > mth ? mx : m;
           const float al = (mn == m) ? 1.f : fast_exp2((m - mn) * sl);   // 0 while m is -inf
           const float2 a2 = make_float2(al, al);
 #pragma unroll
@@ -685,18 +770,24 @@ __device__ __forceinline__ void consumer_loop(const AttnParams& p, unsigned char
           mth = (m == -INFINITY) ? -INFINITY : m + lazy;
           msl = (m == -INFINITY) ? 0.f : m * sl;
         }
-        const float pr = fast_exp2(fmaf(sv, sl, -msl));   // 0 for rows not taken
-        l += pr;
-        // ---- P.V on the same row and quarter
-        const float2 p2 = make_float2(pr, pr);
+        // ---- P.V on the same rows and quarter
 #pragma unroll
-        for (int cc = 0; cc < CPL; ++cc) {
-          float2 vx[E / 2];
-          Vec<T>::widen(vraw[cc], vx);
+        for (int u = 0; u < NBAT; ++u) {
+          const float pr = fast_exp2(fmaf(svu[u], sl, -msl));   // 0 for rows not taken
+          l += pr;
+          const float2 p2 = make_float2(pr, pr);
 #pragma unroll
-          for (int e = 0; e < E / 2; ++e) acc[cc][e] = __ffma2_rn(p2, vx[e], acc[cc][e]);
+          for (int cc = 0; cc < CPL; ++cc) {
+            float2 vx[E / 2];
+            Vec<T>::widen(raw[u][cc], vx);
+#pragma unroll
+            for (int e = 0; e < E / 2; ++e) acc[cc][e] = __ffma2_rn(p2, vx[e], acc[cc][e]);
+          }
         }
       }
+      };
+      if (ident) run(std::integral_constant<int, ILP>{});
+      else run(std::integral_constant<int, 1>{});
     }
     __syncwarp();
     if (lane == 0) mbar_arrive(&empty[s]);
@@ -770,6 +861,13 @@ cudaError_t launch_attn_t(const AttnParams& p, int num_sms, cudaStream_t st) {
     cudaError_t e =
         cudaFuncSetAttribute(kfn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)C::SMEM);
     if (e != cudaSuccess) return e;
+    if (ilp_of<T, D>() > 1 && LYCHEE_ATTN_REGSPLIT) {
+      // the register split assumes 128 registers per thread at launch
+      cudaFuncAttributes fa{};
+      e = cudaFuncGetAttributes(&fa, kfn);
+      if (e != cudaSuccess) return e;
+      if (fa.numRegs != 128) return cudaErrorInvalidConfiguration;
+    }
     attr_set = true;
   }
   const int grid = max(1, min(num_sms, p.n_items));
