@@ -274,6 +274,8 @@ __global__ void __launch_bounds__((NW + NP) * 32, 1)
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int Hq = p.Hq, Hkv = p.Hkv, N_max = p.N_max, B = p.B;
   const bool compact = B <= kMaxBatchCompact;
+  pdl_launch_dependents();
+  pdl_wait();
   // the combine kernel that follows counts its finished CTAs from zero
   for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < B * Hq; i += gridDim.x * blockDim.x)
     p.ccnt[i] = 0u;
@@ -871,7 +873,8 @@ cudaError_t launch_attn_t(const AttnParams& p, int num_sms, cudaStream_t st) {
     attr_set = true;
   }
   const int grid = max(1, min(num_sms, p.n_items));
-  kfn<<<grid, C::NT, C::SMEM, st>>>(p);
+  const cudaError_t e = launch_pdl(kfn, dim3(grid), dim3(C::NT), (size_t)C::SMEM, st, p);
+  if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
 

@@ -25,13 +25,17 @@ namespace {
 template <typename T, int D>
 __global__ void __launch_bounds__(kCombThreads) combine_kernel(const __grid_constant__ CombineParams p) {
   extern __shared__ __align__(16) unsigned char csm[];
+  pdl_launch_dependents();
+  pdl_wait();
   combine_body<T, D>(p, blockIdx.x, csm);
 }
 
 template <typename T, int D>
 cudaError_t launch_combine_t(const CombineParams& p, cudaStream_t st) {
   const unsigned grid = (unsigned)(p.B * p.Hq * kCombineSplit);
-  combine_kernel<T, D><<<grid, kCombThreads, combine_smem_bytes<D>(), st>>>(p);
+  const cudaError_t e =
+      launch_pdl(combine_kernel<T, D>, dim3(grid), dim3(kCombThreads), combine_smem_bytes<D>(), st, p);
+  if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
 

@@ -161,6 +161,17 @@ __device__ __forceinline__ void tma_gather4(void* dst, const void* tmap, int x, 
       : "memory");
 }
 
+// ---- programmatic dependent launch -------------------------------------------------
+// Every kernel of the library lets the next kernel of its stream start launching
+// at once (its CTAs become resident as SMs free up) and, before touching any
+// memory, waits until the previous kernel of the stream has completed and its
+// writes are visible.  With the launch attribute below this hides the launch
+// gap between dependent kernels; without it both are no-ops.
+__device__ __forceinline__ void pdl_launch_dependents() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
 // ---- named barriers (a subset of the CTA's warps) ------------------------------
 __device__ __forceinline__ void named_bar_sync(uint32_t id, uint32_t nthreads) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
@@ -213,6 +224,23 @@ __device__ __forceinline__ uint32_t float_to_key(float f) {
 // bf16x2 in one 32-bit word -> two fp32 (exact widening).
 __device__ __forceinline__ float2 bf16x2_to_float2(uint32_t w) {
   return make_float2(__uint_as_float(w << 16), __uint_as_float(w & 0xffff0000u));
+}
+
+// Launch with programmatic stream serialization (see pdl_wait above).
+template <typename... KArgs, typename... Args>
+inline cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                              cudaStream_t st, Args... args) {
+  cudaLaunchConfig_t cfg{};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute at[1];
+  at[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  at[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = at;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, args...);
 }
 
 }  // namespace lychee

@@ -24,6 +24,8 @@ constexpr int kEntriesPerCta = 4 * kThreads;   // set entries one build_bits CTA
 // predecessor sets kErrBadIndex; the row is then not a set and its bitmap is
 // unspecified, but every store still stays inside the row.
 __global__ void __launch_bounds__(kThreads) build_bits_kernel(const __grid_constant__ BuildBitsParams p) {
+  pdl_launch_dependents();
+  pdl_wait();
   const int b = blockIdx.y / p.nheads, h = p.heads[blockIdx.y % p.nheads];
   const int n = min(max(p.seqlens[b], 1), p.N_max);
   int kb = p.k_per_seq ? p.k_per_seq[b] : p.k;
@@ -64,6 +66,8 @@ __global__ void __launch_bounds__(kThreads) build_bits_kernel(const __grid_const
 
 // Bitmaps -> index rows for every head: ascending positions, -1 padded to k.
 __global__ void __launch_bounds__(kThreads) export_kernel(const __grid_constant__ ExportParams p) {
+  pdl_launch_dependents();
+  pdl_wait();
   __shared__ uint32_t wsum[kThreads / 32];
   const int bh = blockIdx.x, b = bh / p.Hq;
   const int n = min(max(p.seqlens[b], 1), p.N_max);
@@ -107,12 +111,15 @@ __global__ void __launch_bounds__(kThreads) export_kernel(const __grid_constant_
 cudaError_t launch_build_bits(const BuildBitsParams& p, cudaStream_t st) {
   if (p.nheads <= 0) return cudaSuccess;
   const dim3 grid((unsigned)((p.k + kEntriesPerCta - 1) / kEntriesPerCta), (unsigned)(p.B * p.nheads));
-  build_bits_kernel<<<grid, kThreads, 0, st>>>(p);
+  const cudaError_t e = launch_pdl(build_bits_kernel, grid, dim3(kThreads), 0, st, p);
+  if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
 
 cudaError_t launch_export(const ExportParams& p, cudaStream_t st) {
-  export_kernel<<<(unsigned)(p.B * p.Hq), kThreads, 0, st>>>(p);
+  const cudaError_t e =
+      launch_pdl(export_kernel, dim3((unsigned)(p.B * p.Hq)), dim3(kThreads), 0, st, p);
+  if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
 

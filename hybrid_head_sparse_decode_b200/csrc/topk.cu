@@ -231,6 +231,8 @@ template <int C>
 __global__ void __launch_bounds__(kThreads, 1)
     topk_kernel(const __grid_constant__ TopkParams p, int keys_cap, int wpc_cap) {
   extern __shared__ __align__(16) uint32_t dsm[];
+  pdl_launch_dependents();
+  pdl_wait();
   topk_body<C>(p, keys_cap, wpc_cap, blockIdx.x, dsm);
 }
 
@@ -244,6 +246,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     topk_combine_kernel(const __grid_constant__ TopkParams p, const __grid_constant__ CombineParams cp,
                         int keys_cap, int wpc_cap, int ntopk, int ncomb) {
   extern __shared__ __align__(16) uint32_t dsm[];
+  pdl_launch_dependents();
+  pdl_wait();
   const int cta = blockIdx.x;
   if (cta < ntopk) topk_body<C>(p, keys_cap, wpc_cap, cta, dsm);
   else if (cta - ntopk < ncomb) combine_body<T, D>(cp, cta - ntopk, reinterpret_cast<unsigned char*>(dsm));
@@ -278,8 +282,10 @@ void fill_config(cudaLaunchConfig_t& cfg, cudaLaunchAttribute* at, unsigned grid
   at[0].val.clusterDim.x = C;
   at[0].val.clusterDim.y = 1;
   at[0].val.clusterDim.z = 1;
+  at[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  at[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = at;
-  cfg.numAttrs = 1;
+  cfg.numAttrs = 2;
 }
 
 template <int C>
@@ -301,7 +307,7 @@ cudaError_t launch_c(const TopkParams& p, cudaStream_t st) {
   cudaError_t e = set_attributes<C>();
   if (e != cudaSuccess) return e;
   cudaLaunchConfig_t cfg;
-  cudaLaunchAttribute at[1];
+  cudaLaunchAttribute at[2];
   fill_config<C>(cfg, at, (unsigned)(C * p.B * p.nheads), g.smem, st);
   e = cudaLaunchKernelEx(&cfg, topk_kernel<C>, p, g.keys_cap, g.wpc_cap);
   if (e != cudaSuccess) return e;
@@ -318,8 +324,9 @@ bool cluster16_ok(int N_max, cudaStream_t st) {
   bool ok = g.ok && set_attributes<16>() == cudaSuccess;
   if (ok) {
     cudaLaunchConfig_t cfg;
-    cudaLaunchAttribute at[1];
+    cudaLaunchAttribute at[2];
     fill_config<16>(cfg, at, 16u, g.smem, st);
+    cfg.numAttrs = 1;   // the occupancy query needs only the cluster shape
     int nclusters = 0;
     ok = cudaOccupancyMaxActiveClusters(&nclusters, topk_kernel<16>, &cfg) == cudaSuccess &&
          nclusters >= 1;
@@ -348,7 +355,7 @@ cudaError_t launch_tc(const TopkParams& p, const CombineParams& cp, cudaStream_t
   const int grid = (ntopk + ncomb + C - 1) / C * C;
   const size_t smem = std::max(g.smem, combine_smem_bytes<D>());
   cudaLaunchConfig_t cfg;
-  cudaLaunchAttribute at[1];
+  cudaLaunchAttribute at[2];
   fill_config<C>(cfg, at, (unsigned)grid, smem, st);
   cudaError_t e = cudaLaunchKernelEx(&cfg, kfn, p, cp, g.keys_cap, g.wpc_cap, ntopk, ncomb);
   if (e != cudaSuccess) return e;
