@@ -4,6 +4,7 @@
 #include <cudaTypedefs.h>
 
 #include <cmath>
+#include <cstdlib>
 #include <cstdint>
 #include <cstring>
 #include <mutex>
@@ -116,6 +117,17 @@ PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
     cudaGetLastError();
   });
   return fn;
+}
+
+// LYCHEE_NO_TMA_GATHER=1 in the environment (read once) makes every sparse row
+// gather use 16-byte copies, the path taken when no tensor map can describe the
+// cache; for testing that path.
+bool tma_gathers_disabled() {
+  static const bool off = [] {
+    const char* v = std::getenv("LYCHEE_NO_TMA_GATHER");
+    return v && v[0] == '1';
+  }();
+  return off;
 }
 
 // The cache [B, Hkv, N_max, d] as rows of d elements, box one row high and one
@@ -241,7 +253,8 @@ lychee_status run_layer(const Ctx& c, const void* q, const void* kc, const void*
   ap.n_items = s->B * s->Hkv * c.L.nchunk;
   ap.scale_log2 = (float)(1.4426950408889634 / std::sqrt((double)s->d));
   fill_roles(ap.role, role, Hq);
-  ap.gather_tma = (encode_row_map(&ap.tmk, kc, s) && encode_row_map(&ap.tmv, vc, s)) ? 1 : 0;
+  ap.gather_tma = !tma_gathers_disabled() && encode_row_map(&ap.tmk, kc, s) &&
+                   encode_row_map(&ap.tmv, vc, s) ? 1 : 0;
   e = timed(kKindAttn, c.st, [&] { return launch_attn(ap, s->dtype, s->d, G, c.sms, c.st); });
   if (e != cudaSuccess) return LYCHEE_ERR_CUDA;
   // top-k of the retrieval heads and the combine of every head: independent

@@ -643,6 +643,7 @@ __device__ __forceinline__ void consumer_loop(const AttnParams& p, unsigned char
   float2 acc[CPL][E / 2];
   float m = -INFINITY, mth = -INFINITY, msl = 0.f, l = 0.f;
   int myh = -1, slot = 0, nh = 1, buf = 0;
+  int kfirst = 0;                          // first batch of this tile for the warp
 
   bool ident = false, lg_on = false;
   float* lg = nullptr;
@@ -665,6 +666,7 @@ __device__ __forceinline__ void consumer_loop(const AttnParams& p, unsigned char
       const uint8_t a = ib[C::IB_ASG + warp];
       myh = a == kNoHead ? -1 : (a & 15);
       slot = a >> 4;
+      kfirst = slot;
       if (myh >= 0) {
         nh = ib[C::IB_ASG + NW + myh];
         ident = (i1.y >> myh) & 1;
@@ -699,8 +701,8 @@ __device__ __forceinline__ void consumer_loop(const AttnParams& p, unsigned char
       const unsigned char* vt = smem + C::OFF_V + s * C::kStageKV;
       // batch k is served by slot (k + tt) % nh: the first batch of a tile
       // moves from slot to slot so that no warp of the head always gets the most
-      int k = slot - tt % nh;
-      if (k < 0) k += nh;
+      int k = kfirst;
+      kfirst = kfirst == 0 ? nh - 1 : kfirst - 1;
       // NBAT batches per iteration (k, k + nh, ...) so that their dependency
       // chains overlap; batches past the last are empty (no pair taken).  A
       // retrieval head fills whole tiles, so its warps take ILP batches at

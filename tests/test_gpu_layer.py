@@ -180,3 +180,20 @@ def test_graph_capture_replays_identically():
     g.replay()
     torch.cuda.synchronize()
     assert torch.equal(out, ref_o) and torch.equal(io, ref_i)
+
+
+def test_sparse_row_copies_without_tensor_maps():
+    """The 16-byte-copy gather path (taken when no tensor map can describe the
+    cache) gives the same parity results: rerun a set of layer cases in a fresh
+    process with the row gathers forced onto that path."""
+    import os
+    import subprocess
+    import sys
+    here = os.path.dirname(os.path.abspath(__file__))
+    env = dict(os.environ, LYCHEE_NO_TMA_GATHER="1")
+    cmd = [sys.executable, "-m", "pytest", "-x", "-q", "-m", "gpu", "-p", "no:cacheprovider",
+           os.path.join(here, "test_gpu_layer.py") + "::test_random_shapes",
+           os.path.join(here, "test_gpu_layer.py") + "::test_qwen3_layer_32k_full_size",
+           os.path.join(here, "test_gpu_layer.py") + "::test_deterministic_bitwise"]
+    r = subprocess.run(cmd, env=env, capture_output=True, text=True, timeout=900)
+    assert r.returncode == 0, r.stdout[-3000:] + r.stderr[-3000:]
