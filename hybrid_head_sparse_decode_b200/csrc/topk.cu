@@ -28,49 +28,103 @@ namespace {
 constexpr uint32_t kFull = 0xffffffffu;
 constexpr int kThreads = 512;
 constexpr int kWarps = kThreads / 32;
+constexpr int kPasses = 4;                 // 8-bit digits of a 32-bit key
+constexpr int kHists = kWarps / 2;         // CTA-local histograms, one per pair of warps
 constexpr size_t kSmemBudget = 200 * 1024;
 
-// Exclusive scan of one value per thread over the CTA; *total gets the sum.
-__device__ __forceinline__ uint32_t block_exclusive_scan(uint32_t v, uint32_t* wsum,
-                                                         uint32_t* total) {
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  uint32_t x = v;
+// Dynamic shared memory of one selection CTA, in 32-bit words from its start:
+//   bar   [kPasses] mbarriers (one per radix pass; 2 words each)
+//   recv  [kPasses][C][256]  every CTA's digit histogram of each pass
+//   whist [kHists][256]      this CTA's histograms, one per pair of warps
+//   misc  [kMisc]            scan totals, the chosen digit, per-rank/per-warp counts
+//   keys  [keys_cap]         this CTA's logits as order-preserving keys (16-byte
+//                            aligned: written four at a time)
+//   wa,wb [wpc_cap]          per word: keys equal to T, keys above T (bits)
+constexpr int kMisc = 128;
+enum : int { kMiscWtot = 0, kMiscBc = 8, kMiscRankGt = 16, kMiscRankEq = 32, kMiscWarpGt = 48,
+             kMiscWarpEq = 64 };
+template <int C>
+struct TopkSmem {
+  static constexpr int kBar = 0;
+  static constexpr int kRecv = 2 * kPasses;
+  static constexpr int kWhist = kRecv + kPasses * C * 256;
+  static constexpr int kMiscOff = kWhist + kHists * 256;
+  static constexpr int kKeys = kMiscOff + kMisc;
+  static_assert(kRecv % 4 == 0 && kKeys % 4 == 0, "16-byte aligned histogram rows and keys");
+  static size_t bytes(int wpc_cap, int keys_cap) {
+    return (size_t)(kKeys + keys_cap + 2 * wpc_cap) * 4;
+  }
+};
+
+__device__ __forceinline__ uint32_t warp_sum(uint32_t v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(kFull, v, o);
+  return v;
+}
+__device__ __forceinline__ uint32_t warp_inclusive_scan(uint32_t v, int lane) {
 #pragma unroll
   for (int o = 1; o < 32; o <<= 1) {
-    const uint32_t y = __shfl_up_sync(kFull, x, o);
-    if (lane >= o) x += y;
+    const uint32_t y = __shfl_up_sync(kFull, v, o);
+    if (lane >= o) v += y;
   }
-  if (lane == 31) wsum[warp] = x;
-  __syncthreads();
-  if (warp == 0) {
-    uint32_t t = lane < kWarps ? wsum[lane] : 0u;
+  return v;
+}
+
+// The lowest `a` set bits of x (a <= popc(x)).
+__device__ __forceinline__ uint32_t lowest_set_bits(uint32_t x, uint32_t a) {
+  uint32_t keep = 0;
+  for (uint32_t i = 0; i < a; ++i) {
+    const uint32_t b = x & (0u - x);
+    keep |= b;
+    x ^= b;
+  }
+  return keep;
+}
+
+// Entries t < m of per-lane counts (gt_t: keys above T, eq_t: keys equal to T),
+// in order after `eq0` keys equal to T already seen: the keys they select
+// (every key above T, plus keys equal to T while fewer than kties were taken
+// before them) and the keys equal to T among them.  Lanes >= n hold zeros.
+__device__ __forceinline__ void prefix_take(uint32_t gt, uint32_t eq, int m, uint32_t eq0,
+                                            uint32_t kties, int lane, uint32_t& sel, uint32_t& eqs) {
+  const uint32_t run = eq0 + warp_inclusive_scan(eq, lane) - eq;
+  const uint32_t take = kties > run ? min(eq, kties - run) : 0u;
+  sel = warp_sum(lane < m ? gt + take : 0u);
+  eqs = warp_sum(lane < m ? eq : 0u);
+}
+
+// Before the previous kernel's results are needed: set up the per-pass
+// barriers (each expects one histogram from every CTA of the cluster), clear
+// the warp histograms and announce this to the cluster.
+template <int C>
+__device__ __forceinline__ void topk_prologue(uint32_t* dsm) {
+  using L = TopkSmem<C>;
+  uint64_t* bar = reinterpret_cast<uint64_t*>(dsm + L::kBar);
+  if (threadIdx.x == 0) {
 #pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      const uint32_t y = __shfl_up_sync(kFull, t, o);
-      if (lane >= o) t += y;
-    }
-    wsum[lane] = t;
+    for (int ps = 0; ps < kPasses; ++ps) mbar_init(&bar[ps], 1);
+    fence_mbar_init();
+#pragma unroll
+    for (int ps = 0; ps < kPasses; ++ps) mbar_arrive_expect_tx(&bar[ps], C * 256 * 4);
   }
-  __syncthreads();
-  const uint32_t before = warp > 0 ? wsum[warp - 1] : 0u;
-  *total = wsum[kWarps - 1];
-  __syncthreads();
-  return before + x - v;
+  for (int i = threadIdx.x; i < kHists * 256; i += kThreads) dsm[L::kWhist + i] = 0u;
+  cluster_arrive_relaxed();
 }
 
 // One CTA of the selection: CTA `cta` of cluster cta / C (its rank in the
-// cluster is the hardware rank), dynamic shared memory at dsm.
+// cluster is the hardware rank), dynamic shared memory at dsm, after
+// topk_prologue.
 template <int C>
 __device__ __forceinline__ void topk_body(const TopkParams& p, int keys_cap, int wpc_cap, int cta,
                                           uint32_t* dsm) {
-  uint32_t* keys = dsm;                    // [keys_cap]
-  uint32_t* wa = keys + keys_cap;          // [wpc_cap] tie bits, then selected bits
-  uint32_t* wb = wa + wpc_cap;             // [wpc_cap] greater bits, then output offsets
-  uint32_t* whist = wb + wpc_cap;          // [kWarps][256] warp-private histograms
-  __shared__ uint32_t hist[2][256];        // CTA histograms, read by the cluster
-  __shared__ uint32_t wsum[32];
-  __shared__ uint32_t cta_tot[2];
-  __shared__ uint32_t bc[4];
+  using L = TopkSmem<C>;
+  uint64_t* bar = reinterpret_cast<uint64_t*>(dsm + L::kBar);
+  uint32_t* recv = dsm + L::kRecv;
+  uint32_t* whist = dsm + L::kWhist;
+  uint32_t* misc = dsm + L::kMiscOff;
+  uint32_t* keys = dsm + L::kKeys;
+  uint32_t* wa = keys + keys_cap;
+  uint32_t* wb = wa + wpc_cap;
 
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const uint32_t rank = cluster_ctarank();
@@ -103,135 +157,179 @@ __device__ __forceinline__ void topk_body(const TopkParams& p, int keys_cap, int
   auto key_at = [&](int i) -> uint32_t {
     return i < keys_cap ? keys[i] : float_to_key(__ldcg(row + i));
   };
-  uint32_t* myhist = whist + warp * 256;
+  uint32_t* myhist = whist + (warp >> 1) * 256;
+  const int ncache = min(npos, keys_cap);
+  cluster_wait();    // every CTA's barriers are set up: histograms may be sent
 
   // ---- radix select, 8-bit digits, most significant first
   uint32_t prefix = 0, pmask = 0;
   uint32_t krem = (uint32_t)kb;
+  // rank `warp`'s selected keys so far (warps < C; per-lane partial sums): keys
+  // whose digit beat the chosen one in some pass, plus (exact) the keys equal
+  // to T or (otherwise) the whole chosen bucket of the last pass
+  uint32_t rk_gt = 0, rk_eq = 0;
+  auto rank_counts = [&](int ps, bool last_pass, bool exact_last) {
+    if (warp < C) {
+      const uint32_t d = (prefix >> (24 - 8 * ps)) & 255u;
+      const uint32_t* hr = recv + (ps * C + warp) * 256;
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        const uint32_t bn = (uint32_t)(j * 32 + lane);
+        if (bn > d) rk_gt += hr[bn];
+      }
+      if (last_pass && lane == 0) {
+        if (exact_last) rk_eq += hr[d];
+        else rk_gt += hr[d];
+      }
+    }
+  };
   int pass = 0;
-  for (; pass < 4; ++pass) {
+  for (; pass < kPasses; ++pass) {
     const int shift = 24 - 8 * pass;
-    const int buf = pass & 1;
-    for (int i = lane; i < 256; i += 32) myhist[i] = 0u;
-    __syncwarp();
-    for (int i = tid; i < npos; i += kThreads) {
+#pragma unroll 4
+    for (int i = tid; i < ncache; i += kThreads) {
+      const uint32_t key = keys[i];
+      if ((key & pmask) == prefix) atomicAdd(&myhist[(key >> shift) & 255u], 1u);
+    }
+    for (int i = ncache + tid; i < npos; i += kThreads) {
       const uint32_t key = key_at(i);
       if ((key & pmask) == prefix) atomicAdd(&myhist[(key >> shift) & 255u], 1u);
     }
     __syncthreads();
+    uint32_t* rv = recv + pass * C * 256;
     if (tid < 256) {
+      // this CTA's count of bin tid (the histograms are cleared for the next
+      // pass as they are read), sent to slot `rank` of every CTA
       uint32_t s = 0;
 #pragma unroll
-      for (int w = 0; w < kWarps; ++w) s += whist[w * 256 + tid];
-      hist[buf][tid] = s;   // buffer last read in pass-2, before cluster barrier pass-1
+      for (int w = 0; w < kHists; ++w) {
+        s += whist[w * 256 + tid];
+        whist[w * 256 + tid] = 0u;
+      }
+      const int q = lane & ~3;
+      const uint4 v = make_uint4(__shfl_sync(kFull, s, q), __shfl_sync(kFull, s, q + 1),
+                                 __shfl_sync(kFull, s, q + 2), __shfl_sync(kFull, s, q + 3));
+      const uint32_t dst = smem_u32(rv + rank * 256 + (tid & ~3));
+      const uint32_t bl = smem_u32(&bar[pass]);
+      for (int r2 = lane & 3; r2 < C; r2 += 4) st_async_v4(dsmem_map(dst, r2), v, dsmem_map(bl, r2));
     }
-    cluster_sync();
+    if (pass > 0) rank_counts(pass - 1, false, false);   // while the histograms travel
+    mbar_wait_cluster(&bar[pass], 0u, p.err);   // all C histograms of this pass are here
     // cluster-wide histogram; bins enumerated from the top so that an inclusive
     // prefix sum at bin d counts the candidates whose digit is >= d
     const int bin = 255 - tid;
-    uint32_t tot = 0;
+    uint32_t tot = 0, incl = 0;
     if (tid < 256) {
 #pragma unroll
-      for (int r2 = 0; r2 < C; ++r2) tot += dsmem_ld_u32(dsmem_addr(&hist[buf][bin], r2));
-    }
-    uint32_t all;
-    const uint32_t above = block_exclusive_scan(tid < 256 ? tot : 0u, wsum, &all);
-    if (tid < 256 && above + tot >= krem && above < krem) {
-      bc[0] = (uint32_t)bin;
-      bc[1] = above;
-      bc[2] = tot;
+      for (int r2 = 0; r2 < C; ++r2) tot += rv[r2 * 256 + bin];
+      incl = warp_inclusive_scan(tot, lane);
+      if (lane == 31) misc[kMiscWtot + warp] = incl;
     }
     __syncthreads();
-    prefix |= bc[0] << shift;
+    if (tid < 256) {
+      uint32_t above = incl - tot;
+      for (int w = 0; w < warp; ++w) above += misc[kMiscWtot + w];
+      if (above < krem && above + tot >= krem) {
+        misc[kMiscBc + 0] = (uint32_t)bin;
+        misc[kMiscBc + 1] = above;
+        misc[kMiscBc + 2] = tot;
+      }
+    }
+    __syncthreads();
+    prefix |= (misc[kMiscBc + 0] & 255u) << shift;
     pmask |= 255u << shift;
-    krem -= bc[1];
-    const bool whole_bucket = bc[2] == krem;   // the same decision in every CTA
-    __syncthreads();
-    if (whole_bucket) break;
+    krem -= misc[kMiscBc + 1];
+    if (misc[kMiscBc + 2] == krem) break;   // the same decision in every CTA
   }
+  cluster_arrive_relaxed();  // no more histograms will arrive here (checked before exit)
   // exact: T is the k_b-th key and krem of the keys equal to T are taken;
   // otherwise every key whose top bits are >= the chosen prefix is taken
-  const bool exact = pass == 4;
+  const bool exact = pass == kPasses;
+  const int last = exact ? kPasses - 1 : pass;
   const uint32_t T = prefix;
-
-  // ---- compaction in position order
-  for (int wl = warp; wl < mywords; wl += kWarps) {
-    const int i = wl * 32 + lane;
+  const uint32_t kties = exact ? krem : 0u;
+  rank_counts(last, true, exact);
+  if (warp < C) {
+    const uint32_t g = warp_sum(rk_gt);
+    if (lane == 0) {
+      misc[kMiscRankGt + warp] = g;
+      misc[kMiscRankEq + warp] = rk_eq;
+    }
+  }
+  // ---- this CTA's words: per warp a contiguous run, bits of keys equal to /
+  // above T, and the warp's totals
+  const int wpw = (mywords + kWarps - 1) / kWarps;
+  const int j0 = min(mywords, warp * wpw), j1 = min(mywords, j0 + wpw);
+  uint32_t ceq = 0, cgt = 0;
+  for (int j = j0; j < j1; ++j) {
+    const int i = j * 32 + lane;
     const bool v = i < npos;
     const uint32_t key = v ? key_at(i) : 0u;
     const uint32_t eq = __ballot_sync(kFull, v && exact && key == T);
     const uint32_t gt = __ballot_sync(kFull, v && (exact ? key > T : (key & pmask) >= T));
     if (lane == 0) {
-      wa[wl] = eq;
-      wb[wl] = gt;
+      wa[j] = eq;
+      wb[j] = gt;
     }
+    ceq += __popc(eq);
+    cgt += __popc(gt);
+  }
+  if (lane == 0) {
+    misc[kMiscWarpGt + warp] = cgt;
+    misc[kMiscWarpEq + warp] = ceq;
   }
   __syncthreads();
-  const int wpt = (mywords + kThreads - 1) / kThreads;
-  const int ta = min(mywords, tid * wpt), tb = min(mywords, ta + wpt);
-  uint32_t ceq = 0, cgt = 0;
-  for (int w = ta; w < tb; ++w) {
-    ceq += __popc(wa[w]);
-    cgt += __popc(wb[w]);
-  }
-  uint32_t eq_total, gt_total;
-  const uint32_t eq_ex = block_exclusive_scan(ceq, wsum, &eq_total);
-  (void)block_exclusive_scan(cgt, wsum, &gt_total);
-  if (tid == 0) {
-    cta_tot[0] = eq_total;
-    cta_tot[1] = gt_total;
-  }
-  cluster_sync();
-  const uint32_t kties = exact ? krem : 0u;
-  uint32_t eq_before = 0, sel_before = 0;
-  for (uint32_t r2 = 0; r2 < rank; ++r2) {
-    const uint32_t e = dsmem_ld_u32(dsmem_addr(&cta_tot[0], r2));
-    const uint32_t g = dsmem_ld_u32(dsmem_addr(&cta_tot[1], r2));
-    const uint32_t take = kties > eq_before ? min(e, kties - eq_before) : 0u;
-    sel_before += g + take;
-    eq_before += e;
-  }
-  uint32_t run_eq = eq_before + eq_ex, csel = 0;
+
+  // ---- selected keys before this warp's run: earlier ranks, then earlier warps
+  uint32_t sel_r, eq_r, sel_w, eq_w;
+  prefix_take(lane < C ? misc[kMiscRankGt + lane] : 0u, lane < C ? misc[kMiscRankEq + lane] : 0u,
+              (int)rank, 0u, kties, lane, sel_r, eq_r);
+  prefix_take(lane < kWarps ? misc[kMiscWarpGt + lane] : 0u,
+              lane < kWarps ? misc[kMiscWarpEq + lane] : 0u, warp, eq_r, kties, lane, sel_w, eq_w);
+  uint32_t run_eq = eq_r + eq_w, run_sel = sel_r + sel_w;
+
+  // ---- the selected bits of each word and the output positions, 32 words at a time
   uint32_t* brow = p.bitmaps ? p.bitmaps + (size_t)(b * p.Hq + h) * p.nwords + w0 : nullptr;
-  for (int w = ta; w < tb; ++w) {
-    const uint32_t eq = wa[w];
+  int32_t* orow = p.idx_out ? p.idx_out + (size_t)(b * p.Hq + h) * p.k : nullptr;
+  for (int g0 = j0; g0 < j1; g0 += 32) {
+    const int j = g0 + lane;
+    const bool in = j < j1;
+    const uint32_t eq = in ? wa[j] : 0u, gt = in ? wb[j] : 0u;
     const uint32_t ce = __popc(eq);
-    const uint32_t allow = kties > run_eq ? min(ce, kties - run_eq) : 0u;
-    uint32_t keep = eq;
-    for (uint32_t c2 = ce; c2 > allow; --c2) keep &= ~(1u << (31 - __clz(keep)));
-    const uint32_t sel = wb[w] | keep;
-    wa[w] = sel;
-    run_eq += ce;
-    csel += __popc(sel);
-    if (brow) brow[w] = sel;
-  }
-  uint32_t sel_total;
-  uint32_t off = block_exclusive_scan(csel, wsum, &sel_total);
-  for (int w = ta; w < tb; ++w) {
-    wb[w] = off;
-    off += __popc(wa[w]);
-  }
-  __syncthreads();
-  if (p.idx_out) {
-    int32_t* orow = p.idx_out + (size_t)(b * p.Hq + h) * p.k;
-    for (int wl = warp; wl < mywords; wl += kWarps) {
-      const uint32_t sel = wa[wl];
-      if ((sel >> lane) & 1u) {
-        const uint32_t o = sel_before + wb[wl] + __popc(sel & ((1u << lane) - 1u));
-        if (o < (uint32_t)p.k) orow[o] = pos0 + wl * 32 + lane;
+    const uint32_t ie = warp_inclusive_scan(ce, lane);
+    const uint32_t r0 = run_eq + ie - ce;
+    const uint32_t allow = kties > r0 ? min(ce, kties - r0) : 0u;
+    const uint32_t keep = allow == ce ? eq : lowest_set_bits(eq, allow);
+    const uint32_t sel = gt | keep;
+    const uint32_t cs = __popc(sel);
+    const uint32_t is = warp_inclusive_scan(cs, lane);
+    const uint32_t off = run_sel + is - cs;
+    if (in && brow) brow[j] = sel;
+    if (orow) {
+      const int nw = min(32, j1 - g0);
+      for (int t = 0; t < nw; ++t) {
+        const uint32_t s2 = __shfl_sync(kFull, sel, t);
+        const uint32_t o2 = __shfl_sync(kFull, off, t);
+        if ((s2 >> lane) & 1u) {
+          const uint32_t o = o2 + __popc(s2 & ((1u << lane) - 1u));
+          if (o < (uint32_t)p.k) orow[o] = pos0 + (g0 + t) * 32 + lane;
+        }
       }
     }
-    if (rank == 0)
-      for (int t = kb + tid; t < p.k; t += kThreads) orow[t] = -1;
+    run_eq += __shfl_sync(kFull, ie, 31);
+    run_sel += __shfl_sync(kFull, is, 31);
   }
-  cluster_sync();  // no CTA leaves while a peer may still read its shared memory
+  if (orow)
+    for (int t = kb + (int)rank * kThreads + tid; t < p.k; t += C * kThreads) orow[t] = -1;
+  cluster_wait();    // no CTA leaves while a histogram may still be on its way to it
 }
 
 template <int C>
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(kThreads, 2)
     topk_kernel(const __grid_constant__ TopkParams p, int keys_cap, int wpc_cap) {
   extern __shared__ __align__(16) uint32_t dsm[];
   pdl_launch_dependents();
+  topk_prologue<C>(dsm);
   pdl_wait();
   topk_body<C>(p, keys_cap, wpc_cap, blockIdx.x, dsm);
 }
@@ -242,13 +340,14 @@ __global__ void __launch_bounds__(kThreads, 1)
 // The two read disjoint data (logits; partial states) and write disjoint
 // outputs (sets; the attention output).
 template <int C, typename T, int D>
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(kThreads, D >= 128 ? 2 : 1)
     topk_combine_kernel(const __grid_constant__ TopkParams p, const __grid_constant__ CombineParams cp,
                         int keys_cap, int wpc_cap, int ntopk, int ncomb) {
   extern __shared__ __align__(16) uint32_t dsm[];
   pdl_launch_dependents();
-  pdl_wait();
   const int cta = blockIdx.x;
+  if (cta < ntopk) topk_prologue<C>(dsm);
+  pdl_wait();
   if (cta < ntopk) topk_body<C>(p, keys_cap, wpc_cap, cta, dsm);
   else if (cta - ntopk < ncomb) combine_body<T, D>(cp, cta - ntopk, reinterpret_cast<unsigned char*>(dsm));
 }
@@ -262,10 +361,10 @@ struct Geometry {
   explicit Geometry(int N_max) {
     const int words_max = (N_max + 31) / 32;
     wpc_cap = (words_max + C - 1) / C;
-    const size_t fixed = (size_t)(2 * wpc_cap + kWarps * 256) * 4;
+    const size_t fixed = TopkSmem<C>::bytes(wpc_cap, 0);
     if (fixed + 4096 > kSmemBudget) return;
     keys_cap = (int)std::min<size_t>((size_t)wpc_cap * 32, (kSmemBudget - fixed) / 4);
-    smem = (size_t)keys_cap * 4 + fixed;
+    smem = TopkSmem<C>::bytes(wpc_cap, keys_cap);
     ok = true;
   }
 };
