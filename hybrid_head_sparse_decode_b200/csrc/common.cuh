@@ -198,67 +198,10 @@ __device__ __forceinline__ uint32_t dsmem_addr(const void* p, uint32_t rank) {
   return out;
 }
 
-// The same shared-window offset (a shared::cta address) in CTA `rank`'s window.
-__device__ __forceinline__ uint32_t dsmem_map(uint32_t local, uint32_t rank) {
-  uint32_t out;
-  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(out) : "r"(local), "r"(rank));
-  return out;
-}
-
 __device__ __forceinline__ uint32_t dsmem_ld_u32(uint32_t addr) {
   uint32_t v;
   asm volatile("ld.shared::cluster.u32 %0, [%1];" : "=r"(v) : "r"(addr) : "memory");
   return v;
-}
-
-// Split cluster barrier: every thread of every CTA of the cluster arrives, and
-// a later wait returns once all have.
-__device__ __forceinline__ void cluster_arrive() {
-  asm volatile("barrier.cluster.arrive.release.aligned;" ::: "memory");
-}
-// The same arrival without ordering this thread's earlier memory accesses (for
-// a barrier that only marks progress, or after fence_mbar_init).
-__device__ __forceinline__ void cluster_arrive_relaxed() {
-  asm volatile("barrier.cluster.arrive.relaxed.aligned;" ::: "memory");
-}
-__device__ __forceinline__ void cluster_wait() {
-  asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory");
-}
-
-// 16-byte store into another CTA's shared memory (both addresses from
-// dsmem_addr); its bytes count as transaction bytes on that CTA's mbarrier.
-__device__ __forceinline__ void st_async_v4(uint32_t remote, uint4 v, uint32_t remote_bar) {
-  asm volatile(
-      "st.async.shared::cluster.mbarrier::complete_tx::bytes.v4.b32 [%0], {%1, %2, %3, %4}, [%5];" ::"r"(
-          remote),
-      "r"(v.x), "r"(v.y), "r"(v.z), "r"(v.w), "r"(remote_bar)
-      : "memory");
-}
-
-// Bounded wait on a local mbarrier whose transaction bytes come from other CTAs
-// of the cluster: acquire at cluster scope, so their stores are visible after.
-__device__ __forceinline__ bool mbar_try_wait_cluster(uint64_t* bar, uint32_t parity,
-                                                      uint32_t hint_ns = 1000000u) {
-  uint32_t ok;
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2, %3;\n\t"
-      "selp.u32 %0, 1, 0, p;\n\t}"
-      : "=r"(ok)
-      : "r"(smem_u32(bar)), "r"(parity), "r"(hint_ns)
-      : "memory");
-  return ok != 0;
-}
-__device__ __forceinline__ bool mbar_wait_cluster(uint64_t* bar, uint32_t parity, uint32_t* err) {
-  if (mbar_try_wait_cluster(bar, parity)) return true;
-  const uint64_t t0 = globaltimer();
-  while (!mbar_try_wait_cluster(bar, parity)) {
-    if (globaltimer() - t0 > kWaitLimitNs) {
-      flag_error(err, kErrTimeout);
-      return false;
-    }
-  }
-  return true;
 }
 
 // ---- numeric helpers --------------------------------------------------------------

@@ -18,6 +18,7 @@
 // selecting on attention weights.
 #include <algorithm>
 
+#include "cluster.cuh"
 #include "combine_body.cuh"
 #include "common.cuh"
 #include "kernels.h"
