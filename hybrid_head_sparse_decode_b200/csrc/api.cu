@@ -21,7 +21,7 @@ namespace {
 constexpr int kVersion = 100;   // 0.1.0
 
 struct Layout {
-  size_t logits, part_ml, part_acc, part_n, part2, ccnt, bitmaps, total;
+  size_t logits, part_ml, part_acc, part_n, bitmaps, total;
   int nchunk, nwords;
 };
 
@@ -59,10 +59,6 @@ Layout layout_of(const lychee_shape* s) {
   off += align256(bh * L.nchunk * kPartSlots * s->d * 4);
   L.part_n = off;
   off += align256(bh * L.nchunk * 4);
-  L.part2 = off;
-  off += align256(bh * kCombineSplit * (s->d + 4) * 4);
-  L.ccnt = off;
-  off += align256(bh * 4);
   L.bitmaps = off;
   off += align256(bh * L.nwords * 4);
   L.total = off;
@@ -211,8 +207,6 @@ lychee_status run_layer(const Ctx& c, const void* q, const void* kc, const void*
   float* part_ml = reinterpret_cast<float*>(c.ws + c.L.part_ml);
   float* part_acc = reinterpret_cast<float*>(c.ws + c.L.part_acc);
   int32_t* part_n = reinterpret_cast<int32_t*>(c.ws + c.L.part_n);
-  float* part2 = reinterpret_cast<float*>(c.ws + c.L.part2);
-  uint32_t* ccnt = reinterpret_cast<uint32_t*>(c.ws + c.L.ccnt);
   uint32_t* bitmaps = reinterpret_cast<uint32_t*>(c.ws + c.L.bitmaps);
   uint8_t rheads[kMaxHq], sheads[kMaxHq];
   int nr = 0, ns = 0;
@@ -243,7 +237,6 @@ lychee_status run_layer(const Ctx& c, const void* q, const void* kc, const void*
   ap.part_ml = part_ml;
   ap.part_acc = part_acc;
   ap.part_n = part_n;
-  ap.ccnt = ccnt;
   ap.k_per_seq = k_per_seq;
   ap.err = err;
   ap.counter = counter;
@@ -273,10 +266,9 @@ lychee_status run_layer(const Ctx& c, const void* q, const void* kc, const void*
   cp.part_ml = part_ml;
   cp.part_acc = part_acc;
   cp.part_n = part_n;
-  cp.part2 = part2;
-  cp.ccnt = ccnt;
   cp.seqlens = seqlens;
   cp.out = out;
+  cp.err = err;
   cp.B = s->B; cp.Hq = Hq; cp.N_max = s->N_max; cp.nchunk = c.L.nchunk;
   cp.scale_log2 = ap.scale_log2;
   e = timed(nr > 0 ? kKindTopkCombine : kKindCombine, c.st,

@@ -276,9 +276,6 @@ __global__ void __launch_bounds__((NW + NP) * 32, 1)
   const bool compact = B <= kMaxBatchCompact;
   pdl_launch_dependents();
   pdl_wait();
-  // the combine kernel that follows counts its finished CTAs from zero
-  for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < B * Hq; i += gridDim.x * blockDim.x)
-    p.ccnt[i] = 0u;
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
       mbar_init(&full[s], NS);

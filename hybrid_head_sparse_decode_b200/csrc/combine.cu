@@ -14,9 +14,11 @@
 // loading kBatch states before merging them into its running sums (rescaled
 // when the maximum grows), so that the slot's loads are in flight together.
 // The slots are merged in a fixed order in shared memory into one state per
-// CTA; the last CTA of the head (counted with an atomic) merges the
-// kCombineSplit states in order and writes the output.  The result does not
-// depend on scheduling.
+// CTA.  The head's CTAs form one group of a thread-block cluster: each sends its
+// state into the shared memory of the group's first CTA (16-byte st.async
+// stores that complete that CTA's mbarrier), which merges the kCombineSplit
+// states in order and writes the output.  The result does not depend on
+// scheduling.
 #include "combine_body.cuh"
 
 namespace lychee {
@@ -26,15 +28,30 @@ template <typename T, int D>
 __global__ void __launch_bounds__(kCombThreads) combine_kernel(const __grid_constant__ CombineParams p) {
   extern __shared__ __align__(16) unsigned char csm[];
   pdl_launch_dependents();
+  combine_prologue<D>(csm);
   pdl_wait();
   combine_body<T, D>(p, blockIdx.x, csm);
 }
 
 template <typename T, int D>
 cudaError_t launch_combine_t(const CombineParams& p, cudaStream_t st) {
+  // clusters of kCombineSplit CTAs (a portable size): one head per cluster
   const unsigned grid = (unsigned)(p.B * p.Hq * kCombineSplit);
-  const cudaError_t e =
-      launch_pdl(combine_kernel<T, D>, dim3(grid), dim3(kCombThreads), combine_smem_bytes<D>(), st, p);
+  cudaLaunchConfig_t cfg{};
+  cfg.gridDim = dim3(grid);
+  cfg.blockDim = dim3(kCombThreads);
+  cfg.dynamicSmemBytes = combine_smem_bytes<D>();
+  cfg.stream = st;
+  cudaLaunchAttribute at[2];
+  at[0].id = cudaLaunchAttributeClusterDimension;
+  at[0].val.clusterDim.x = kCombineSplit;
+  at[0].val.clusterDim.y = 1;
+  at[0].val.clusterDim.z = 1;
+  at[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  at[1].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = at;
+  cfg.numAttrs = 2;
+  const cudaError_t e = cudaLaunchKernelEx(&cfg, combine_kernel<T, D>, p);
   if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }

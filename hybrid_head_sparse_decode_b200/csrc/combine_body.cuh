@@ -3,6 +3,7 @@
 // top-k + combine launch (topk.cu).
 #pragma once
 
+#include "cluster.cuh"
 #include "common.cuh"
 #include "kernels.h"
 
@@ -46,26 +47,69 @@ __device__ __forceinline__ void absorb(float2 e, float4 a, float sl, float& m, f
   }
 }
 
-// Shared memory one combine CTA uses (16-byte aligned start).
+constexpr int kCombineSplit = 8;   // combine CTAs per (sequence, head): one group of a cluster
+
+// Shared memory of one combine CTA, in bytes from its (16-byte aligned) start:
+//   bar   one mbarrier (8 bytes, padded to 16)
+//   recv  [kCombineSplit][D + 4] floats: the head's CTA states (leader CTA only)
+//   red   [NS][D + 4] floats: this CTA's slot states, then its own state
+//   slist [kCombThreads * kPartSlots] u16: the states of a block of chunks, in order
+//   wsum  [kCombWarps + 1] ints
+template <int D>
+struct CombineSmem {
+  static constexpr int RS = D + 4;                       // state row: acc[D], m, l, pad
+  static constexpr int NS = kCombWarps * (32 / (D / 4)); // slots of the CTA
+  static constexpr size_t kRecv = 16;
+  static constexpr size_t kRed = kRecv + (size_t)kCombineSplit * RS * 4;
+  static constexpr size_t kSlist = kRed + (size_t)(NS + 1) * RS * 4;
+  static constexpr size_t kWsum = kSlist + (size_t)kCombThreads * kPartSlots * 2;
+  static constexpr size_t kBytes = kWsum + (kCombWarps + 1) * 4;
+  static_assert(kRed % 16 == 0 && kSlist % 16 == 0 && (RS * 4) % 16 == 0, "16-byte rows");
+};
 template <int D>
 constexpr size_t combine_smem_bytes() {
-  return (size_t)(kCombWarps * (32 / (D / 4)) * (D + 4)) * 4 + kCombThreads * kPartSlots * 2 +
-         kCombWarps * 4 + 16;
+  return CombineSmem<D>::kBytes;
 }
 
-// One combine CTA: `cta` numbers the CTA among all combine CTAs, `sm` is its
-// shared memory (combine_smem_bytes<D>() bytes).  kCombThreads threads.
+// Before the previous kernel's results are needed: the CTA's mbarrier expects
+// the states of the other kCombineSplit - 1 CTAs of its head (only the head's
+// first CTA, its leader, receives any), and the cluster learns it is set up.
+// Every CTA of a launch whose clusters hold combine CTAs runs this, idle ones too.
+template <int D>
+__device__ __forceinline__ void combine_prologue(unsigned char* sm) {
+  uint64_t* bar = reinterpret_cast<uint64_t*>(sm);
+  if (threadIdx.x == 0) {
+    mbar_init(bar, 1);
+    fence_mbar_init();
+    mbar_arrive_expect_tx(bar, (kCombineSplit - 1) * CombineSmem<D>::RS * 4);
+  }
+  cluster_arrive_relaxed();
+}
+
+// The two remaining cluster barriers of a CTA that has no state to combine.
+__device__ __forceinline__ void combine_idle() {
+  cluster_wait();
+  cluster_arrive_relaxed();
+  cluster_wait();
+}
+
+// One combine CTA, after combine_prologue: `cta` numbers the CTA among all
+// combine CTAs (the kCombineSplit CTAs of a head are consecutive and start a
+// group of the cluster), `sm` is its shared memory (combine_smem_bytes<D>()
+// bytes).  kCombThreads threads.
 template <typename T, int D>
 __device__ __forceinline__ void combine_body(const CombineParams& p, int cta, unsigned char* sm) {
+  using L = CombineSmem<D>;
   constexpr int kThreads = kCombThreads, kWarps = kCombWarps;
   constexpr int LPR = D / 4;             // lanes per state row
   constexpr int SLOTS = 32 / LPR;        // state rows a warp reads at once
-  constexpr int NS = kWarps * SLOTS;     // slots of the CTA
-  constexpr int RS = D + 4;              // smem row: acc[D], m, l, pad
-  float* red = reinterpret_cast<float*>(sm);                                     // [NS * RS]
-  uint16_t* slist = reinterpret_cast<uint16_t*>(sm + NS * RS * 4);               // (chunk, state)
-  int* wsum = reinterpret_cast<int*>(sm + NS * RS * 4 + kThreads * kPartSlots * 2);
-  int& is_last = wsum[kWarps];
+  constexpr int NS = L::NS;
+  constexpr int RS = L::RS;
+  uint64_t* bar = reinterpret_cast<uint64_t*>(sm);
+  float* recv = reinterpret_cast<float*>(sm + L::kRecv);
+  float* red = reinterpret_cast<float*>(sm + L::kRed);
+  uint16_t* slist = reinterpret_cast<uint16_t*>(sm + L::kSlist);
+  int* wsum = reinterpret_cast<int*>(sm + L::kWsum);
   const int bh = cta / kCombineSplit, sp = cta % kCombineSplit;
   const int b = bh / p.Hq;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -130,54 +174,63 @@ __device__ __forceinline__ void combine_body(const CombineParams& p, int cta, un
     row[D + 1] = l;
   }
   __syncthreads();
-  // this CTA's state, merged over the slots in order
-  float* st = p.part2 + (size_t)cta * RS;
+  // this CTA's state, merged over the slots in order: the leader keeps it in
+  // its first receive row, the others stage it for sending
+  float* mine = sp == 0 ? recv : red + NS * RS;
   if (tid < D) {
     float M = -INFINITY;
     for (int s2 = 0; s2 < NS; ++s2) M = fmaxf(M, red[s2 * RS + D]);
-    float A = 0.f, L = 0.f;
+    float A = 0.f, Lsum = 0.f;
     if (M != -INFINITY) {
       for (int s2 = 0; s2 < NS; ++s2) {
         const float ms = red[s2 * RS + D];
         const float w = ms == -INFINITY ? 0.f : fast_exp2((ms - M) * sl);
         A = fmaf(w, red[s2 * RS + tid], A);
-        L = fmaf(w, red[s2 * RS + D + 1], L);
+        Lsum = fmaf(w, red[s2 * RS + D + 1], Lsum);
       }
     }
-    st[tid] = A;
+    mine[tid] = A;
     if (tid == 0) {
-      st[D] = M;
-      st[D + 1] = L;
+      mine[D] = M;
+      mine[D + 1] = Lsum;
+      mine[D + 2] = 0.f;
+      mine[D + 3] = 0.f;
     }
   }
   __syncthreads();
-  if (tid == 0) {
-    __threadfence();
-    is_last = atomicAdd(&p.ccnt[bh], 1u) == kCombineSplit - 1;
+  cluster_wait();   // every leader's barrier is set up
+  const uint32_t leader = cluster_ctarank() - (uint32_t)sp;
+  if (sp != 0) {
+    // send the state to row sp of the leader's receive rows
+    if (tid < RS / 4) {
+      const float4 v = reinterpret_cast<const float4*>(mine)[tid];
+      st_async_v4(dsmem_map(smem_u32(recv + sp * RS + 4 * tid), leader),
+                  make_uint4(__float_as_uint(v.x), __float_as_uint(v.y), __float_as_uint(v.z),
+                             __float_as_uint(v.w)),
+                  dsmem_map(smem_u32(bar), leader));
+    }
+  } else {
+    mbar_wait_cluster(bar, 0u, p.err);   // the head's other states are here
   }
-  __syncthreads();
-  if (!is_last) return;
-  // the head's last CTA: merge the kCombineSplit states in order
-  __threadfence();
-  if (tid < D) {
-    const float* s0 = p.part2 + (size_t)bh * kCombineSplit * RS;
+  cluster_arrive_relaxed();   // nothing more will arrive here (checked before exit)
+  if (sp == 0 && tid < D) {
+    // the head's kCombineSplit states, merged in order
     float M = -INFINITY;
 #pragma unroll
-    for (int k = 0; k < kCombineSplit; ++k) M = fmaxf(M, __ldcg(s0 + k * RS + D));
-    float A = 0.f, L = 0.f;
+    for (int k = 0; k < kCombineSplit; ++k) M = fmaxf(M, recv[k * RS + D]);
+    float A = 0.f, Lsum = 0.f;
     if (M != -INFINITY) {
 #pragma unroll
       for (int k = 0; k < kCombineSplit; ++k) {
-        const float ms = __ldcg(s0 + k * RS + D);
+        const float ms = recv[k * RS + D];
         const float w = ms == -INFINITY ? 0.f : fast_exp2((ms - M) * sl);
-        A = fmaf(w, __ldcg(s0 + k * RS + tid), A);
-        L = fmaf(w, __ldcg(s0 + k * RS + D + 1), L);
+        A = fmaf(w, recv[k * RS + tid], A);
+        Lsum = fmaf(w, recv[k * RS + D + 1], Lsum);
       }
     }
-    store_out<T>(reinterpret_cast<T*>(p.out) + (size_t)bh * D + tid, L > 0.f ? A / L : 0.f);
+    store_out<T>(reinterpret_cast<T*>(p.out) + (size_t)bh * D + tid, Lsum > 0.f ? A / Lsum : 0.f);
   }
-  if (tid == 0) p.ccnt[bh] = 0u;   // ready for the next launch
+  cluster_wait();   // no CTA leaves while a state may still be on its way to it
 }
-
 
 }  // namespace lychee

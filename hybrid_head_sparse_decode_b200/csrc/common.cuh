@@ -31,7 +31,6 @@ static_assert(sizeof(WsHeader) == 256, "header is 256 bytes");
 
 constexpr int kChunk = 960;           // positions per attention work item (30 words)
 constexpr int kPartSlots = 12;        // partial states per (sequence, head, chunk): one per warp
-constexpr int kCombineSplit = 4;      // combine CTAs per (sequence, head)
 constexpr int kMaxHq = 128;           // query heads supported
 constexpr uint64_t kWaitLimitNs = 2000000000ull;   // 2 s: a wait this long is a fault
 

@@ -18,7 +18,6 @@ struct AttnParams {
   float* part_ml;           // [B, Hq, nchunk, kPartSlots, 2]: (max raw dot, sum of weights)
   float* part_acc;          // [B, Hq, nchunk, kPartSlots, D]: unnormalised weighted values
   int32_t* part_n;          // [B, Hq, nchunk]: partial states written for the chunk
-  uint32_t* ccnt;           // [B, Hq]: combine counters, zeroed here for the combine kernel
   const int32_t* k_per_seq; // [B] or null (validated here)
   uint32_t* err;
   uint32_t* counter;        // work-item counter, 0 at launch, 0 again at exit
@@ -53,10 +52,9 @@ struct CombineParams {
   const float* part_ml;      // [B, Hq, nchunk, kPartSlots, 2]
   const float* part_acc;     // [B, Hq, nchunk, kPartSlots, D]
   const int32_t* part_n;     // [B, Hq, nchunk]: states used per chunk
-  float* part2;              // [B, Hq, kCombineSplit, D + 4]: one state per combine CTA
-  uint32_t* ccnt;            // [B, Hq]: finished combine CTAs (0 at launch, 0 again at exit)
   const int32_t* seqlens;    // [B]
   void* out;                 // [B, Hq, D]
+  uint32_t* err;
   int B, Hq, N_max, nchunk;
   float scale_log2;
 };

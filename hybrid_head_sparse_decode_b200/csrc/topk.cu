@@ -336,8 +336,10 @@ __global__ void __launch_bounds__(kThreads, 2)
 }
 
 // Top-k of the retrieval heads and the combine of all heads in one launch: the
-// first ntopk CTAs (whole clusters) select, the next ncomb CTAs combine (their
-// clusters never synchronise), the rest of the last cluster has nothing to do.
+// first ntopk CTAs (whole clusters) select, the next ncomb CTAs combine (each
+// head's kCombineSplit CTAs are one group of a cluster, since C is a multiple
+// of kCombineSplit), the rest of the last cluster only takes part in its
+// cluster barriers.
 // The two read disjoint data (logits; partial states) and write disjoint
 // outputs (sets; the attention output).
 template <int C, typename T, int D>
@@ -346,11 +348,15 @@ __global__ void __launch_bounds__(kThreads, D >= 128 ? 2 : 1)
                         int keys_cap, int wpc_cap, int ntopk, int ncomb) {
   extern __shared__ __align__(16) uint32_t dsm[];
   pdl_launch_dependents();
+  static_assert(C % kCombineSplit == 0, "a head's combine CTAs share a cluster");
   const int cta = blockIdx.x;
+  unsigned char* csm = reinterpret_cast<unsigned char*>(dsm);
   if (cta < ntopk) topk_prologue<C>(dsm);
+  else combine_prologue<D>(csm);
   pdl_wait();
   if (cta < ntopk) topk_body<C>(p, keys_cap, wpc_cap, cta, dsm);
-  else if (cta - ntopk < ncomb) combine_body<T, D>(cp, cta - ntopk, reinterpret_cast<unsigned char*>(dsm));
+  else if (cta - ntopk < ncomb) combine_body<T, D>(cp, cta - ntopk, csm);
+  else combine_idle();
 }
 
 // Launch geometry of a cluster size C for rows of up to N_max logits.
