@@ -96,6 +96,16 @@ constexpr int kConsRegs = LYCHEE_ATTN_CONS_REGS;
 #ifndef LYCHEE_ATTN_TMA_ROWS
 #define LYCHEE_ATTN_TMA_ROWS 8
 #endif
+// bf16 caches: consumer warps contract on the tensor cores (mma.sync, see
+// consumer_loop_mma); 0: the fp32-FMA consumer for every type.
+#ifndef LYCHEE_ATTN_MMA
+#define LYCHEE_ATTN_MMA 1
+#endif
+template <typename T>
+constexpr bool mma_path() {
+  return LYCHEE_ATTN_MMA && std::is_same<T, __nv_bfloat16>::value;
+}
+
 // 1: the TMA part of a sparse tile goes as 1-D bulk copies of runs of
 // consecutive positions instead of tile::gather4 copies
 #ifndef LYCHEE_ATTN_RUNS
@@ -142,19 +152,27 @@ struct AttnCfg {
   static constexpr int MAXT = (kChunk + TT - 1) / TT;   // tiles per item at most
   static_assert(CPL >= 2 && DL % E == 0 && CPL % 2 == 0, "lane mapping");
   static_assert(TT % kPairsPerBatch == 0 && TT % 4 == 0 && TT <= 255, "tile rows");
-  static_assert(G <= NW && NW <= kPartSlots && NW <= 16, "warps per head fit the partial slots");
+  static constexpr bool MMA = mma_path<T>();
+  static_assert(MMA ? (G <= 8 && NW <= kPartSlots && TT % 16 == 0)
+                    : (G <= NW && NW <= kPartSlots && NW <= 16),
+                "warps per head fit the partial slots; tensor-core slabs of 16 rows");
   static_assert(NP >= 2, "a builder and at least one streaming warp");
   static_assert(kChunk % 32 == 0 && kChunk <= 1024, "builder holds one word per lane");
   static_assert(MAXT < 32, "one lane per tile start");
 
-  // item buffer (two of them): descriptor, warp assignment, where each tile
-  // starts in each sparse head's row list, the row lists (union indices of the
-  // head's rows, in order), the gather positions
+  // item buffer (two of them): descriptor, then for the fp32-FMA consumers the
+  // warp assignment, where each tile starts in each sparse head's row list and
+  // the row lists (union indices of the head's rows, in order), for the
+  // tensor-core consumers each head's membership word for every 32 positions
+  // of the chunk ([word][8] u32, head t at t; heads >= G zero), then the gather
+  // positions
   static constexpr int ASGB = NW + G;             // warp -> (head, slot), warps per head
   static constexpr int IB_ASG = 32;
-  static constexpr int IB_TST = IB_ASG + (ASGB + 15) / 16 * 16;          // [G][32] u16
-  static constexpr int IB_HROW = IB_TST + G * 32 * 2;                    // [G][kChunk] u16
-  static constexpr int IB_LPOS = IB_HROW + G * kChunk * 2;               // [kChunk] i32
+  static constexpr int IB_TST = IB_ASG + (MMA ? 0 : (ASGB + 15) / 16 * 16);   // [G][32] u16
+  static constexpr int IB_HROW = IB_TST + (MMA ? 0 : G * 32 * 2);             // [G][kChunk] u16
+  static constexpr int IB_HW = IB_HROW + (MMA ? 0 : G * kChunk * 2);          // [kChunk/32][8] u32
+  static constexpr int IB_LPOS = IB_HW + (MMA ? kChunk : 0);                  // [kChunk] i32
+  static_assert(IB_LPOS % 16 == 0, "positions read four at a time");
   static constexpr int IBUF = IB_LPOS + kChunk * 4;
 
   // shared memory layout (byte offsets from a 128-byte aligned base)
@@ -252,6 +270,9 @@ __device__ __forceinline__ MergeW merge_weights(float& m, float& l, float m2, fl
 template <typename T, int D, int G, int NW, int NP, int TT, int STAGES>
 __device__ __forceinline__ void consumer_loop(const AttnParams& p, unsigned char* smem,
                                               uint64_t* full, uint64_t* empty, uint64_t* freeb);
+template <typename T, int D, int G, int NW, int NP, int TT, int STAGES>
+__device__ __forceinline__ void consumer_loop_mma(const AttnParams& p, unsigned char* smem,
+                                                  uint64_t* full, uint64_t* empty, uint64_t* freeb);
 
 template <typename T, int D, int G, int NW, int NP, int TT, int STAGES>
 __global__ void __launch_bounds__((NW + NP) * 32, 1)
@@ -308,7 +329,7 @@ __global__ void __launch_bounds__((NW + NP) * 32, 1)
   __syncthreads();
 
   constexpr int ILP = ilp_of<T, D>();
-  if constexpr (ILP > 1 && LYCHEE_ATTN_REGSPLIT) {
+  if constexpr (!C::MMA && ILP > 1 && LYCHEE_ATTN_REGSPLIT) {
     static_assert(NW % 4 == 0 && NP == 4, "whole warpgroups: NW consumers, 4 producers");
     static_assert(4 * 32 * kProdRegs + NW * 32 * kConsRegs <= (NW + NP) * 32 * 128,
                   "register split within the launch's registers");
@@ -404,54 +425,68 @@ __global__ void __launch_bounds__((NW + NP) * 32, 1)
               lpos[o++] = p0 + 32 * lane + j;
             }
           }
-          // each sparse head's rows as union indices, in order (lane w places
-          // the rows of word w), and where each tile starts in that list: a
-          // tile boundary (a multiple of TT > 32 union rows) falls inside at
-          // most one word, whose lane writes the start (a retrieval head takes
-          // every row: no list)
-          uint16_t* hrow = reinterpret_cast<uint16_t*>(ib + C::IB_HROW);
-          uint16_t* tst = reinterpret_cast<uint16_t*>(ib + C::IB_TST);
-          const int ntile = (total + TT - 1) / TT;
-          const int tb = (ubase + TT - 1) / TT;         // first tile starting at or after ubase
-          const bool has_bound = tb * TT < ubase + cnt;  // ... and inside this word
-          int bpos = 0;                                  // position of that boundary row
-          if (has_bound) {
-            uint32_t u = uni;
-            for (int r2 = tb * TT - ubase; r2 > 0; --r2) u &= u - 1;
-            bpos = __ffs(u) - 1;
-          }
-          int work[G];
+          if constexpr (C::MMA) {
+            // the heads' membership words (a retrieval head's: every valid row)
+            if (lane < kChunk / 32) {
+              uint32_t hv[8];
 #pragma unroll
-          for (int t = 0; t < G; ++t) {
-            const int ct = __popc(bits[t]);
-            int ic = ct;
+              for (int t = 0; t < 8; ++t) hv[t] = t < G ? bits[t] : 0u;
+              uint4* hw = reinterpret_cast<uint4*>(ib + C::IB_HW) + 2 * lane;
+              hw[0] = make_uint4(hv[0], hv[1], hv[2], hv[3]);
+              hw[1] = make_uint4(hv[4], hv[5], hv[6], hv[7]);
+            }
+            // every consumer warp writes a partial state for every head
+            if (lane < G) p.part_n[(size_t)(b * Hq + h0 + lane) * p.nchunk + c] = NW;
+          } else {
+            // each sparse head's rows as union indices, in order (lane w places
+            // the rows of word w), and where each tile starts in that list: a
+            // tile boundary (a multiple of TT > 32 union rows) falls inside at
+            // most one word, whose lane writes the start (a retrieval head takes
+            // every row: no list)
+            uint16_t* hrow = reinterpret_cast<uint16_t*>(ib + C::IB_HROW);
+            uint16_t* tst = reinterpret_cast<uint16_t*>(ib + C::IB_TST);
+            const int ntile = (total + TT - 1) / TT;
+            const int tb = (ubase + TT - 1) / TT;         // first tile starting at or after ubase
+            const bool has_bound = tb * TT < ubase + cnt;  // ... and inside this word
+            int bpos = 0;                                  // position of that boundary row
+            if (has_bound) {
+              uint32_t u = uni;
+              for (int r2 = tb * TT - ubase; r2 > 0; --r2) u &= u - 1;
+              bpos = __ffs(u) - 1;
+            }
+            int work[G];
 #pragma unroll
-            for (int o = 1; o < 32; o <<= 1) {
-              const int y = __shfl_up_sync(kFull, ic, o);
-              if (lane >= o) ic += y;
+            for (int t = 0; t < G; ++t) {
+              const int ct = __popc(bits[t]);
+              int ic = ct;
+#pragma unroll
+              for (int o = 1; o < 32; o <<= 1) {
+                const int y = __shfl_up_sync(kFull, ic, o);
+                if (lane >= o) ic += y;
+              }
+              work[t] = __shfl_sync(kFull, ic, 31);
+              if ((rmask >> t) & 1u) continue;
+              uint16_t* hl = hrow + t * kChunk;
+              int k = ic - ct;
+              uint32_t u = bits[t];
+              while (u) {
+                const int j = __ffs(u) - 1;
+                u &= u - 1;
+                hl[k++] = (uint16_t)(ubase + __popc(uni & ((1u << j) - 1u)));
+              }
+              uint16_t* ts = tst + t * 32;
+              if (has_bound) ts[tb] = (uint16_t)(ic - ct + __popc(bits[t] & ((1u << bpos) - 1u)));
+              if (lane == 0) {
+                ts[0] = 0;
+                ts[ntile] = (uint16_t)work[t];
+              }
             }
-            work[t] = __shfl_sync(kFull, ic, 31);
-            if ((rmask >> t) & 1u) continue;
-            uint16_t* hl = hrow + t * kChunk;
-            int k = ic - ct;
-            uint32_t u = bits[t];
-            while (u) {
-              const int j = __ffs(u) - 1;
-              u &= u - 1;
-              hl[k++] = (uint16_t)(ubase + __popc(uni & ((1u << j) - 1u)));
-            }
-            uint16_t* ts = tst + t * 32;
-            if (has_bound) ts[tb] = (uint16_t)(ic - ct + __popc(bits[t] & ((1u << bpos) - 1u)));
-            if (lane == 0) {
-              ts[0] = 0;
-              ts[ntile] = (uint16_t)work[t];
-            }
+            if (lane == 0) assign_warps<G, NW>(work, asg, asg + NW);
+            __syncwarp();
+            // partial states each head's warps will write for this chunk
+            if (lane < G)
+              p.part_n[(size_t)(b * Hq + h0 + lane) * p.nchunk + c] = (int)asg[NW + lane];
           }
-          if (lane == 0) assign_warps<G, NW>(work, asg, asg + NW);
-          __syncwarp();
-          // partial states each head's warps will write for this chunk
-          if (lane < G)
-            p.part_n[(size_t)(b * Hq + h0 + lane) * p.nchunk + c] = (int)asg[NW + lane];
         }
         cur = nxt;
         cur_n = nxt_n;
@@ -597,7 +632,8 @@ __global__ void __launch_bounds__((NW + NP) * 32, 1)
       if (lane == 0) mbar_arrive(&freeb[buf]);   // done reading this item's positions
     }
   } else if (warp < NW) {
-    consumer_loop<T, D, G, NW, NP, TT, STAGES>(p, smem, full, empty, freeb);
+    if constexpr (C::MMA) consumer_loop_mma<T, D, G, NW, NP, TT, STAGES>(p, smem, full, empty, freeb);
+    else consumer_loop<T, D, G, NW, NP, TT, STAGES>(p, smem, full, empty, freeb);
   }
   // ---- the last CTA to leave resets the launch counters for the next launch
   __syncthreads();
@@ -853,6 +889,253 @@ __device__ __forceinline__ void consumer_loop(const AttnParams& p, unsigned char
   }
 }
 
+// ---- tensor-core consumers (bf16 caches) -------------------------------------
+// D += A * B on one warp: A 16x16 bf16 (row-major fragments), B 16x8 bf16
+// (column fragments), D and C 16x8 fp32.  Lane (g = lane / 4, t = lane % 4)
+// holds A rows g, g + 8 at columns 2t, 2t + 1 and 2t + 8, 2t + 9; B rows 2t,
+// 2t + 1 and 2t + 8, 2t + 9 of column g; C rows g, g + 8 at columns 2t, 2t + 1.
+__device__ __forceinline__ void mma_16816(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2,
+                                          uint32_t a3, uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, "
+      "{%8, %9}, {%0, %1, %2, %3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+// Transpose of an 8x8 matrix of 16-bit elements held one row per four lanes
+// (lane g * 4 + t: row g, columns 2t, 2t + 1).
+__device__ __forceinline__ uint32_t transpose8x8(uint32_t x) {
+  uint32_t y;
+  asm volatile("movmatrix.sync.aligned.m8n8.trans.b16 %0, %1;" : "=r"(y) : "r"(x));
+  return y;
+}
+__device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
+  const __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
+  return *reinterpret_cast<const uint32_t*>(&v);
+}
+__device__ __forceinline__ uint32_t word_of(const uint4& v, int i) {
+  return i == 0 ? v.x : i == 1 ? v.y : i == 2 ? v.z : v.w;
+}
+
+// Consumer warps of attn_kernel for bf16 caches.  A warp takes whole slabs of
+// 16 rows of a tile (slab sigma of an item, counted over its tiles, goes to warp
+// sigma mod NW) and serves every head of the group on them at once:
+//   S^T (16 rows x 8 heads; heads >= G are zero columns) = K_slab . q^T on the
+//   tensor cores, bf16 operands and fp32 accumulation; the head dimension is
+//   visited in a fixed permutation (lane t of a 32-dimension block reads
+//   dimensions 8t..8t+7 and feeds them as k = 2t, 2t+1, 2t+8, 2t+9 of two
+//   16-deep steps), the same for K and q, so every K row is read with plain
+//   16-byte loads;
+//   rows a head does not use (the heads' membership words of the item), rows
+//   past the tile and padding heads get score -inf; retrieval heads' raw scores go to the logits;
+//   online softmax per head with the lazy maximum;
+//   O^T (d x 8 heads) += V_slab^T . P on the tensor cores, P rounded to bf16
+//   (the weights summed into l are the rounded ones), V and P brought into
+//   fragment layout by 8x8 transposes in registers.
+// At the end of an item each warp writes one partial state per head of the
+// group into its own slot (slot = warp).
+template <typename T, int D, int G, int NW, int NP, int TT, int STAGES>
+__device__ __forceinline__ void consumer_loop_mma(const AttnParams& p, unsigned char* smem,
+                                                  uint64_t* full, uint64_t* empty, uint64_t* freeb) {
+  using C = AttnCfg<T, D, G, NW, NP, TT, STAGES>;
+  constexpr int ROWB = C::ROWB;
+  constexpr int NPB = D / 32;            // 32-dimension blocks
+  constexpr int SPT = TT / 16;           // slabs per tile
+  constexpr uint32_t kAll = (1u << G) - 1u;
+  const int4* info = reinterpret_cast<const int4*>(smem + C::OFF_INFO);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int g = lane >> 2, t = lane & 3;
+  const int hx = 2 * t, hy = 2 * t + 1;  // the lane's two heads (columns of S^T, O^T)
+  const float sl = p.scale_log2;
+  const float lazy = kLazyLog2 / sl;
+
+  uint4 qf[NPB];                         // q of head g, dimensions 32P + 8t .. + 7
+  float o[2 * NPB][4];                   // O^T fragments, block 2P + jp
+  float m[2], mth[2], msl[2], l[2];      // per lane head (hx, hy)
+  uint32_t rm = 0;
+  int b = 0, h0 = 0, c = 0, buf = 0;
+
+  uint32_t s = 0, ph = 0;
+  for (;;) {
+    if (!mbar_wait(&full[s], ph, p.err)) break;
+    const int4 i0 = info[2 * s], i1 = info[2 * s + 1];
+    const int flags = i1.x;
+    if (flags & kTerm) break;
+    const int nrows = i0.w, t0 = i1.z, tt = i1.w >> 8;
+    const unsigned char* ib = smem + C::OFF_ITEM + (i1.w & 1) * C::IBUF;
+
+    if (flags & kFirst) {
+      b = i0.x;
+      h0 = i0.y;
+      c = i0.z;
+      buf = i1.w & 1;
+      rm = (uint32_t)i1.y;
+      const unsigned char* qs = smem + C::OFF_Q + s * C::QSTRIDE + g * ROWB + 16 * t;
+#pragma unroll
+      for (int P = 0; P < NPB; ++P)
+        qf[P] = g < G ? *reinterpret_cast<const uint4*>(qs + 64 * P) : make_uint4(0u, 0u, 0u, 0u);
+#pragma unroll
+      for (int k = 0; k < 2 * NPB; ++k) o[k][0] = o[k][1] = o[k][2] = o[k][3] = 0.f;
+#pragma unroll
+      for (int e = 0; e < 2; ++e) {
+        m[e] = -INFINITY;
+        mth[e] = -INFINITY;
+        msl[e] = 0.f;
+        l[e] = 0.f;
+      }
+    }
+
+    const bool masked = rm != kAll;       // some head of the group uses only some rows
+    const uint32_t* hw = reinterpret_cast<const uint32_t*>(ib + C::IB_HW) + 2 * t;
+    const int32_t* lpos = reinterpret_cast<const int32_t*>(ib + C::IB_LPOS) + t0;
+    // bit 0 / 1: head hx / hy uses union row r of this tile (a group with a
+    // retrieval head reads every position of the chunk in order)
+    auto lane_heads = [&](int r) -> uint32_t {
+      const int po = rm ? t0 + r : lpos[r] - c * kChunk;
+      const uint2 w = *reinterpret_cast<const uint2*>(hw + (po >> 5) * 8);
+      return ((w.x >> (po & 31)) & 1u) | (((w.y >> (po & 31)) & 1u) << 1);
+    };
+    const uint32_t lane_all = (hx < G ? 1u : 0u) | (hy < G ? 2u : 0u);
+    const unsigned char* kt = smem + C::OFF_K + s * C::kStageKV + 16 * t;
+    const unsigned char* vt = smem + C::OFF_V + s * C::kStageKV + 16 * t;
+    const int nsl = (nrows + 15) >> 4;
+    int j = (warp - (tt * SPT) % NW) % NW;
+    if (j < 0) j += NW;
+    for (; j < nsl; j += NW) {
+      const int rA = 16 * j + g, rB = rA + 8;
+      const bool vA = rA < nrows, vB = rB < nrows;
+      const unsigned char* ka = kt + (vA ? rA : 0) * ROWB;
+      const unsigned char* kb = kt + (vB ? rB : 0) * ROWB;
+      uint4 KA[NPB], KB[NPB];
+#pragma unroll
+      for (int P = 0; P < NPB; ++P) {
+        KA[P] = *reinterpret_cast<const uint4*>(ka + 64 * P);
+        KB[P] = *reinterpret_cast<const uint4*>(kb + 64 * P);
+      }
+      // ---- S^T = K q^T (two accumulation chains)
+      float sc[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+#pragma unroll
+      for (int P = 0; P < NPB; ++P) {
+        mma_16816(sc[P & 1], KA[P].x, KB[P].x, KA[P].y, KB[P].y, qf[P].x, qf[P].y);
+        mma_16816(sc[P & 1], KA[P].z, KB[P].z, KA[P].w, KB[P].w, qf[P].z, qf[P].w);
+      }
+      // V of the same rows, loaded while the scores finish
+      const unsigned char* va = vt + (vA ? rA : 0) * ROWB;
+      const unsigned char* vb = vt + (vB ? rB : 0) * ROWB;
+      uint4 VA[NPB], VB[NPB];
+#pragma unroll
+      for (int P = 0; P < NPB; ++P) {
+        VA[P] = *reinterpret_cast<const uint4*>(va + 64 * P);
+        VB[P] = *reinterpret_cast<const uint4*>(vb + 64 * P);
+      }
+      // raw scores: (rA, hx), (rA, hy), (rB, hx), (rB, hy)
+      float sv[4];
+#pragma unroll
+      for (int e = 0; e < 4; ++e) sv[e] = sc[0][e] + sc[1][e];
+      if (rm) {
+        // retrieval heads' raw scores for the top-k (union index = position here)
+#pragma unroll
+        for (int e = 0; e < 2; ++e) {
+          const int h = 2 * t + e;
+          if (h < G && ((rm >> h) & 1u)) {
+            float* lg = p.logits + (size_t)(b * p.Hq + h0 + h) * p.N_max + (size_t)c * kChunk + t0;
+            if (vA) lg[rA] = sv[e];
+            if (vB) lg[rB] = sv[2 + e];
+          }
+        }
+      }
+      const uint32_t mkA = vA ? (masked ? lane_heads(rA) : lane_all) : 0u;
+      const uint32_t mkB = vB ? (masked ? lane_heads(rB) : lane_all) : 0u;
+      sv[0] = (mkA & 1u) ? sv[0] : -INFINITY;
+      sv[1] = (mkA & 2u) ? sv[1] : -INFINITY;
+      sv[2] = (mkB & 1u) ? sv[2] : -INFINITY;
+      sv[3] = (mkB & 2u) ? sv[3] : -INFINITY;
+      // ---- online softmax per head, lazy maximum (warp-uniform branch)
+      float mx[2] = {fmaxf(sv[0], sv[2]), fmaxf(sv[1], sv[3])};
+#pragma unroll
+      for (int o2 = 4; o2 < 32; o2 <<= 1) {
+        mx[0] = fmaxf(mx[0], __shfl_xor_sync(kFull, mx[0], o2));
+        mx[1] = fmaxf(mx[1], __shfl_xor_sync(kFull, mx[1], o2));
+      }
+      if (__any_sync(kFull, mx[0] > mth[0] || mx[1] > mth[1])) {
+        float al[2];
+#pragma unroll
+        for (int e = 0; e < 2; ++e) {
+          const float mn = mx[e] > mth[e] ? mx[e] : m[e];
+          al[e] = (mn == m[e]) ? 1.f : fast_exp2((m[e] - mn) * sl);   // 0 while m is -inf
+          l[e] *= al[e];
+          m[e] = mn;
+          mth[e] = (mn == -INFINITY) ? -INFINITY : mn + lazy;
+          msl[e] = (mn == -INFINITY) ? 0.f : mn * sl;
+        }
+#pragma unroll
+        for (int k = 0; k < 2 * NPB; ++k) {
+          o[k][0] *= al[0];
+          o[k][2] *= al[0];
+          o[k][1] *= al[1];
+          o[k][3] *= al[1];
+        }
+      }
+      const uint32_t pa = pack_bf16(fast_exp2(fmaf(sv[0], sl, -msl[0])),
+                                    fast_exp2(fmaf(sv[1], sl, -msl[1])));
+      const uint32_t pb = pack_bf16(fast_exp2(fmaf(sv[2], sl, -msl[0])),
+                                    fast_exp2(fmaf(sv[3], sl, -msl[1])));
+      {
+        const float2 fa = bf16x2_to_float2(pa), fb = bf16x2_to_float2(pb);
+        l[0] += fa.x + fb.x;
+        l[1] += fa.y + fb.y;
+      }
+      // P as the B operand (rows x heads), then O^T += V^T P per 16 dimensions
+      const uint32_t b0 = transpose8x8(pa), b1 = transpose8x8(pb);
+#pragma unroll
+      for (int P = 0; P < NPB; ++P) {
+#pragma unroll
+        for (int jp = 0; jp < 2; ++jp) {
+          const uint32_t x0 = transpose8x8(word_of(VA[P], 2 * jp));
+          const uint32_t x1 = transpose8x8(word_of(VA[P], 2 * jp + 1));
+          const uint32_t y0 = transpose8x8(word_of(VB[P], 2 * jp));
+          const uint32_t y1 = transpose8x8(word_of(VB[P], 2 * jp + 1));
+          mma_16816(o[2 * P + jp], x0, x1, y0, y1, b0, b1);
+        }
+      }
+    }
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&empty[s]);
+    if (++s == STAGES) {
+      s = 0;
+      ph ^= 1u;
+    }
+
+    if (flags & kLast) {
+      if (lane == 0) mbar_arrive(&freeb[buf]);   // done with this item's buffer
+      // the warp's state for each head of the group: l summed over the rows
+      // (lanes g), acc held once (block 2P + jp, rows g / g + 8 of O^T are
+      // dimensions 32P + 8(g/2) + 4jp + (g%2) and that + 2)
+#pragma unroll
+      for (int o2 = 4; o2 < 32; o2 <<= 1) {
+        l[0] += __shfl_xor_sync(kFull, l[0], o2);
+        l[1] += __shfl_xor_sync(kFull, l[1], o2);
+      }
+#pragma unroll
+      for (int e = 0; e < 2; ++e) {
+        const int h = 2 * t + e;
+        if (h < G) {
+          const size_t ps = ((size_t)(b * p.Hq + h0 + h) * p.nchunk + c) * kPartSlots + warp;
+          float* dst = p.part_acc + ps * D + 8 * (g >> 1) + (g & 1);
+#pragma unroll
+          for (int P = 0; P < NPB; ++P)
+#pragma unroll
+            for (int jp = 0; jp < 2; ++jp) {
+              dst[32 * P + 4 * jp] = o[2 * P + jp][e];
+              dst[32 * P + 4 * jp + 2] = o[2 * P + jp][2 + e];
+            }
+          if (g == 0) *reinterpret_cast<float2*>(p.part_ml + ps * 2) = make_float2(m[e], l[e]);
+        }
+      }
+    }
+  }
+}
+
 template <typename T, int D, int G, int NW, int NP, int TT, int STAGES>
 cudaError_t launch_attn_t(const AttnParams& p, int num_sms, cudaStream_t st) {
   using C = AttnCfg<T, D, G, NW, NP, TT, STAGES>;
@@ -862,7 +1145,7 @@ cudaError_t launch_attn_t(const AttnParams& p, int num_sms, cudaStream_t st) {
     cudaError_t e =
         cudaFuncSetAttribute(kfn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)C::SMEM);
     if (e != cudaSuccess) return e;
-    if (ilp_of<T, D>() > 1 && LYCHEE_ATTN_REGSPLIT) {
+    if (!C::MMA && ilp_of<T, D>() > 1 && LYCHEE_ATTN_REGSPLIT) {
       // the register split assumes 128 registers per thread at launch
       cudaFuncAttributes fa{};
       e = cudaFuncGetAttributes(&fa, kfn);
@@ -881,6 +1164,10 @@ cudaError_t launch_attn_t(const AttnParams& p, int num_sms, cudaStream_t st) {
 // warps on each SM sub-partition with up to 128 registers per thread.
 #ifndef LYCHEE_ATTN_NW
 #define LYCHEE_ATTN_NW 12
+#endif
+// tensor-core consumers: far fewer instructions per row, so fewer warps
+#ifndef LYCHEE_ATTN_NW_MMA
+#define LYCHEE_ATTN_NW_MMA 4
 #endif
 #ifndef LYCHEE_ATTN_NP
 #define LYCHEE_ATTN_NP 4
@@ -914,7 +1201,7 @@ constexpr int ring_stages() {
 
 template <typename T, int D, int G>
 cudaError_t launch_attn_g(const AttnParams& p, int num_sms, cudaStream_t st) {
-  constexpr int NW = LYCHEE_ATTN_NW, NP = LYCHEE_ATTN_NP;
+  constexpr int NW = mma_path<T>() ? LYCHEE_ATTN_NW_MMA : LYCHEE_ATTN_NW, NP = LYCHEE_ATTN_NP;
   constexpr int TT = tile_rows<T, D>();
   constexpr int STAGES = ring_stages<T, D, G, NW, NP, TT>();
   static_assert(AttnCfg<T, D, G, NW, NP, TT, STAGES>::SMEM <= 227 * 1024, "shared memory");
