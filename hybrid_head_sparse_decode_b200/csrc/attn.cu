@@ -15,11 +15,13 @@
 // group that uses it (GQA deduplication).
 //
 // CTA layout (persistent, one CTA per SM, items taken from an atomic counter):
-//   * a builder warp claims items and turns each into its row list R, each
-//     sparse head's list of the rows of R it uses (with per-tile offsets), and
-//     a share of the consumer warps for every head proportional to its rows.
-//     It fills two alternating item buffers, so the next item is built while
-//     the current one streams and is consumed.
+//   * a builder warp claims items and turns each into its row list R and
+//     what the consumers need to know which head uses which row: for the
+//     tensor-core consumers each head's membership words of the chunk, for
+//     the fp32 consumers each sparse head's list of the rows of R it uses
+//     (with per-tile offsets) and a share of the consumer warps for every head
+//     proportional to its rows.  It fills two alternating item buffers, so the
+//     next item is built while the current one streams and is consumed.
 //   * streaming warps move each built item through a ring of shared-memory
 //     stages in tiles of TT rows of R.  A dense tile (consecutive positions)
 //     arrives as two 1-D bulk copies (cp.async.bulk) of its K rows and V rows,
@@ -28,22 +30,26 @@
 //     (four rows each, through a tensor map over the cache rows) issued by the
 //     first streaming warp, the rest as 16-byte cp.async by the other streaming
 //     warps (whole 32-byte sectors either way).  No copy uses multicast.
-//   * NW consumer warps: during an item each warp serves one head and only
-//     that head's rows (pairs (row, head)), so a sparse head costs work in
-//     proportion to its own set, not to the group's union.  Four lanes share a
-//     pair, each holding a quarter of q (fp32 registers) and of the output
-//     accumulator; eight pairs are in flight per warp.  q.K: K widened from
-//     bf16 in registers, packed fp32x2 FMA, two shuffles to finish the dot
-//     product.  Online softmax per pair slot with a lazy maximum: the running
-//     maximum moves only when a score exceeds it by 2^8 in probability, so the
-//     accumulator is rarely rescaled.  P.V on the same lanes and rows.  At the
-//     end of an item a warp merges its eight slots with shuffles and writes one
-//     partial state (m, l, acc[d]) to its own slot of the workspace; the
-//     combine kernel merges the warps and chunks in a fixed order, so the
-//     result does not depend on scheduling and no warp waits for another.
-// Tensor cores are not used: per K/V row a group does at most 4 * 2d FMAs
-// against 2d * sizeof(T) bytes -- a batched GEMV that HBM, not math, bounds.
-//
+//   * NW consumer warps, in one of two forms.
+//     - bf16 caches (consumer_loop_mma): a warp takes whole slabs of 16 rows
+//       and serves every head of the group on them at once on the tensor cores
+//       (mma.sync m16n8k16, bf16 operands, fp32 accumulation): S^T = K q^T for
+//       the slab, scores of rows a head does not use set to -inf from the
+//       heads' membership words, an online softmax per head with a lazy
+//       maximum, O^T += V^T P with P rounded to bf16.  A row of the union
+//       costs the same few instructions whichever heads use it, so the warps
+//       keep pace with HBM; the arithmetic is a skinny GEMM (at most 8 heads
+//       wide) that the warp-level MMA serves without any staging.
+//     - fp32 caches (consumer_loop): during an item each warp serves one head
+//       and only that head's rows (pairs (row, head)).  Four lanes share a
+//       pair, each holding a quarter of q (fp32 registers) and of the output
+//       accumulator; eight pairs are in flight per warp.  q.K with packed
+//       fp32x2 FMA and two shuffles to finish the dot product, the same lazy
+//       online softmax per pair slot, P.V on the same lanes and rows.
+//     At the end of an item each warp writes its partial state (m, l, acc[d])
+//     for each head it served to its own slot of the workspace; the combine
+//     kernel merges the warps and chunks in a fixed order, so the result does
+//     not depend on scheduling and no warp waits for another.
 // Logits of retrieval heads (raw q.k in fp32, not divided by sqrt(d)) are
 // written to the workspace for the top-k kernel.
 #include <type_traits>
@@ -1012,12 +1018,12 @@ __device__ __forceinline__ void consumer_loop_mma(const AttnParams& p, unsigned 
         KA[P] = *reinterpret_cast<const uint4*>(ka + 64 * P);
         KB[P] = *reinterpret_cast<const uint4*>(kb + 64 * P);
       }
-      // ---- S^T = K q^T (two accumulation chains)
-      float sc[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+      // ---- S^T = K q^T (four accumulation chains)
+      float sc[4][4] = {};
 #pragma unroll
       for (int P = 0; P < NPB; ++P) {
-        mma_16816(sc[P & 1], KA[P].x, KB[P].x, KA[P].y, KB[P].y, qf[P].x, qf[P].y);
-        mma_16816(sc[P & 1], KA[P].z, KB[P].z, KA[P].w, KB[P].w, qf[P].z, qf[P].w);
+        mma_16816(sc[(2 * P) & 3], KA[P].x, KB[P].x, KA[P].y, KB[P].y, qf[P].x, qf[P].y);
+        mma_16816(sc[(2 * P + 1) & 3], KA[P].z, KB[P].z, KA[P].w, KB[P].w, qf[P].z, qf[P].w);
       }
       // V of the same rows, loaded while the scores finish
       const unsigned char* va = vt + (vA ? rA : 0) * ROWB;
@@ -1031,7 +1037,7 @@ __device__ __forceinline__ void consumer_loop_mma(const AttnParams& p, unsigned 
       // raw scores: (rA, hx), (rA, hy), (rB, hx), (rB, hy)
       float sv[4];
 #pragma unroll
-      for (int e = 0; e < 4; ++e) sv[e] = sc[0][e] + sc[1][e];
+      for (int e = 0; e < 4; ++e) sv[e] = (sc[0][e] + sc[2][e]) + (sc[1][e] + sc[3][e]);
       if (rm) {
         // retrieval heads' raw scores for the top-k (union index = position here)
 #pragma unroll
