@@ -39,7 +39,7 @@ lychee_status check_shape(const lychee_shape* s) {
   if (s->Hq > kMaxHq) return LYCHEE_ERR_UNSUPPORTED;
   if (s->d != 64 && s->d != 128) return LYCHEE_ERR_UNSUPPORTED;
   if (s->N_max > (1 << 24)) return LYCHEE_ERR_UNSUPPORTED;
-  const long long nchunk = (s->N_max + kChunk - 1) / kChunk;
+  const long long nchunk = (s->N_max + kChunkMin - 1) / kChunkMin;
   if ((long long)s->B * s->Hkv * nchunk >= (1LL << 31)) return LYCHEE_ERR_UNSUPPORTED;
   if ((long long)s->B * s->Hq >= (1LL << 24)) return LYCHEE_ERR_UNSUPPORTED;
   return LYCHEE_OK;
@@ -47,7 +47,7 @@ lychee_status check_shape(const lychee_shape* s) {
 
 Layout layout_of(const lychee_shape* s) {
   Layout L{};
-  L.nchunk = (s->N_max + kChunk - 1) / kChunk;
+  L.nchunk = (s->N_max + kChunkMin - 1) / kChunkMin;   // room for the shortest chunk
   L.nwords = (s->N_max + 31) / 32;
   const size_t bh = (size_t)s->B * s->Hq;
   size_t off = sizeof(WsHeader);
@@ -193,6 +193,25 @@ struct Ctx {
   WsHeader* hdr() const { return reinterpret_cast<WsHeader*>(ws); }
 };
 
+// Positions per attention work item: among the multiples of 32 in
+// [kChunkMin, kChunk], the one that minimises the work of the busiest SM for
+// full-length sequences, (items per SM, rounded up) x positions per item;
+// ties go to the longer chunk (fewer partial states).  Items are claimed
+// dynamically, so this only evens out the last wave.
+int pick_chunk(const lychee_shape* s, int sms) {
+  int best = kChunk;
+  long long best_cost = -1;
+  for (int cs = kChunk; cs >= kChunkMin; cs -= 32) {
+    const long long items = (long long)s->B * s->Hkv * ((s->N_max + cs - 1) / cs);
+    const long long cost = (items + sms - 1) / sms * cs;
+    if (best_cost < 0 || cost < best_cost) {
+      best_cost = cost;
+      best = cs;
+    }
+  }
+  return best;
+}
+
 // One layer's launches.  bitmaps carry the sets of sparse heads in and (when
 // write_bits) the sets of retrieval heads out.
 lychee_status run_layer(const Ctx& c, const void* q, const void* kc, const void* vc,
@@ -243,7 +262,9 @@ lychee_status run_layer(const Ctx& c, const void* q, const void* kc, const void*
   ap.exits = &c.hdr()->counters[1];
   ap.B = s->B; ap.Hq = Hq; ap.Hkv = s->Hkv; ap.N_max = s->N_max;
   ap.nwords = c.L.nwords; ap.nchunk = c.L.nchunk;
-  ap.n_items = s->B * s->Hkv * c.L.nchunk;
+  ap.chunk = pick_chunk(s, c.sms);
+  ap.nchunk_run = (s->N_max + ap.chunk - 1) / ap.chunk;
+  ap.n_items = s->B * s->Hkv * ap.nchunk_run;
   ap.scale_log2 = (float)(1.4426950408889634 / std::sqrt((double)s->d));
   fill_roles(ap.role, role, Hq);
   ap.gather_tma = !tma_gathers_disabled() && encode_row_map(&ap.tmk, kc, s) &&
@@ -270,6 +291,7 @@ lychee_status run_layer(const Ctx& c, const void* q, const void* kc, const void*
   cp.out = out;
   cp.err = err;
   cp.B = s->B; cp.Hq = Hq; cp.N_max = s->N_max; cp.nchunk = c.L.nchunk;
+  cp.chunk = ap.chunk;
   cp.scale_log2 = ap.scale_log2;
   e = timed(nr > 0 ? kKindTopkCombine : kKindCombine, c.st,
             [&] { return launch_topk_combine(tp, cp, s->dtype, s->d, c.st); });

@@ -320,7 +320,7 @@ __global__ void __launch_bounds__((NW + NP) * 32, 1)
     for (int b0 = 0; b0 < B; b0 += 32) {
       const int b = b0 + lane;
       const int n = b < B ? min(max(__ldg(&p.seqlens[b]), 1), N_max) : 0;
-      const int nc = (n + kChunk - 1) / kChunk;
+      const int nc = (n + p.chunk - 1) / p.chunk;
       int incl = nc;
 #pragma unroll
       for (int o = 1; o < 32; o <<= 1) {
@@ -353,10 +353,10 @@ __global__ void __launch_bounds__((NW + NP) * 32, 1)
       for (int t = 0; t < G; ++t) w[t] = 0u;
       if (item >= n_items) return;
       int b, c, g;
-      decode_item(item, compact, cum, B, Hkv, p.nchunk, b, c, g);
+      decode_item(item, compact, cum, B, Hkv, p.nchunk_run, b, c, g);
       nraw = __ldg(&p.seqlens[b]);
-      const int word = c * (kChunk / 32) + lane;
-      if (lane < kChunk / 32 && word < p.nwords) {
+      const int word = c * (p.chunk / 32) + lane;
+      if (lane < p.chunk / 32 && word < p.nwords) {
         const size_t wbase = (size_t)(b * Hq + g * G) * p.nwords + word;
 #pragma unroll
         for (int t = 0; t < G; ++t) w[t] = __ldg(&p.bitmaps[wbase + (size_t)t * p.nwords]);
@@ -387,9 +387,9 @@ __global__ void __launch_bounds__((NW + NP) * 32, 1)
           total = -1;
           break;
         }
-        decode_item(cur, compact, cum, B, Hkv, p.nchunk, b, c, g);
+        decode_item(cur, compact, cum, B, Hkv, p.nchunk_run, b, c, g);
         const int n = min(max(cur_n, 1), N_max);
-        p0 = c * kChunk;
+        p0 = c * p.chunk;
         const int h0 = g * G;
         // claim and load the item after this one while this one is built
         int nxt_n = 1;
@@ -398,7 +398,7 @@ __global__ void __launch_bounds__((NW + NP) * 32, 1)
         prefetch(nxt, nxt_n, nxt_w);
         claimed = claim();
         if (p0 < n) {
-          const int p1 = min(p0 + kChunk, n);
+          const int p1 = min(p0 + p.chunk, n);
           rmask = 0;
 #pragma unroll
           for (int t = 0; t < G; ++t) rmask |= ((p.role[(h0 + t) >> 5] >> ((h0 + t) & 31)) & 1u) << t;
@@ -433,7 +433,7 @@ __global__ void __launch_bounds__((NW + NP) * 32, 1)
           }
           if constexpr (C::MMA) {
             // the heads' membership words (a retrieval head's: every valid row)
-            if (lane < kChunk / 32) {
+            if (lane < p.chunk / 32) {
               uint32_t hv[8];
 #pragma unroll
               for (int t = 0; t < 8; ++t) hv[t] = t < G ? bits[t] : 0u;
@@ -710,7 +710,7 @@ __device__ __forceinline__ void consumer_loop(const AttnParams& p, unsigned char
         nh = ib[C::IB_ASG + NW + myh];
         ident = (i1.y >> myh) & 1;
         lg_on = ident && pp == 0;
-        lg = p.logits + (size_t)(b * p.Hq + h0 + myh) * p.N_max + (size_t)c * kChunk;
+        lg = p.logits + (size_t)(b * p.Hq + h0 + myh) * p.N_max + (size_t)c * p.chunk;
         const unsigned char* qs = smem + C::OFF_Q + s * C::QSTRIDE + myh * ROWB;
 #pragma unroll
         for (int cc = 0; cc < CPL; ++cc) {
@@ -997,7 +997,7 @@ __device__ __forceinline__ void consumer_loop_mma(const AttnParams& p, unsigned 
     // bit 0 / 1: head hx / hy uses union row r of this tile (a group with a
     // retrieval head reads every position of the chunk in order)
     auto lane_heads = [&](int r) -> uint32_t {
-      const int po = rm ? t0 + r : lpos[r] - c * kChunk;
+      const int po = rm ? t0 + r : lpos[r] - c * p.chunk;
       const uint2 w = *reinterpret_cast<const uint2*>(hw + (po >> 5) * 8);
       return ((w.x >> (po & 31)) & 1u) | (((w.y >> (po & 31)) & 1u) << 1);
     };
@@ -1044,7 +1044,7 @@ __device__ __forceinline__ void consumer_loop_mma(const AttnParams& p, unsigned 
         for (int e = 0; e < 2; ++e) {
           const int h = 2 * t + e;
           if (h < G && ((rm >> h) & 1u)) {
-            float* lg = p.logits + (size_t)(b * p.Hq + h0 + h) * p.N_max + (size_t)c * kChunk + t0;
+            float* lg = p.logits + (size_t)(b * p.Hq + h0 + h) * p.N_max + (size_t)c * p.chunk + t0;
             if (vA) lg[rA] = sv[e];
             if (vB) lg[rB] = sv[2 + e];
           }

@@ -114,7 +114,7 @@ __device__ __forceinline__ void combine_body(const CombineParams& p, int cta, un
   const int b = bh / p.Hq;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int n = min(max(p.seqlens[b], 1), p.N_max);
-  const int nc = (n + kChunk - 1) / kChunk;
+  const int nc = (n + p.chunk - 1) / p.chunk;
   const int cps = (nc + kCombineSplit - 1) / kCombineSplit;
   const int c_lo = min(nc, sp * cps), c_hi = min(nc, c_lo + cps);
   const float2* ml = reinterpret_cast<const float2*>(p.part_ml) + (size_t)bh * p.nchunk * kPartSlots;

@@ -29,7 +29,8 @@ struct WsHeader {
 };
 static_assert(sizeof(WsHeader) == 256, "header is 256 bytes");
 
-constexpr int kChunk = 960;           // positions per attention work item (30 words)
+constexpr int kChunk = 960;           // positions per attention work item, at most (30 words)
+constexpr int kChunkMin = 768;        // ... and at least (the host picks one per launch)
 constexpr int kPartSlots = 12;        // partial states per (sequence, head, chunk): one per warp
 constexpr int kMaxHq = 128;           // query heads supported
 constexpr uint64_t kWaitLimitNs = 2000000000ull;   // 2 s: a wait this long is a fault

@@ -23,6 +23,8 @@ struct AttnParams {
   uint32_t* counter;        // work-item counter, 0 at launch, 0 again at exit
   uint32_t* exits;          // CTAs that finished, 0 at launch, 0 again at exit
   int B, Hq, Hkv, N_max, nwords, nchunk, n_items;
+  int chunk;                // positions per work item (multiple of 32, kChunkMin..kChunk)
+  int nchunk_run;           // chunks of N_max at that length (<= nchunk, the partials' stride)
   float scale_log2;         // log2(e) / sqrt(D)
   uint32_t role[4];         // bit h set: head h is a retrieval head
   int gather_tma;           // 1: sparse rows are gathered through tmk / tmv
@@ -55,7 +57,8 @@ struct CombineParams {
   const int32_t* seqlens;    // [B]
   void* out;                 // [B, Hq, D]
   uint32_t* err;
-  int B, Hq, N_max, nchunk;
+  int B, Hq, N_max, nchunk;  // nchunk: the partials' chunk stride
+  int chunk;                 // positions per attention work item
   float scale_log2;
 };
 cudaError_t launch_combine(const CombineParams& p, int dtype, int D, cudaStream_t st);
