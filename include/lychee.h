@@ -125,7 +125,7 @@ LYCHEE_API lychee_status lychee_hybrid_decode_attn(const lychee_shape* s, const 
 
 /* Size of the static device scratch behind lychee_hybrid_decode_attn_noalloc:
  * 64 MiB per device, enough for a layer whose lychee_workspace_size() is at
- * most that (e.g. B = 1, Hq = 32, d = 128, N_max = 131072 needs about 43 MiB). */
+ * most that (e.g. B = 1, Hq = 32, d = 128, N_max = 131072 needs about 49 MiB). */
 #define LYCHEE_NOALLOC_SCRATCH_BYTES (64u << 20)
 
 /* lychee_hybrid_decode_attn without a caller-owned workspace and without any
