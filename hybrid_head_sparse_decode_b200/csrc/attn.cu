@@ -102,6 +102,10 @@ constexpr int kConsRegs = LYCHEE_ATTN_CONS_REGS;
 #ifndef LYCHEE_ATTN_TMA_ROWS
 #define LYCHEE_ATTN_TMA_ROWS 8
 #endif
+// ... with the tensor-core consumers (more streaming warps share the 16-byte copies)
+#ifndef LYCHEE_ATTN_TMA_ROWS_MMA
+#define LYCHEE_ATTN_TMA_ROWS_MMA 6
+#endif
 // bf16 caches: consumer warps contract on the tensor cores (mma.sync, see
 // consumer_loop_mma); 0: the fp32-FMA consumer for every type.
 #ifndef LYCHEE_ATTN_MMA
@@ -159,6 +163,7 @@ struct AttnCfg {
   static_assert(CPL >= 2 && DL % E == 0 && CPL % 2 == 0, "lane mapping");
   static_assert(TT % kPairsPerBatch == 0 && TT % 4 == 0 && TT <= 255, "tile rows");
   static constexpr bool MMA = mma_path<T>();
+  static constexpr int TMA_ROWS = MMA ? LYCHEE_ATTN_TMA_ROWS_MMA : LYCHEE_ATTN_TMA_ROWS;
   static_assert(MMA ? (G <= 8 && NW <= kPartSlots && TT % 16 == 0)
                     : (G <= NW && NW <= kPartSlots && NW <= 16),
                 "warps per head fit the partial slots; tensor-core slabs of 16 rows");
@@ -516,7 +521,7 @@ __global__ void __launch_bounds__((NW + NP) * 32, 1)
     // ------------------------------------------------------ streaming warps
     const int sw = warp == NW ? 0 : warp - NW - 1;   // 0: publishes tiles, bulk copies
     const uint64_t pol = l2_evict_first_policy();
-    const bool tma_rows = LYCHEE_ATTN_TMA_ROWS > 0 && NS > 1 && p.gather_tma != 0;
+    const bool tma_rows = C::TMA_ROWS > 0 && NS > 1 && p.gather_tma != 0;
     uint32_t s = 0, ph = 0;                // ring stage and its phase parity
     bool ok = true;
     for (uint32_t it = 0;; ++it) {
@@ -556,7 +561,7 @@ __global__ void __launch_bounds__((NW + NP) * 32, 1)
         // when it ends the tile), rows [nt, nrows) by 16-byte copies
         const int nt = !gather || !tma_rows
                            ? 0
-                           : (nrows <= 4 ? nrows : ((nrows * LYCHEE_ATTN_TMA_ROWS) >> 4) & ~3);
+                           : (nrows <= 4 ? nrows : ((nrows * C::TMA_ROWS) >> 4) & ~3);
         const int ngrp = (nt + 3) >> 2;
         const int csw = tma_rows ? sw - 1 : sw, ncs = tma_rows ? NS - 1 : NS;
         if (gather && csw >= 0) {
@@ -1166,14 +1171,19 @@ cudaError_t launch_attn_t(const AttnParams& p, int num_sms, cudaStream_t st) {
   return cudaGetLastError();
 }
 
-// 16 warps per CTA: NW consumers and NP producers (builder, streaming warps), 4
-// warps on each SM sub-partition with up to 128 registers per thread.
+// fp32 caches: 16 warps per CTA, NW consumers and NP producers (builder,
+// streaming warps), 4 warps on each SM sub-partition with up to 128 registers
+// per thread.
 #ifndef LYCHEE_ATTN_NW
 #define LYCHEE_ATTN_NW 12
 #endif
-// tensor-core consumers: far fewer instructions per row, so fewer warps
+// tensor-core consumers: far fewer instructions per row, so fewer consumer
+// warps and more streaming warps (a builder and seven streaming warps)
 #ifndef LYCHEE_ATTN_NW_MMA
 #define LYCHEE_ATTN_NW_MMA 4
+#endif
+#ifndef LYCHEE_ATTN_NP_MMA
+#define LYCHEE_ATTN_NP_MMA 8
 #endif
 #ifndef LYCHEE_ATTN_NP
 #define LYCHEE_ATTN_NP 4
@@ -1207,7 +1217,8 @@ constexpr int ring_stages() {
 
 template <typename T, int D, int G>
 cudaError_t launch_attn_g(const AttnParams& p, int num_sms, cudaStream_t st) {
-  constexpr int NW = mma_path<T>() ? LYCHEE_ATTN_NW_MMA : LYCHEE_ATTN_NW, NP = LYCHEE_ATTN_NP;
+  constexpr int NW = mma_path<T>() ? LYCHEE_ATTN_NW_MMA : LYCHEE_ATTN_NW;
+  constexpr int NP = mma_path<T>() ? LYCHEE_ATTN_NP_MMA : LYCHEE_ATTN_NP;
   constexpr int TT = tile_rows<T, D>();
   constexpr int STAGES = ring_stages<T, D, G, NW, NP, TT>();
   static_assert(AttnCfg<T, D, G, NW, NP, TT, STAGES>::SMEM <= 227 * 1024, "shared memory");
