@@ -69,9 +69,11 @@ def _load():
         vp, ip = ctypes.c_void_p, ctypes.c_int
         lib.oracle_topk.argtypes = [vp, ip, ip, ip, vp]
         lib.oracle_topk.restype = ip
-        lib.oracle_hybrid_layer.argtypes = [ip] * 7 + [vp] * 10 + [ip]
+        lib.oracle_block_select.argtypes = [vp, ip, ip, ip, ip, vp]
+        lib.oracle_block_select.restype = ip
+        lib.oracle_hybrid_layer.argtypes = [ip] * 8 + [vp] * 10 + [ip]
         lib.oracle_hybrid_layer.restype = ip
-        lib.oracle_stack.argtypes = [ip] * 8 + [vp] * 9 + [ip]
+        lib.oracle_stack.argtypes = [ip] * 9 + [vp] * 9 + [ip]
         lib.oracle_stack.restype = ip
         lib.oracle_attention_weights.argtypes = [ip, ip, ip, vp, vp, vp]
         lib.oracle_attention_weights.restype = ip
@@ -108,6 +110,18 @@ def topk(s: np.ndarray, k: int, cap: int | None = None) -> np.ndarray:
     return out
 
 
+def block_select(s: np.ndarray, kb: int, block: int, cap: int) -> np.ndarray:
+    """Block-granular selection: blocks of ``block`` positions scored by their
+    largest score, the max(1, kb // block) best blocks (ties: lower block index)
+    taken whole; their positions in ascending order, padded with -1 to ``cap``."""
+    s = np.ascontiguousarray(s, dtype=np.float64)
+    out = np.empty(cap, dtype=np.int32)
+    rc = _load().oracle_block_select(_p(s), int(s.size), int(kb), int(block), int(cap), _p(out))
+    if rc < 0:
+        raise OracleError(rc, "block_select")
+    return out
+
+
 def attention_weights(q: np.ndarray, Kg: np.ndarray) -> np.ndarray:
     """A = softmax(q Kg^T / sqrt(d)) for one query head over all rows of Kg [n, d]."""
     dt = _dtype_code(q)
@@ -122,9 +136,10 @@ def attention_weights(q: np.ndarray, Kg: np.ndarray) -> np.ndarray:
 
 
 def hybrid_layer(q, K, V, seqlens, role, idx_in, k, k_per_seq=None, want_logits=False,
-                 nthreads=0):
+                 nthreads=0, block=1):
     """One hybrid-head layer.  Returns (out [B,Hq,d] f64, idx_out [B,Hq,k] i32,
-    logits [B,Hq,N_max] f64 or None).  Raises OracleError on a bad index or shape."""
+    logits [B,Hq,N_max] f64 or None).  block > 1: retrieval heads select whole
+    blocks of that many positions.  Raises OracleError on a bad index or shape."""
     dt = _dtype_code(q)
     q = np.ascontiguousarray(q)
     K = np.ascontiguousarray(K)
@@ -138,7 +153,7 @@ def hybrid_layer(q, K, V, seqlens, role, idx_in, k, k_per_seq=None, want_logits=
     out = np.zeros((B, Hq, d), dtype=np.float64)
     idx_out = np.full((B, Hq, k), -1, dtype=np.int32)
     logits = np.full((B, Hq, N_max), np.nan, dtype=np.float64) if want_logits else None
-    rc = _load().oracle_hybrid_layer(B, Hq, Hkv, d, N_max, int(k), dt, _p(q), _p(K), _p(V),
+    rc = _load().oracle_hybrid_layer(B, Hq, Hkv, d, N_max, int(k), dt, int(block), _p(q), _p(K), _p(V),
                                      _p(seqlens), _p(kps), _p(role), _p(idx_in), _p(out),
                                      _p(logits), _p(idx_out), int(nthreads))
     if rc:
@@ -146,7 +161,7 @@ def hybrid_layer(q, K, V, seqlens, role, idx_in, k, k_per_seq=None, want_logits=
     return out, idx_out, logits
 
 
-def stack(q, Ks, Vs, seqlens, roles, k, k_per_seq=None, want_layers=False, nthreads=0):
+def stack(q, Ks, Vs, seqlens, roles, k, k_per_seq=None, want_layers=False, nthreads=0, block=1):
     """L chained layers.  q [L,B,Hq,d]; Ks/Vs: lists of L arrays [B,Hkv,N_max,d];
     roles [L,Hq].  Returns (out [L,B,Hq,d] f64, idx_final [B,Hq,k],
     idx_layers [L,B,Hq,k] or None)."""
@@ -164,7 +179,7 @@ def stack(q, Ks, Vs, seqlens, roles, k, k_per_seq=None, want_layers=False, nthre
     out = np.zeros((L, B, Hq, d), dtype=np.float64)
     idx_final = np.full((B, Hq, k), -1, dtype=np.int32)
     idx_layers = np.full((L, B, Hq, k), -1, dtype=np.int32) if want_layers else None
-    rc = _load().oracle_stack(L, B, Hq, Hkv, d, N_max, int(k), dt, _p(q),
+    rc = _load().oracle_stack(L, B, Hq, Hkv, d, N_max, int(k), dt, int(block), _p(q),
                               ctypes.cast(kptr, ctypes.c_void_p),
                               ctypes.cast(vptr, ctypes.c_void_p), _p(seqlens), _p(kps),
                               _p(roles), _p(out), _p(idx_layers), _p(idx_final), int(nthreads))

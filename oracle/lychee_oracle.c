@@ -30,6 +30,14 @@
  *   - GQA: query head h reads KV head floor(h / G), G = Hq / Hkv.
  *   - A sparse head reads its own layer's K/V at the inherited positions; only
  *     the index set is shared between layers.
+ *   - A set row ends at its first -1 (at most k_b entries are read), so a set
+ *     may hold fewer than k_b positions; a head with an empty set outputs 0.
+ *   - Block-granular selection (the block-sparse decoding kernel of the same
+ *     page; the block-level maximum scores and the k/B top blocks of the
+ *     HySparse page, B = 64): a block's score is the largest logit among its
+ *     positions, the max(1, floor(k_b / B)) best blocks (ties: lower block
+ *     index) are taken whole, and the set lists their positions in ascending
+ *     order.  Selected when the caller passes block = B > 1.
  *
  * All arithmetic is fp64.  Inputs are bf16 (raw 16-bit patterns) or fp32 and are
  * widened exactly to double when read.  The only parallelism is an optional
@@ -148,12 +156,56 @@ int oracle_topk(const double *s, int n, int k, int cap, int32_t *idx) {
   return kk;
 }
 
+/* Block-granular argsTopK: blocks [B c, min(B c + B, n)) scored by their largest
+ * s_j; the kblk = max(1, floor(kb / B)) blocks ranked first by (larger score,
+ * then lower block index) are taken whole.  idx[0:m] = their positions in
+ * ascending order, idx[m:cap] = -1.  Returns m, or a negative code (the set
+ * must fit in cap). */
+int oracle_block_select(const double *s, int n, int kb, int block, int cap, int32_t *idx) {
+  if (n < 1 || block < 1 || kb < 1) return OR_EARG;
+  int nblk = (n + block - 1) / block;
+  int kblk = kb / block;
+  if (kblk < 1) kblk = 1;
+  if (kblk > nblk) kblk = nblk;
+  double *bs = (double *)calloc((size_t)nblk, sizeof(double));
+  int32_t *sel = (int32_t *)malloc(sizeof(int32_t) * (size_t)nblk);
+  int m = 0, rc = OR_OK;
+  if (!bs || !sel) {
+    rc = OR_ENOMEM;
+    goto done;
+  }
+  for (int c = 0; c < nblk; ++c) {
+    double best = -INFINITY;
+    for (int j = c * block; j < n && j < (c + 1) * block; ++j)
+      if (s[j] > best) best = s[j];
+    bs[c] = best;
+  }
+  if (oracle_topk(bs, nblk, kblk, nblk, sel) < 0) {
+    rc = OR_ENOMEM;
+    goto done;
+  }
+  for (int i = 0; i < kblk; ++i)
+    for (int j = sel[i] * block; j < n && j < (sel[i] + 1) * block; ++j) {
+      if (m >= cap) {
+        rc = OR_EARG;
+        goto done;
+      }
+      idx[m++] = j;
+    }
+  for (int t = m; t < cap; ++t) idx[t] = -1;
+done:
+  free(bs);
+  free(sel);
+  return rc ? rc : m;
+}
+
 /* ---- one head ------------------------------------------------------------ */
 
 /* Full (retrieval) attention of query head h of sequence b over rows [0, n).
- * out[d]; s_all[n] receives the logits (may be NULL); idx_out[cap] the top-k set. */
+ * out[d]; s_all[n] receives the logits (may be NULL); idx_out[cap] the top-k set
+ * (block > 1: the block-granular set). */
 static int retrieval_head(const void *q, size_t q_off, const void *K, const void *V,
-                          size_t kv_off, int n, int d, int dt, int kb, int cap,
+                          size_t kv_off, int n, int d, int dt, int kb, int cap, int block,
                           double *out, double *s_all, int32_t *idx_out) {
   int32_t *rows = (int32_t *)malloc(sizeof(int32_t) * (size_t)n);
   double *s = (double *)malloc(sizeof(double) * (size_t)n);
@@ -168,7 +220,11 @@ static int retrieval_head(const void *q, size_t q_off, const void *K, const void
   double z = softmax_unnormalised(s, n, p);
   weighted_values(p, z, V, kv_off, d, dt, rows, n, out);
   if (s_all) memcpy(s_all, s, sizeof(double) * (size_t)n);
-  if (idx_out && oracle_topk(s, n, kb, cap, idx_out) < 0) rc = OR_ENOMEM;
+  if (idx_out) {
+    const int m = block > 1 ? oracle_block_select(s, n, kb, block, cap, idx_out)
+                            : oracle_topk(s, n, kb, cap, idx_out);
+    if (m < 0) rc = m;
+  }
 done:
   free(rows);
   free(s);
@@ -176,12 +232,24 @@ done:
   return rc;
 }
 
-/* Sparse attention over the first kb entries of S (which must be distinct and
- * in [0, n)).  idx_out (may be NULL) receives S unchanged (all cap entries). */
+/* Sparse attention over S: its entries before the first -1, at most kb of them
+ * (distinct and in [0, n); a non-negative entry after a -1 is an error).  An
+ * empty set gives out = 0.  idx_out (may be NULL) receives S unchanged (all cap
+ * entries). */
 static int sparse_head(const void *q, size_t q_off, const void *K, const void *V,
                        size_t kv_off, int n, int d, int dt, const int32_t *S, int kb,
                        int cap, double *out, int32_t *idx_out) {
   if (kb < 1) return OR_EARG;
+  int kv = 0;
+  while (kv < kb && S[kv] >= 0) ++kv;
+  for (int t = kv; t < kb; ++t)
+    if (S[t] >= 0) return OR_EINDEX;
+  if (kv == 0) {
+    for (int i = 0; i < d; ++i) out[i] = 0.0;
+    if (idx_out) memcpy(idx_out, S, sizeof(int32_t) * (size_t)cap);
+    return OR_OK;
+  }
+  kb = kv;
   unsigned char *seen = (unsigned char *)calloc((size_t)n, 1);
   double *s = (double *)malloc(sizeof(double) * (size_t)kb);
   double *p = (double *)malloc(sizeof(double) * (size_t)kb);
@@ -235,15 +303,17 @@ static int check_shape(int B, int Hq, int Hkv, int d, int N_max, int k, int dt) 
  *   out      [B, Hq, d]   double
  *   logits   [B, Hq, N_max] double or NULL: s_j of retrieval heads for j < n_b
  *   idx_out  [B, Hq, k]             retrieval: top-k set; sparse: idx_in row copied
+ *   block    1: token-level argsTopK; B > 1: block-granular selection (k >= B)
  *   nthreads OpenMP threads over (b, h) pairs (<= 0: library default)
  * Returns OR_OK or a negative code.
  */
-int oracle_hybrid_layer(int B, int Hq, int Hkv, int d, int N_max, int k, int dt,
+int oracle_hybrid_layer(int B, int Hq, int Hkv, int d, int N_max, int k, int dt, int block,
                         const void *q, const void *K, const void *V, const int32_t *seqlens,
                         const int32_t *k_per_seq, const uint8_t *role, const int32_t *idx_in,
                         double *out, double *logits, int32_t *idx_out, int nthreads) {
   int rc = check_shape(B, Hq, Hkv, d, N_max, k, dt);
   if (rc) return rc;
+  if (block < 1 || (block > 1 && k < block)) return OR_EARG;
   for (int b = 0; b < B; ++b)
     if (seqlens[b] < 1 || seqlens[b] > N_max) return OR_EARG;
   int G = Hq / Hkv;
@@ -262,7 +332,7 @@ int oracle_hybrid_layer(int B, int Hq, int Hkv, int d, int N_max, int k, int dt,
     size_t row = (size_t)b * Hq + h;
     int r;
     if (role[h] == OR_ROLE_RETRIEVAL) {
-      r = retrieval_head(q, q_off, K, V, kv_off, n, d, dt, kb, k, out + row * (size_t)d,
+      r = retrieval_head(q, q_off, K, V, kv_off, n, d, dt, kb, k, block, out + row * (size_t)d,
                          logits ? logits + row * (size_t)N_max : NULL,
                          idx_out ? idx_out + row * (size_t)k : NULL);
     } else {
@@ -293,7 +363,7 @@ int oracle_hybrid_layer(int B, int Hq, int Hkv, int d, int N_max, int k, int dt,
  *   idx_layers [L, B, Hq, k] or NULL: S leaving each layer
  *   idx_final  [B, Hq, k]: S leaving layer L-1
  */
-int oracle_stack(int L, int B, int Hq, int Hkv, int d, int N_max, int k, int dt,
+int oracle_stack(int L, int B, int Hq, int Hkv, int d, int N_max, int k, int dt, int block,
                  const void *q, const void *const *Ks, const void *const *Vs,
                  const int32_t *seqlens, const int32_t *k_per_seq, const uint8_t *role,
                  double *out, int32_t *idx_layers, int32_t *idx_final, int nthreads) {
@@ -314,7 +384,7 @@ int oracle_stack(int L, int B, int Hq, int Hkv, int d, int N_max, int k, int dt,
   size_t qsz = (dt == OR_BF16) ? 2 : 4;
   for (int l = 0; l < L && rc == OR_OK; ++l) {
     const char *ql = (const char *)q + (size_t)l * B * Hq * d * qsz;
-    rc = oracle_hybrid_layer(B, Hq, Hkv, d, N_max, k, dt, ql, Ks[l], Vs[l], seqlens, k_per_seq,
+    rc = oracle_hybrid_layer(B, Hq, Hkv, d, N_max, k, dt, block, ql, Ks[l], Vs[l], seqlens, k_per_seq,
                              role + (size_t)l * Hq, cur, out + (size_t)l * B * Hq * d, NULL, nxt,
                              nthreads);
     if (idx_layers) memcpy(idx_layers + (size_t)l * set_elems, nxt, sizeof(int32_t) * set_elems);

@@ -453,3 +453,116 @@ def test_openmp_thread_count_does_not_change_results():
     a = oracle.hybrid_layer(q, K, V, seq, role, idx, 90, nthreads=1)
     b = oracle.hybrid_layer(q, K, V, seq, role, idx, 90, nthreads=4)
     assert np.array_equal(a[0], b[0]) and np.array_equal(a[1], b[1])
+
+
+# ---- block-granular selection (block-sparse decoding: block-level maximum
+# scores, k/B top blocks; pages "LycheeDecode ..." and "HySparse ...") -------
+
+def _block_props(s, kb, blk, sel):
+    """The properties that fix the block selection: every chosen block's score
+    beats every other block's (ties to the lower block index), the set is made of
+    whole blocks (the tail block cut at n), it holds max(1, kb // blk) blocks (at
+    most all of them), and it is ascending with -1 padding."""
+    n = s.size
+    nblk = -(-n // blk)
+    kblk = min(max(1, kb // blk), nblk)
+    score = [max(s[c * blk:min(n, c * blk + blk)]) for c in range(nblk)]
+    m = int((sel >= 0).sum())
+    assert np.all(sel[m:] == -1) and np.all(np.diff(sel[:m]) > 0)
+    chosen = sorted({int(j) // blk for j in sel[:m]})
+    assert len(chosen) == kblk
+    for c in chosen:   # whole blocks
+        assert set(range(c * blk, min(n, c * blk + blk))) <= set(sel[:m].tolist())
+    assert m == sum(min(n, c * blk + blk) - c * blk for c in chosen)
+    others = [c for c in range(nblk) if c not in chosen]
+    for c in chosen:
+        for o in others:
+            assert score[c] > score[o] or (score[c] == score[o] and c < o)
+
+
+@pytest.mark.parametrize("seed", range(40))
+def test_block_select_properties(seed):
+    g = rng(3000 + seed)
+    n = int(g.integers(1, 400))
+    blk = int(g.choice([2, 4, 8, 64]))
+    kb = int(g.integers(1, n + 1))
+    # integer scores make ties between blocks common
+    s = g.integers(-4, 5, n).astype(np.float64) if seed % 2 else g.standard_normal(n)
+    cap = max(kb, blk) + blk
+    sel = oracle.block_select(s, kb, blk, cap)
+    _block_props(s, kb, blk, sel)
+
+
+def test_block_select_of_one_position_blocks_is_token_topk():
+    g = rng(77)
+    for n in (1, 5, 33, 200):
+        s = g.integers(-3, 4, n).astype(np.float64)
+        for kb in (1, n // 2 + 1, n):
+            assert np.array_equal(oracle.block_select(s, kb, 1, n), oracle.topk(s, kb, n))
+
+
+def test_block_select_single_block_takes_everything():
+    s = rng(5).standard_normal(50)
+    sel = oracle.block_select(s, 10, 64, 64)
+    assert np.array_equal(sel[:50], np.arange(50)) and np.all(sel[50:] == -1)
+
+
+def test_block_layer_with_one_position_blocks_equals_token_layer():
+    """The layer in block mode with blocks of one position is the token-level
+    layer, set for set and output for output."""
+    g = rng(8)
+    B, Hq, Hkv, d, N, k = 1, 4, 2, 16, 40, 12
+    q = g.standard_normal((B, Hq, d)).astype(np.float32)
+    K = g.standard_normal((B, Hkv, N, d)).astype(np.float32)
+    V = g.standard_normal((B, Hkv, N, d)).astype(np.float32)
+    seq = np.array([N], np.int32)
+    idx = np.full((B, Hq, k), -1, np.int32)
+    idx[0, 1] = np.sort(g.choice(N, k, replace=False))
+    idx[0, 3] = np.sort(g.choice(N, k, replace=False))
+    role = np.array([R, S, R, S], np.uint8)
+    a = oracle.hybrid_layer(q, K, V, seq, role, idx, k)
+    b = oracle.hybrid_layer(q, K, V, seq, role, idx, k, block=1)
+    assert np.array_equal(a[0], b[0]) and np.array_equal(a[1], b[1])
+
+
+def test_block_layer_sets_are_whole_blocks_of_the_logits():
+    g = rng(9)
+    B, Hq, Hkv, d, N, k, blk = 2, 4, 2, 16, 300, 100, 8
+    q = g.standard_normal((B, Hq, d)).astype(np.float32)
+    K = g.standard_normal((B, Hkv, N, d)).astype(np.float32)
+    V = g.standard_normal((B, Hkv, N, d)).astype(np.float32)
+    seq = np.array([N, 203], np.int32)
+    out, idx, lg = oracle.hybrid_layer(q, K, V, seq, np.full(Hq, R, np.uint8),
+                                       np.full((B, Hq, k), -1, np.int32), k,
+                                       want_logits=True, block=blk)
+    for b in range(B):
+        n = int(seq[b])
+        for h in range(Hq):
+            _block_props(lg[b, h, :n], min(k, n), blk, idx[b, h])
+
+
+def test_sparse_set_ends_at_first_minus_one():
+    """A sparse head reads its set up to the first -1: the output equals the
+    sparse head over that prefix alone, and an empty set gives 0."""
+    g = rng(10)
+    B, Hq, Hkv, d, N = 1, 2, 1, 16, 64
+    q = g.standard_normal((B, Hq, d)).astype(np.float32)
+    K = g.standard_normal((B, Hkv, N, d)).astype(np.float32)
+    V = g.standard_normal((B, Hkv, N, d)).astype(np.float32)
+    seq = np.array([N], np.int32)
+    role = np.array([R, S], np.uint8)
+    pre = np.sort(g.choice(N, 7, replace=False)).astype(np.int32)
+    full = np.full((B, Hq, 12), -1, np.int32)
+    full[0, 1, :7] = pre
+    a = oracle.hybrid_layer(q, K, V, seq, role, full, 12)
+    short = np.full((B, Hq, 7), -1, np.int32)
+    short[0, 1] = pre
+    b = oracle.hybrid_layer(q, K, V, seq, role, short, 7)
+    assert np.allclose(a[0][0, 1], b[0][0, 1], rtol=0, atol=1e-12)
+    empty = np.full((B, Hq, 12), -1, np.int32)
+    c = oracle.hybrid_layer(q, K, V, seq, role, empty, 12)
+    assert np.all(c[0][0, 1] == 0.0)
+    bad = full.copy()
+    bad[0, 1, 9] = 40   # an entry after the end of the set
+    with pytest.raises(oracle.OracleError):
+        oracle.hybrid_layer(q, K, V, seq, role, bad, 12)
