@@ -41,7 +41,7 @@ EXPORTED = ("lychee_workspace_size", "lychee_workspace_offsets", "lychee_hybrid_
 class Shape(ctypes.Structure):
     _fields_ = [("B", ctypes.c_int32), ("Hq", ctypes.c_int32), ("Hkv", ctypes.c_int32),
                 ("d", ctypes.c_int32), ("N_max", ctypes.c_int32), ("dtype", ctypes.c_int32),
-                ("k", ctypes.c_int32)]
+                ("k", ctypes.c_int32), ("block", ctypes.c_int32)]
 
 
 class LycheeError(RuntimeError):

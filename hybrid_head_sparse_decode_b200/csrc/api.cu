@@ -21,7 +21,7 @@ namespace {
 constexpr int kVersion = 100;   // 0.1.0
 
 struct Layout {
-  size_t logits, part_ml, part_acc, part_n, bitmaps, total;
+  size_t logits, part_ml, part_acc, part_n, bitmaps, bkeys, total;
   int nchunk, nwords;
 };
 
@@ -42,6 +42,11 @@ lychee_status check_shape(const lychee_shape* s) {
   const long long nchunk = (s->N_max + kChunkMin - 1) / kChunkMin;
   if ((long long)s->B * s->Hkv * nchunk >= (1LL << 31)) return LYCHEE_ERR_UNSUPPORTED;
   if ((long long)s->B * s->Hq >= (1LL << 24)) return LYCHEE_ERR_UNSUPPORTED;
+  if (s->block < 0) return LYCHEE_ERR_INVALID_ARG;
+  if (s->block > 1) {
+    if (s->block % 32 != 0 || s->block > 1024 || s->block > s->k) return LYCHEE_ERR_INVALID_ARG;
+    if (block_select_smem(s->N_max, s->block) > kBlockSelSmemMax) return LYCHEE_ERR_UNSUPPORTED;
+  }
   return LYCHEE_OK;
 }
 
@@ -61,6 +66,8 @@ Layout layout_of(const lychee_shape* s) {
   off += align256(bh * L.nchunk * 4);
   L.bitmaps = off;
   off += align256(bh * L.nwords * 4);
+  L.bkeys = off;   // block keys for block-granular selection (blocks of >= 32 positions)
+  off += s->block > 1 ? align256(bh * L.nwords * 4) : 0;
   L.total = off;
   return L;
 }
@@ -293,6 +300,29 @@ lychee_status run_layer(const Ctx& c, const void* q, const void* kc, const void*
   cp.B = s->B; cp.Hq = Hq; cp.N_max = s->N_max; cp.nchunk = c.L.nchunk;
   cp.chunk = ap.chunk;
   cp.scale_log2 = ap.scale_log2;
+  if (s->block > 1 && nr > 0) {
+    // block-granular selection: block keys, the selection, then the combine
+    BlockSelParams bp{};
+    bp.logits = logits;
+    bp.bkeys = reinterpret_cast<uint32_t*>(c.ws + c.L.bkeys);
+    bp.seqlens = seqlens;
+    bp.k_per_seq = k_per_seq;
+    bp.bitmaps = tp.bitmaps;
+    bp.idx_out = tp.idx_out;
+    bp.err = err;
+    bp.B = s->B; bp.Hq = Hq; bp.N_max = s->N_max; bp.nwords = c.L.nwords; bp.k = s->k;
+    bp.nheads = nr;
+    bp.block = s->block;
+    bp.nblk_stride = c.L.nwords;
+    std::memcpy(bp.heads, rheads, nr);
+    for (int stage = 0; stage < 2; ++stage) {
+      e = timed(kKindTopk, c.st, [&] { return launch_block_select(bp, stage, c.st); });
+      if (e != cudaSuccess) return LYCHEE_ERR_CUDA;
+    }
+    e = timed(kKindCombine, c.st, [&] { return launch_combine(cp, s->dtype, s->d, c.st); });
+    if (e != cudaSuccess) return LYCHEE_ERR_CUDA;
+    return LYCHEE_OK;
+  }
   e = timed(nr > 0 ? kKindTopkCombine : kKindCombine, c.st,
             [&] { return launch_topk_combine(tp, cp, s->dtype, s->d, c.st); });
   if (e != cudaSuccess) return LYCHEE_ERR_CUDA;

@@ -20,9 +20,11 @@ constexpr int kEntriesPerCta = 4 * kThreads;   // set entries one build_bits CTA
 // the first entry of a word ORs that word's entries (at most 32, contiguous in
 // the ascending row) and also writes the empty words between the previous
 // entry's word and its own; the first and last entries cover the words before
-// and after the set.  An entry outside [0, n_b) or not strictly above its
-// predecessor sets kErrBadIndex; the row is then not a set and its bitmap is
-// unspecified, but every store still stays inside the row.
+// and after the set.  A set ends at its first -1 (at most k_b entries are
+// read); that entry clears the words after the last member.  An entry outside
+// [0, n_b), not strictly above its predecessor, or after the end of the set
+// sets kErrBadIndex; the row is then not a set and its bitmap is unspecified,
+// but every store still stays inside the row.
 __global__ void __launch_bounds__(kThreads) build_bits_kernel(const __grid_constant__ BuildBitsParams p) {
   pdl_launch_dependents();
   pdl_wait();
@@ -43,7 +45,18 @@ __global__ void __launch_bounds__(kThreads) build_bits_kernel(const __grid_const
     if (p.idx_out) p.idx_out[bh * p.k + t] = j;
     if (t >= kb) continue;
     const int prev = t > 0 ? idx[t - 1] : -1;
-    if (j < 0 || j >= n || j <= prev) {
+    if (j < 0) {
+      // the set ends at its first -1: that entry clears the words after the
+      // last member (all of them for an empty set)
+      if (t == 0 || prev >= 0)
+        for (int g = t == 0 ? 0 : (prev >> 5) + 1; g < words; ++g) row[g] = 0u;
+      continue;
+    }
+    if (t > 0 && prev < 0) {   // a member after the end of the set
+      flag_error(p.err, kErrBadIndex);
+      continue;
+    }
+    if (j >= n || j <= prev) {
       flag_error(p.err, kErrBadIndex);
       continue;
     }

@@ -43,21 +43,23 @@ def _need_cuda(name, t, dtype=None, shape=None):
         raise ValueError(f"{name} must have shape {tuple(shape)}, got {tuple(t.shape)}")
 
 
-def make_shape(B, Hq, Hkv, d, N_max, k, dtype) -> N.Shape:
+def make_shape(B, Hq, Hkv, d, N_max, k, dtype, block=0) -> N.Shape:
+    """block: 0 (token-level argsTopK) or the positions per selected block of a
+    retrieval head's set (a multiple of 32, at most k)."""
     code = _DT.get(dtype, dtype)
-    return N.Shape(int(B), int(Hq), int(Hkv), int(d), int(N_max), int(code), int(k))
+    return N.Shape(int(B), int(Hq), int(Hkv), int(d), int(N_max), int(code), int(k), int(block))
 
 
-def workspace_size(B, Hq, Hkv, d, N_max, k, dtype) -> int:
-    sh = make_shape(B, Hq, Hkv, d, N_max, k, dtype)
+def workspace_size(B, Hq, Hkv, d, N_max, k, dtype, block=0) -> int:
+    sh = make_shape(B, Hq, Hkv, d, N_max, k, dtype, block)
     n = N.load().lychee_workspace_size(ctypes.byref(sh))
     if n == 0:
         raise N.LycheeError(N.ERR_INVALID_ARG, "workspace_size")
     return int(n)
 
 
-def alloc_workspace(B, Hq, Hkv, d, N_max, k, dtype, device=None) -> torch.Tensor:
-    n = workspace_size(B, Hq, Hkv, d, N_max, k, dtype)
+def alloc_workspace(B, Hq, Hkv, d, N_max, k, dtype, device=None, block=0) -> torch.Tensor:
+    n = workspace_size(B, Hq, Hkv, d, N_max, k, dtype, block)
     return torch.empty(n, dtype=torch.uint8, device=device or "cuda")
 
 
@@ -74,10 +76,11 @@ def _check(st, what):
 
 
 def hybrid_decode_attn(q, k_cache, v_cache, seqlens, head_role, idx_in, k, *, k_per_seq=None,
-                       out=None, idx_out=None, workspace=None, stream=None):
+                       out=None, idx_out=None, workspace=None, stream=None, block=0):
     """One hybrid-head layer.  q [B,Hq,d]; caches [B,Hkv,N_max,d] (bf16 or fp32);
     seqlens [B] int32 (device); head_role [Hq] (host, 1 = retrieval);
-    idx_in [B,Hq,k] int32 (device, or None when every head is retrieval).
+    idx_in [B,Hq,k] int32 (device, or None when every head is retrieval);
+    block: 0 for argsTopK sets, else positions per selected block.
     Returns (out [B,Hq,d], idx_out [B,Hq,k])."""
     B, Hq, d = q.shape
     _, Hkv, N_max, _ = k_cache.shape
@@ -97,9 +100,9 @@ def hybrid_decode_attn(q, k_cache, v_cache, seqlens, head_role, idx_in, k, *, k_
     if idx_out is None:
         idx_out = torch.empty((B, Hq, k), dtype=torch.int32, device=q.device)
     _need_cuda("idx_out", idx_out, torch.int32, (B, Hq, k))
-    sh = make_shape(B, Hq, Hkv, d, N_max, k, dt)
+    sh = make_shape(B, Hq, Hkv, d, N_max, k, dt, block)
     if workspace is None:
-        workspace = alloc_workspace(B, Hq, Hkv, d, N_max, k, dt, q.device)
+        workspace = alloc_workspace(B, Hq, Hkv, d, N_max, k, dt, q.device, block)
     _need_cuda("workspace", workspace, torch.uint8)
     st = N.load().lychee_hybrid_decode_attn(
         ctypes.byref(sh), _ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(seqlens), _ptr(k_per_seq),
@@ -111,7 +114,7 @@ def hybrid_decode_attn(q, k_cache, v_cache, seqlens, head_role, idx_in, k, *, k_
 
 def hybrid_decode_attn_noalloc(q, k_cache, v_cache, seqlens, head_role, idx_in, k, *,
                                k_per_seq=None, out=None, idx_out=None, device_error=None,
-                               stream=None):
+                               stream=None, block=0):
     """hybrid_decode_attn served from the library's static device scratch: no
     workspace argument and no device allocation by the library (out / idx_out
     are allocated here only when not given).  device_error: optional device
@@ -129,7 +132,7 @@ def hybrid_decode_attn_noalloc(q, k_cache, v_cache, seqlens, head_role, idx_in, 
         _need_cuda("k_per_seq", k_per_seq, torch.int32, (B,))
     if idx_in is not None:
         _need_cuda("idx_in", idx_in, torch.int32, (B, Hq, k))
-    need = workspace_size(B, Hq, Hkv, d, N_max, k, dt)
+    need = workspace_size(B, Hq, Hkv, d, N_max, k, dt, block)
     if need > N.NOALLOC_SCRATCH_BYTES:
         raise ValueError(f"this layer needs {need} bytes of scratch; the static scratch holds "
                          f"{N.NOALLOC_SCRATCH_BYTES} (use hybrid_decode_attn with a workspace)")
@@ -142,7 +145,7 @@ def hybrid_decode_attn_noalloc(q, k_cache, v_cache, seqlens, head_role, idx_in, 
     _need_cuda("idx_out", idx_out, torch.int32, (B, Hq, k))
     if device_error is not None:
         _need_cuda("device_error", device_error, torch.int32, (1,))
-    sh = make_shape(B, Hq, Hkv, d, N_max, k, dt)
+    sh = make_shape(B, Hq, Hkv, d, N_max, k, dt, block)
     st = N.load().lychee_hybrid_decode_attn_noalloc(
         ctypes.byref(sh), _ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(seqlens), _ptr(k_per_seq),
         ctypes.c_void_p(role.data_ptr()), _ptr(idx_in), _ptr(out), _ptr(idx_out),
@@ -152,10 +155,12 @@ def hybrid_decode_attn_noalloc(q, k_cache, v_cache, seqlens, head_role, idx_in, 
 
 
 def decode_stack(q, k_caches, v_caches, seqlens, head_roles, k, *, k_per_seq=None, out=None,
-                 idx_final=None, idx_layers=None, want_layers=False, workspace=None, stream=None):
+                 idx_final=None, idx_layers=None, want_layers=False, workspace=None, stream=None,
+                 block=0):
     """L chained layers of one decode step.  q [L,B,Hq,d]; k_caches / v_caches:
     sequences of L tensors [B,Hkv,N_max,d]; head_roles [L,Hq] (host, row 0 all
-    retrieval).  Returns (out [L,B,Hq,d], idx_final [B,Hq,k], idx_layers or None)."""
+    retrieval); block as in hybrid_decode_attn.  Returns (out [L,B,Hq,d],
+    idx_final [B,Hq,k], idx_layers or None)."""
     L, B, Hq, d = q.shape
     if len(k_caches) != L or len(v_caches) != L:
         raise ValueError("need one K and one V cache per layer")
@@ -179,9 +184,9 @@ def decode_stack(q, k_caches, v_caches, seqlens, head_roles, k, *, k_per_seq=Non
         idx_layers = torch.empty((L, B, Hq, k), dtype=torch.int32, device=q.device)
     if idx_layers is not None:
         _need_cuda("idx_layers", idx_layers, torch.int32, (L, B, Hq, k))
-    sh = make_shape(B, Hq, Hkv, d, N_max, k, dt)
+    sh = make_shape(B, Hq, Hkv, d, N_max, k, dt, block)
     if workspace is None:
-        workspace = alloc_workspace(B, Hq, Hkv, d, N_max, k, dt, q.device)
+        workspace = alloc_workspace(B, Hq, Hkv, d, N_max, k, dt, q.device, block)
     _need_cuda("workspace", workspace, torch.uint8)
     kp = (ctypes.c_void_p * L)(*[t.data_ptr() for t in k_caches])
     vp = (ctypes.c_void_p * L)(*[t.data_ptr() for t in v_caches])

@@ -70,7 +70,18 @@ typedef enum { LYCHEE_BF16 = 0, LYCHEE_FP32 = 1 } lychee_dtype;
 enum { LYCHEE_ROLE_SPARSE = 0, LYCHEE_ROLE_RETRIEVAL = 1 };
 
 /* Problem shape.  Supported: Hq % Hkv == 0 with G = Hq / Hkv in {1, 2, 4, 8},
- * Hq <= 128, d in {64, 128}, 1 <= k <= N_max <= 2^24, B >= 1. */
+ * Hq <= 128, d in {64, 128}, 1 <= k <= N_max <= 2^24, B >= 1.
+ *
+ * block selects how a retrieval head picks the set it hands on (method step
+ * (3)): 0 or 1, argsTopK of its logits (k_b positions); a multiple of 32 in
+ * [32, 1024] with block <= k and ceil(N_max / block) <= 32768, block-granular
+ * selection: the positions are cut into blocks of `block` (the last one
+ * shorter), a block's score is its largest logit, and the max(1, floor(k_b /
+ * block)) best blocks (ties: lower block index) are taken whole -- the
+ * block-sparse reading of the page's decoding kernel, with the block-level
+ * maximum scores and k/B top blocks of the HySparse page (B = 64).  A set
+ * then holds up to k_b positions (at least one block) and its index row ends
+ * at the first -1. */
 typedef struct {
   int32_t B;      /* batch (sequences)                         */
   int32_t Hq;     /* query heads                               */
@@ -79,6 +90,7 @@ typedef struct {
   int32_t N_max;  /* cache capacity in positions               */
   int32_t dtype;  /* lychee_dtype of q, caches and out         */
   int32_t k;      /* capacity of an index-set row              */
+  int32_t block;  /* 0/1: token-level argsTopK; else positions per selected block */
 } lychee_shape;
 
 /* Bytes of device workspace that lychee_hybrid_decode_attn and
@@ -105,13 +117,14 @@ LYCHEE_API lychee_status lychee_workspace_offsets(const lychee_shape* s, size_t*
  *   seqlens   device [B] int32, 1 <= n_b <= N_max (the current token is included)
  *   k_per_seq device [B] int32 or NULL (then k_b = min(k, n_b))
  *   head_role HOST   [Hq] uint8, LYCHEE_ROLE_RETRIEVAL or LYCHEE_ROLE_SPARSE
- *   idx_in    device [B, Hq, k] int32; rows of sparse heads are read (their first
- *             k_b entries, strictly ascending, in [0, n_b)); may be NULL only
- *             when every head is a retrieval head
+ *   idx_in    device [B, Hq, k] int32; rows of sparse heads are read (their
+ *             entries before the first -1, at most k_b of them, strictly
+ *             ascending, in [0, n_b)); may be NULL only when every head is a
+ *             retrieval head
  *   out       device [B, Hq, d] dtype
  *   idx_out   device [B, Hq, k] int32: retrieval heads get argsTopK of their
- *             logits (ascending, -1 padded); sparse heads get their idx_in row
- *             copied bit for bit
+ *             logits, or their block-granular set (s->block), ascending, -1
+ *             padded; sparse heads get their idx_in row copied bit for bit
  *   workspace device, >= lychee_workspace_size(s) bytes, 256-byte aligned
  *   stream    cudaStream_t
  * The call overwrites the whole workspace header, so device errors reported by
