@@ -235,7 +235,8 @@ def run_lychee(args, rank, world, device):
     L, B, Hq, Hkv, d, N = prob.shape
     dt = prob.q.dtype
     row_bytes = 2 * d * prob.q.element_size()
-    ws = ops.alloc_workspace(B, Hq, Hkv, d, N, prob.k, dt, device)
+    blk = args.block
+    ws = ops.alloc_workspace(B, Hq, Hkv, d, N, prob.k, dt, device, block=blk)
     out = torch.empty((L, B, Hq, d), dtype=dt, device=device)
     fin = torch.empty((B, Hq, prob.k), dtype=torch.int32, device=device)
     idx_layers = torch.empty((L, B, Hq, prob.k), dtype=torch.int32, device=device)
@@ -243,12 +244,13 @@ def run_lychee(args, rank, world, device):
 
     def step(r=roles, o=out):
         ops.decode_stack(prob.q, prob.k_caches, prob.v_caches, prob.seqlens, r, prob.k,
-                         k_per_seq=prob.k_per_seq, out=o, idx_final=fin, workspace=ws)
+                         k_per_seq=prob.k_per_seq, out=o, idx_final=fin, workspace=ws,
+                         block=blk)
 
     # untimed pass that also records every layer's sets, to count algorithmic bytes
     ops.decode_stack(prob.q, prob.k_caches, prob.v_caches, prob.seqlens, roles, prob.k,
                      k_per_seq=prob.k_per_seq, out=out, idx_final=fin, idx_layers=idx_layers,
-                     workspace=ws)
+                     workspace=ws, block=blk)
     st, bits = ops.check_device_error(ws)
     if st != 0:
         raise SystemExit(f"device error {st} bits {bits}")
@@ -282,7 +284,7 @@ def run_lychee(args, rank, world, device):
     ms_total = t0.elapsed_time(t1)
     # the same steps again with every library launch bracketed by CUDA events on
     # its stream: per-kernel durations for the roofline of the attention kernel
-    prof = ops.Profile(max_launches=args.steps * (3 * L + 2) + 16)
+    prof = ops.Profile(max_launches=args.steps * (4 * L + 2) + 16)
     torch.cuda.synchronize()
     with prof:
         for _ in range(args.steps):
@@ -335,7 +337,7 @@ def run_lychee(args, rank, world, device):
         sl_d.copy_(sl_h, non_blocking=True)
         kb_d.copy_(kb_h, non_blocking=True)
         ops.decode_stack(q_d, prob.k_caches, prob.v_caches, sl_d, roles, prob.k, k_per_seq=kb_d,
-                         out=out, idx_final=fin, workspace=ws)
+                         out=out, idx_final=fin, workspace=ws, block=blk)
         out_h.copy_(out, non_blocking=True)
         fin_h.copy_(fin, non_blocking=True)
 
@@ -361,7 +363,8 @@ def run_lychee(args, rank, world, device):
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_step, 5),
         "higher_is_better": False, "scaling": "weak", "vs_baseline": None,
         "dtype": "fp32", "data": "synthetic (seeded; planted high-affinity keys)",
-        "config": describe(args.workload, prob),
+        "config": dict(describe(args.workload, prob),
+                       select="argsTopK" if blk <= 1 else f"blocks of {blk}"),
         "us_per_layer": round(ms_step * 1e3 / L, 3),
         "step_hbm_gbs_union": round(sum(union_bytes) / (ms_step * 1e-3) / 1e9, 1),
         "step_hbm_gbs_literal": round(sum(literal_bytes) / (ms_step * 1e-3) / 1e9, 1),
@@ -475,6 +478,9 @@ def main():
     ap.add_argument("--impl", default="lychee", choices=["lychee", "reference"])
     ap.add_argument("--workload", default="qwen3_stack_128k")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--block", type=int, default=0,
+                    help="0: retrieval heads hand on argsTopK sets (the method's step); "
+                         "B > 1: block-granular sets of B positions")
     args = ap.parse_args()
     if args.warmup < 3 and args.impl == "lychee":
         args.warmup = 3

@@ -11,6 +11,7 @@
 #include <vector>
 
 #include "common.cuh"
+#include "blocksel.h"
 #include "kernels.h"
 #include "lychee.h"
 
@@ -21,7 +22,7 @@ namespace {
 constexpr int kVersion = 100;   // 0.1.0
 
 struct Layout {
-  size_t logits, part_ml, part_acc, part_n, bitmaps, bkeys, total;
+  size_t logits, part_ml, part_acc, part_n, bitmaps, total;
   int nchunk, nwords;
 };
 
@@ -66,8 +67,6 @@ Layout layout_of(const lychee_shape* s) {
   off += align256(bh * L.nchunk * 4);
   L.bitmaps = off;
   off += align256(bh * L.nwords * 4);
-  L.bkeys = off;   // block keys for block-granular selection (blocks of >= 32 positions)
-  off += s->block > 1 ? align256(bh * L.nwords * 4) : 0;
   L.total = off;
   return L;
 }
@@ -301,10 +300,9 @@ lychee_status run_layer(const Ctx& c, const void* q, const void* kc, const void*
   cp.chunk = ap.chunk;
   cp.scale_log2 = ap.scale_log2;
   if (s->block > 1 && nr > 0) {
-    // block-granular selection: block keys, the selection, then the combine
+    // block-granular selection and the combine in one launch
     BlockSelParams bp{};
     bp.logits = logits;
-    bp.bkeys = reinterpret_cast<uint32_t*>(c.ws + c.L.bkeys);
     bp.seqlens = seqlens;
     bp.k_per_seq = k_per_seq;
     bp.bitmaps = tp.bitmaps;
@@ -313,13 +311,9 @@ lychee_status run_layer(const Ctx& c, const void* q, const void* kc, const void*
     bp.B = s->B; bp.Hq = Hq; bp.N_max = s->N_max; bp.nwords = c.L.nwords; bp.k = s->k;
     bp.nheads = nr;
     bp.block = s->block;
-    bp.nblk_stride = c.L.nwords;
     std::memcpy(bp.heads, rheads, nr);
-    for (int stage = 0; stage < 2; ++stage) {
-      e = timed(kKindTopk, c.st, [&] { return launch_block_select(bp, stage, c.st); });
-      if (e != cudaSuccess) return LYCHEE_ERR_CUDA;
-    }
-    e = timed(kKindCombine, c.st, [&] { return launch_combine(cp, s->dtype, s->d, c.st); });
+    e = timed(kKindTopkCombine, c.st,
+              [&] { return launch_block_select_combine(bp, cp, s->dtype, s->d, c.st); });
     if (e != cudaSuccess) return LYCHEE_ERR_CUDA;
     return LYCHEE_OK;
   }

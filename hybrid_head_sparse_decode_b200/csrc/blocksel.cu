@@ -11,13 +11,18 @@
 // index) are taken whole.  The set is written as a membership bitmap row and/or
 // an ascending index row padded with -1.
 //
-// Two launches: one thread per block reduces the block to an order-preserving
-// key (many CTAs per head, so the 4 n_b bytes of logits stream from L2 in
-// parallel); then one CTA per (sequence, head) runs a radix select over the
-// block keys in shared memory (8-bit digits, most significant first, stopping
-// once the chosen bucket holds exactly the blocks still to take) and writes
-// the set.
+// One CTA per (sequence, head) reduces each block of the head's logits to the
+// order-preserving key of its largest logit (one block per thread, 16-byte
+// loads from L2, where the attention kernel just wrote them), runs a radix
+// select over the keys in shared memory (8-bit digits, most significant first,
+// stopping once the chosen bucket holds exactly the blocks still to take) and
+// writes the set.
+// The same launch runs the combine of every head (combine_body.cuh) on its
+// other CTAs: the two read disjoint data and write disjoint outputs.
+#include "cluster.cuh"
+#include "combine_body.cuh"
 #include "common.cuh"
+#include "blocksel.h"
 #include "kernels.h"
 
 namespace lychee {
@@ -35,28 +40,6 @@ __device__ __forceinline__ void head_of(const BlockSelParams& p, int pair, int& 
   n = min(max(p.seqlens[b], 1), p.N_max);
   kb = p.k_per_seq ? p.k_per_seq[b] : p.k;
   kb = min(min(max(kb, 1), p.k), n);
-}
-
-// One thread per block: the key of the block's largest logit.
-__global__ void __launch_bounds__(kKeyThreads) block_keys_kernel(const __grid_constant__ BlockSelParams p) {
-  pdl_launch_dependents();
-  pdl_wait();
-  int b, h, n, kb;
-  head_of(p, blockIdx.y, b, h, n, kb);
-  const int nblk = (n + p.block - 1) / p.block;
-  const int c = blockIdx.x * kKeyThreads + threadIdx.x;
-  if (c >= nblk) return;
-  const float* row = p.logits + (size_t)(b * p.Hq + h) * p.N_max;
-  const int j0 = c * p.block, j1 = min(n, j0 + p.block);
-  float mx = -INFINITY;
-  int j = j0;
-  if ((reinterpret_cast<uintptr_t>(row + j0) & 15u) == 0)
-    for (; j + 4 <= j1; j += 4) {
-      const float4 v = *reinterpret_cast<const float4*>(row + j);
-      mx = fmaxf(mx, fmaxf(fmaxf(v.x, v.y), fmaxf(v.z, v.w)));
-    }
-  for (; j < j1; ++j) mx = fmaxf(mx, row[j]);
-  p.bkeys[(size_t)(b * p.Hq + h) * p.nblk_stride + c] = float_to_key(mx);
 }
 
 // Exclusive scan of one value per thread over the CTA; *total gets the sum.
@@ -82,24 +65,33 @@ __device__ __forceinline__ uint32_t cta_scan(uint32_t v, uint32_t* wsum, uint32_
   return before + x - v;
 }
 
-// One CTA per (sequence, retrieval head): the selection and the output rows.
-// keys (dynamic shared memory) hold the block keys, then per block the output
-// offset of a selected block, or kFull.
-__global__ void __launch_bounds__(kSelThreads, 1) block_select_kernel(const __grid_constant__ BlockSelParams p) {
-  extern __shared__ __align__(16) uint32_t keys[];
+// One CTA of the selection: (sequence, retrieval head) number `pair`.  keys
+// (dynamic shared memory) hold the block keys, then per block the output offset
+// of a selected block, or kFull.
+__device__ __forceinline__ void block_select_body(const BlockSelParams& p, int pair, uint32_t* keys) {
   __shared__ uint32_t hist[256];
   __shared__ uint32_t wsum[kSelWarps];
   __shared__ uint32_t bc[4];
-  pdl_launch_dependents();
-  pdl_wait();
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   int b, h, n, kb;
-  head_of(p, blockIdx.x, b, h, n, kb);
+  head_of(p, pair, b, h, n, kb);
   const int block = p.block;
   const int nblk = (n + block - 1) / block;
   const int kblk = min(max(1, kb / block), nblk);
   const size_t bh = (size_t)b * p.Hq + h;
-  for (int c = tid; c < nblk; c += kSelThreads) keys[c] = p.bkeys[bh * p.nblk_stride + c];
+  const float* row = p.logits + bh * p.N_max;
+  for (int c = tid; c < nblk; c += kSelThreads) {
+    const int j0 = c * block, j1 = min(n, j0 + block);
+    float mx = -INFINITY;
+    int j = j0;
+    if ((reinterpret_cast<uintptr_t>(row + j0) & 15u) == 0)
+      for (; j + 4 <= j1; j += 4) {
+        const float4 v = *reinterpret_cast<const float4*>(row + j);
+        mx = fmaxf(mx, fmaxf(fmaxf(v.x, v.y), fmaxf(v.z, v.w)));
+      }
+    for (; j < j1; ++j) mx = fmaxf(mx, row[j]);
+    keys[c] = float_to_key(mx);
+  }
 
   // ---- radix select of the kblk-th largest key T
   uint32_t prefix = 0, pmask = 0, krem = (uint32_t)kblk;
@@ -192,36 +184,73 @@ __global__ void __launch_bounds__(kSelThreads, 1) block_select_kernel(const __gr
   }
 }
 
+// The selection on the first nsel CTAs (whole clusters up to nsel_pad), the
+// combine of every head on the next ncomb (the kCombineSplit CTAs of a head are
+// one cluster).
+template <typename T, int D>
+__global__ void __launch_bounds__(kSelThreads, 1)
+    block_select_combine_kernel(const __grid_constant__ BlockSelParams p,
+                                const __grid_constant__ CombineParams cp, int nsel, int nsel_pad) {
+  static_assert(kSelThreads == kCombThreads, "one block size for both roles");
+  extern __shared__ __align__(16) uint32_t dsm[];
+  unsigned char* csm = reinterpret_cast<unsigned char*>(dsm);
+  pdl_launch_dependents();
+  const int cta = blockIdx.x;
+  if (cta >= nsel_pad) combine_prologue<D>(csm);
+  pdl_wait();
+  if (cta < nsel) block_select_body(p, cta, dsm);
+  else if (cta >= nsel_pad) combine_body<T, D>(cp, cta - nsel_pad, csm);
+}
+
+template <typename T, int D>
+cudaError_t launch_bsc(const BlockSelParams& p, const CombineParams& cp, cudaStream_t st) {
+  auto kfn = block_select_combine_kernel<T, D>;
+  static bool attr = false;
+  if (!attr) {
+    const cudaError_t e = cudaFuncSetAttribute(kfn, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                               (int)kBlockSelSmemMax);
+    if (e != cudaSuccess) return e;
+    attr = true;
+  }
+  const int nsel = p.B * p.nheads;
+  const int nsel_pad = (nsel + kCombineSplit - 1) / kCombineSplit * kCombineSplit;
+  const int ncomb = cp.B * cp.Hq * kCombineSplit;
+  size_t smem = block_select_smem(p.N_max, p.block);
+  if (smem > kBlockSelSmemMax) return cudaErrorInvalidValue;
+  if (combine_smem_bytes<D>() > smem) smem = combine_smem_bytes<D>();
+  cudaLaunchConfig_t cfg{};
+  cfg.gridDim = dim3((unsigned)(nsel_pad + ncomb));
+  cfg.blockDim = dim3(kSelThreads);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute at[2];
+  at[0].id = cudaLaunchAttributeClusterDimension;
+  at[0].val.clusterDim.x = kCombineSplit;
+  at[0].val.clusterDim.y = 1;
+  at[0].val.clusterDim.z = 1;
+  at[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  at[1].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = at;
+  cfg.numAttrs = 2;
+  const cudaError_t e = cudaLaunchKernelEx(&cfg, kfn, p, cp, nsel, nsel_pad);
+  if (e != cudaSuccess) return e;
+  return cudaGetLastError();
+}
+
 }  // namespace
 
 size_t block_select_smem(int N_max, int block) {
   return (size_t)((N_max + block - 1) / block) * 4;
 }
 
-cudaError_t launch_block_select(const BlockSelParams& p, int stage, cudaStream_t st) {
-  if (p.nheads <= 0) return cudaSuccess;
-  const int nblk_max = (p.N_max + p.block - 1) / p.block;
-  const size_t smem = block_select_smem(p.N_max, p.block);
-  if (smem > kBlockSelSmemMax) return cudaErrorInvalidValue;
-  static bool attr = false;
-  if (!attr) {
-    const cudaError_t e = cudaFuncSetAttribute(block_select_kernel,
-                                               cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                               (int)kBlockSelSmemMax);
-    if (e != cudaSuccess) return e;
-    attr = true;
-  }
-  cudaError_t e;
-  if (stage == 0)
-    e = launch_pdl(block_keys_kernel,
-                   dim3((unsigned)((nblk_max + kKeyThreads - 1) / kKeyThreads),
-                        (unsigned)(p.B * p.nheads)),
-                   dim3(kKeyThreads), 0, st, p);
-  else
-    e = launch_pdl(block_select_kernel, dim3((unsigned)(p.B * p.nheads)), dim3(kSelThreads), smem,
-                   st, p);
-  if (e != cudaSuccess) return e;
-  return cudaGetLastError();
+cudaError_t launch_block_select_combine(const BlockSelParams& p, const CombineParams& cp,
+                                        int dtype, int D, cudaStream_t st) {
+  if (p.nheads <= 0) return launch_combine(cp, dtype, D, st);
+  if (dtype == 0 && D == 128) return launch_bsc<__nv_bfloat16, 128>(p, cp, st);
+  if (dtype == 0 && D == 64) return launch_bsc<__nv_bfloat16, 64>(p, cp, st);
+  if (dtype == 1 && D == 128) return launch_bsc<float, 128>(p, cp, st);
+  if (dtype == 1 && D == 64) return launch_bsc<float, 64>(p, cp, st);
+  return cudaErrorInvalidValue;
 }
 
 }  // namespace lychee

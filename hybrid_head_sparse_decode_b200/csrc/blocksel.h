@@ -1,0 +1,29 @@
+// blocksel.h -- parameter block and launcher of the block-granular selection
+// (blocksel.cu), internal.
+#pragma once
+
+#include "kernels.h"
+
+namespace lychee {
+
+// Block-granular selection of retrieval heads' sets (blocksel.cu): blocks of
+// `block` positions scored by their largest logit, the max(1, k_b / block) best
+// taken whole.  block is a multiple of 32 (whole bitmap words).
+struct BlockSelParams {
+  const float* logits;       // [B, Hq, N_max]: raw q.k of the retrieval heads
+  const int32_t* seqlens;    // [B]
+  const int32_t* k_per_seq;  // [B] or null
+  uint32_t* bitmaps;         // [B, Hq, nwords] or null
+  int32_t* idx_out;          // [B, Hq, k] or null: ascending, -1 padded
+  uint32_t* err;
+  int B, Hq, N_max, nwords, k, nheads, block;
+  uint8_t heads[128];        // the retrieval heads handled by this launch
+};
+constexpr size_t kBlockSelSmemMax = 128 * 1024;   // block keys of one head, at most
+size_t block_select_smem(int N_max, int block);
+// The selection of the retrieval heads and the combine of every head in one
+// launch; just the combine when p.nheads is 0.
+cudaError_t launch_block_select_combine(const BlockSelParams& p, const CombineParams& cp,
+                                        int dtype, int D, cudaStream_t st);
+
+}  // namespace lychee

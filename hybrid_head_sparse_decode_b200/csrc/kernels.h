@@ -63,25 +63,6 @@ struct CombineParams {
 };
 cudaError_t launch_combine(const CombineParams& p, int dtype, int D, cudaStream_t st);
 
-// Block-granular selection of retrieval heads' sets (blocksel.cu): blocks of
-// `block` positions scored by their largest logit, the max(1, k_b / block) best
-// taken whole.  block is a multiple of 32 (whole bitmap words).
-struct BlockSelParams {
-  const float* logits;       // [B, Hq, N_max]
-  uint32_t* bkeys;           // [B, Hq, nblk_stride]: block keys (scratch)
-  const int32_t* seqlens;    // [B]
-  const int32_t* k_per_seq;  // [B] or null
-  uint32_t* bitmaps;         // [B, Hq, nwords] or null
-  int32_t* idx_out;          // [B, Hq, k] or null: ascending, -1 padded
-  uint32_t* err;
-  int B, Hq, N_max, nwords, k, nheads, block, nblk_stride;
-  uint8_t heads[128];        // the retrieval heads handled by this launch
-};
-constexpr size_t kBlockSelSmemMax = 128 * 1024;   // block keys of one head, at most
-size_t block_select_smem(int N_max, int block);
-// stage 0: the block keys; stage 1: the selection (launch both, in order)
-cudaError_t launch_block_select(const BlockSelParams& p, int stage, cudaStream_t st);
-
 // The top-k of the retrieval heads and the combine of every head in one launch
 // (topk.cu); just the combine when p.nheads is 0.
 cudaError_t launch_topk_combine(const TopkParams& p, const CombineParams& cp, int dtype, int D,
