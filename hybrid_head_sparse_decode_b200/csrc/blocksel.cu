@@ -11,12 +11,13 @@
 // index) are taken whole.  The set is written as a membership bitmap row and/or
 // an ascending index row padded with -1.
 //
-// One CTA per (sequence, head) reduces each block of the head's logits to the
-// order-preserving key of its largest logit (one block per thread, 16-byte
-// loads from L2, where the attention kernel just wrote them), runs a radix
-// select over the keys in shared memory (8-bit digits, most significant first,
-// stopping once the chosen bucket holds exactly the blocks still to take) and
-// writes the set.
+// A cluster of kSelCtas CTAs per (sequence, head): each reduces its share of the
+// head's blocks to the order-preserving keys of their largest logits (one block
+// per thread, 16-byte loads from L2, where the attention kernel just wrote
+// them) and sends the keys into the shared memory of the cluster's first CTA
+// (16-byte st.async stores that complete its mbarrier).  That CTA runs a radix
+// select over all the keys (8-bit digits, most significant first, stopping once
+// the chosen bucket holds exactly the blocks still to take) and writes the set.
 // The same launch runs the combine of every head (combine_body.cuh) on its
 // other CTAs: the two read disjoint data and write disjoint outputs.
 #include "cluster.cuh"
@@ -32,6 +33,8 @@ constexpr uint32_t kFull = 0xffffffffu;
 constexpr int kKeyThreads = 256;
 constexpr int kSelThreads = 512;
 constexpr int kSelWarps = kSelThreads / 32;
+constexpr int kSelCtas = 8;        // CTAs per (sequence, head): one cluster
+static_assert(kSelCtas == kCombineSplit, "one cluster size for both roles");
 
 __device__ __forceinline__ void head_of(const BlockSelParams& p, int pair, int& b, int& h,
                                         int& n, int& kb) {
@@ -65,14 +68,29 @@ __device__ __forceinline__ uint32_t cta_scan(uint32_t v, uint32_t* wsum, uint32_
   return before + x - v;
 }
 
-// One CTA of the selection: (sequence, retrieval head) number `pair`.  keys
-// (dynamic shared memory) hold the block keys, then per block the output offset
-// of a selected block, or kFull.
-__device__ __forceinline__ void block_select_body(const BlockSelParams& p, int pair, uint32_t* keys) {
+// Before the previous kernel's results are needed: the first CTA of each
+// selection cluster sets up the barrier that counts one arrival per CTA of the
+// cluster (plus the bytes each sends), and the cluster learns it is set up.
+__device__ __forceinline__ void block_select_prologue(uint32_t* dsm) {
+  if (cluster_ctarank() == 0 && threadIdx.x == 0) {
+    mbar_init(reinterpret_cast<uint64_t*>(dsm), kSelCtas);
+    fence_mbar_init();
+  }
+  cluster_arrive_relaxed();
+}
+
+// One CTA of the selection of (sequence, retrieval head) number `pair`, after
+// block_select_prologue.  Dynamic shared memory: an mbarrier (16 bytes), then
+// the block keys (in the first CTA: all of them, then per block the output
+// offset of a selected block, or kFull).
+__device__ __forceinline__ void block_select_body(const BlockSelParams& p, int pair, uint32_t* dsm) {
   __shared__ uint32_t hist[256];
   __shared__ uint32_t wsum[kSelWarps];
   __shared__ uint32_t bc[4];
+  uint64_t* bar = reinterpret_cast<uint64_t*>(dsm);
+  uint32_t* keys = dsm + 4;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const uint32_t rank = cluster_ctarank();
   int b, h, n, kb;
   head_of(p, pair, b, h, n, kb);
   const int block = p.block;
@@ -80,7 +98,10 @@ __device__ __forceinline__ void block_select_body(const BlockSelParams& p, int p
   const int kblk = min(max(1, kb / block), nblk);
   const size_t bh = (size_t)b * p.Hq + h;
   const float* row = p.logits + bh * p.N_max;
-  for (int c = tid; c < nblk; c += kSelThreads) {
+  // this CTA's share of the blocks: a multiple of 4 (whole 16-byte pieces)
+  const int per = ((nblk + kSelCtas - 1) / kSelCtas + 3) & ~3;
+  const int cb0 = min(nblk, (int)rank * per), cb1 = min(nblk, cb0 + per);
+  for (int c = cb0 + tid; c < cb1; c += kSelThreads) {
     const int j0 = c * block, j1 = min(n, j0 + block);
     float mx = -INFINITY;
     int j = j0;
@@ -92,6 +113,23 @@ __device__ __forceinline__ void block_select_body(const BlockSelParams& p, int p
     for (; j < j1; ++j) mx = fmaxf(mx, row[j]);
     keys[c] = float_to_key(mx);
   }
+  __syncthreads();
+  cluster_wait();   // the first CTA's barrier is set up
+  const uint32_t lbar = dsmem_map(smem_u32(bar), 0);
+  if (rank != 0) {
+    // send the keys to the same place in the first CTA
+    const int nq = (cb1 - cb0 + 3) / 4;
+    if (tid == 0) mbar_arrive_expect_tx_remote(lbar, (uint32_t)nq * 16u);
+    for (int i = tid; i < nq; i += kSelThreads)
+      st_async_v4(dsmem_map(smem_u32(keys + cb0 + 4 * i), 0),
+                  *reinterpret_cast<const uint4*>(keys + cb0 + 4 * i), lbar);
+    cluster_arrive_relaxed();
+    cluster_wait();   // no CTA leaves while its keys may still be on their way
+    return;
+  }
+  if (tid == 0) mbar_arrive(bar);
+  mbar_wait_cluster(bar, 0u, p.err);   // every CTA's keys are here
+  cluster_arrive_relaxed();
 
   // ---- radix select of the kblk-th largest key T
   uint32_t prefix = 0, pmask = 0, krem = (uint32_t)kblk;
@@ -182,24 +220,26 @@ __device__ __forceinline__ void block_select_body(const BlockSelParams& p, int p
     const int m = (int)sel_seen * block - (keys[nblk - 1] != kFull ? nblk * block - n : 0);
     for (int t = m + tid; t < p.k; t += kSelThreads) orow[t] = -1;
   }
+  cluster_wait();
 }
 
-// The selection on the first nsel CTAs (whole clusters up to nsel_pad), the
+// The selection on the first nsel CTAs (kSelCtas per head, one cluster each), the
 // combine of every head on the next ncomb (the kCombineSplit CTAs of a head are
 // one cluster).
 template <typename T, int D>
 __global__ void __launch_bounds__(kSelThreads, 1)
     block_select_combine_kernel(const __grid_constant__ BlockSelParams p,
-                                const __grid_constant__ CombineParams cp, int nsel, int nsel_pad) {
+                                const __grid_constant__ CombineParams cp, int nsel) {
   static_assert(kSelThreads == kCombThreads, "one block size for both roles");
   extern __shared__ __align__(16) uint32_t dsm[];
   unsigned char* csm = reinterpret_cast<unsigned char*>(dsm);
   pdl_launch_dependents();
   const int cta = blockIdx.x;
-  if (cta >= nsel_pad) combine_prologue<D>(csm);
+  if (cta < nsel) block_select_prologue(dsm);
+  else combine_prologue<D>(csm);
   pdl_wait();
-  if (cta < nsel) block_select_body(p, cta, dsm);
-  else if (cta >= nsel_pad) combine_body<T, D>(cp, cta - nsel_pad, csm);
+  if (cta < nsel) block_select_body(p, cta / kSelCtas, dsm);
+  else combine_body<T, D>(cp, cta - nsel, csm);
 }
 
 template <typename T, int D>
@@ -212,14 +252,13 @@ cudaError_t launch_bsc(const BlockSelParams& p, const CombineParams& cp, cudaStr
     if (e != cudaSuccess) return e;
     attr = true;
   }
-  const int nsel = p.B * p.nheads;
-  const int nsel_pad = (nsel + kCombineSplit - 1) / kCombineSplit * kCombineSplit;
+  const int nsel = p.B * p.nheads * kSelCtas;
   const int ncomb = cp.B * cp.Hq * kCombineSplit;
   size_t smem = block_select_smem(p.N_max, p.block);
   if (smem > kBlockSelSmemMax) return cudaErrorInvalidValue;
   if (combine_smem_bytes<D>() > smem) smem = combine_smem_bytes<D>();
   cudaLaunchConfig_t cfg{};
-  cfg.gridDim = dim3((unsigned)(nsel_pad + ncomb));
+  cfg.gridDim = dim3((unsigned)(nsel + ncomb));
   cfg.blockDim = dim3(kSelThreads);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = st;
@@ -232,7 +271,7 @@ cudaError_t launch_bsc(const BlockSelParams& p, const CombineParams& cp, cudaStr
   at[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = at;
   cfg.numAttrs = 2;
-  const cudaError_t e = cudaLaunchKernelEx(&cfg, kfn, p, cp, nsel, nsel_pad);
+  const cudaError_t e = cudaLaunchKernelEx(&cfg, kfn, p, cp, nsel);
   if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
@@ -240,7 +279,8 @@ cudaError_t launch_bsc(const BlockSelParams& p, const CombineParams& cp, cudaStr
 }  // namespace
 
 size_t block_select_smem(int N_max, int block) {
-  return (size_t)((N_max + block - 1) / block) * 4;
+  // an mbarrier, then the keys of every block (the shares rounded up to 4)
+  return 16 + ((size_t)((N_max + block - 1) / block) + 4 * kSelCtas) * 4;
 }
 
 cudaError_t launch_block_select_combine(const BlockSelParams& p, const CombineParams& cp,

@@ -19,7 +19,8 @@ struct BlockSelParams {
   int B, Hq, N_max, nwords, k, nheads, block;
   uint8_t heads[128];        // the retrieval heads handled by this launch
 };
-constexpr size_t kBlockSelSmemMax = 128 * 1024;   // block keys of one head, at most
+// block keys of one head, at most 32768 blocks (see block_select_smem)
+constexpr size_t kBlockSelSmemMax = 16 + (32768 + 32) * 4;
 size_t block_select_smem(int N_max, int block);
 // The selection of the retrieval heads and the combine of every head in one
 // launch; just the combine when p.nheads is 0.

@@ -36,6 +36,15 @@ __device__ __forceinline__ void st_async_v4(uint32_t remote, uint4 v, uint32_t r
       : "memory");
 }
 
+// Arrival on another CTA's mbarrier (address from dsmem_map) that also raises
+// its expected transaction bytes by `bytes`.
+__device__ __forceinline__ void mbar_arrive_expect_tx_remote(uint32_t remote_bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.release.cluster.shared::cluster.b64 _, [%0], %1;" ::"r"(
+                   remote_bar),
+               "r"(bytes)
+               : "memory");
+}
+
 // Bounded wait on a local mbarrier whose transaction bytes come from other CTAs
 // of the cluster: acquire at cluster scope, so their stores are visible after.
 __device__ __forceinline__ bool mbar_try_wait_cluster(uint64_t* bar, uint32_t parity,
