@@ -35,7 +35,7 @@ NOALLOC_SCRATCH_BYTES = 64 << 20
 EXPORTED = ("lychee_workspace_size", "lychee_workspace_offsets", "lychee_hybrid_decode_attn",
             "lychee_hybrid_decode_attn_noalloc", "lychee_decode_stack",
             "lychee_check_device_error", "lychee_status_string", "lychee_version",
-            "lychee_profile_begin", "lychee_profile_end")
+            "lychee_profile_begin", "lychee_profile_end", "lychee_append_kv")
 
 
 class Shape(ctypes.Structure):
@@ -79,6 +79,8 @@ def load(path: str | None = None):
         lib.lychee_hybrid_decode_attn_noalloc.restype = ctypes.c_int
         lib.lychee_decode_stack.argtypes = [sp, i32] + [vp] * 10 + [ctypes.c_size_t, vp]
         lib.lychee_decode_stack.restype = ctypes.c_int
+        lib.lychee_append_kv.argtypes = [sp] + [vp] * 6
+        lib.lychee_append_kv.restype = ctypes.c_int
         lib.lychee_check_device_error.argtypes = [vp, vp, u32p]
         lib.lychee_check_device_error.restype = ctypes.c_int
         lib.lychee_status_string.argtypes = [ctypes.c_int]

@@ -418,6 +418,27 @@ lychee_status lychee_decode_stack(const lychee_shape* s, int32_t L, const void* 
   return export_sets(c, seqlens, idx_final);
 }
 
+lychee_status lychee_append_kv(const lychee_shape* s, const void* k_new, const void* v_new,
+                               void* k_cache, void* v_cache, const int32_t* seqlens,
+                               void* stream) {
+  lychee_status st = check_shape(s);
+  if (st != LYCHEE_OK) return st;
+  if (!k_new || !v_new || !k_cache || !v_cache || !seqlens) return LYCHEE_ERR_INVALID_ARG;
+  if (!aligned(k_new, 16) || !aligned(v_new, 16) || !aligned(k_cache, 16) ||
+      !aligned(v_cache, 16))
+    return LYCHEE_ERR_INVALID_ARG;
+  AppendParams p{};
+  p.k_new = k_new;
+  p.v_new = v_new;
+  p.k_cache = k_cache;
+  p.v_cache = v_cache;
+  p.seqlens = seqlens;
+  p.B = s->B; p.Hkv = s->Hkv; p.N_max = s->N_max;
+  p.row_bytes = s->d * (int)elem_size(s);
+  return launch_append_kv(p, static_cast<cudaStream_t>(stream)) == cudaSuccess ? LYCHEE_OK
+                                                                               : LYCHEE_ERR_CUDA;
+}
+
 lychee_status lychee_check_device_error(void* workspace, void* stream, uint32_t* detail) {
   if (!workspace) return LYCHEE_ERR_INVALID_ARG;
   cudaStream_t st = static_cast<cudaStream_t>(stream);

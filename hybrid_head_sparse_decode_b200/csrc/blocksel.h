@@ -27,4 +27,15 @@ size_t block_select_smem(int N_max, int block);
 cudaError_t launch_block_select_combine(const BlockSelParams& p, const CombineParams& cp,
                                         int dtype, int D, cudaStream_t st);
 
+// The current token's K and V rows into the caches at row n_b - 1 (sets.cu).
+struct AppendParams {
+  const void* k_new;         // [B, Hkv, row_bytes]
+  const void* v_new;
+  void* k_cache;             // [B, Hkv, N_max, row_bytes]
+  void* v_cache;
+  const int32_t* seqlens;    // [B]
+  int B, Hkv, N_max, row_bytes;
+};
+cudaError_t launch_append_kv(const AppendParams& p, cudaStream_t st);
+
 }  // namespace lychee

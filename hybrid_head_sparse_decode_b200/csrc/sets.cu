@@ -4,6 +4,7 @@
 // an index row (k_b ascending positions, -1 padded) and a membership bitmap
 // (bit j of word w: position 32w + j is in S).  The attention kernel reads sets
 // as bitmaps so that the G heads of a KV group can be merged word by word.
+#include "blocksel.h"
 #include "common.cuh"
 #include "kernels.h"
 
@@ -132,6 +133,41 @@ cudaError_t launch_build_bits(const BuildBitsParams& p, cudaStream_t st) {
 cudaError_t launch_export(const ExportParams& p, cudaStream_t st) {
   const cudaError_t e =
       launch_pdl(export_kernel, dim3((unsigned)(p.B * p.Hq)), dim3(kThreads), 0, st, p);
+  if (e != cudaSuccess) return e;
+  return cudaGetLastError();
+}
+
+}  // namespace lychee
+
+namespace lychee {
+namespace {
+
+// One CTA per (sequence, KV head): the new K and V rows, 16 bytes per thread.
+__global__ void __launch_bounds__(64) append_kv_kernel(const __grid_constant__ AppendParams p) {
+  pdl_launch_dependents();
+  pdl_wait();
+  const int b = blockIdx.x / p.Hkv;
+  const int n = p.seqlens[b];
+  if (n < 1 || n > p.N_max) return;
+  const size_t unit = blockIdx.x;   // b * Hkv + g
+  const int pieces = p.row_bytes / 16;
+  const uint4* kn = reinterpret_cast<const uint4*>(static_cast<const char*>(p.k_new) + unit * p.row_bytes);
+  const uint4* vn = reinterpret_cast<const uint4*>(static_cast<const char*>(p.v_new) + unit * p.row_bytes);
+  uint4* kc = reinterpret_cast<uint4*>(static_cast<char*>(p.k_cache) +
+                                       (unit * p.N_max + (size_t)(n - 1)) * p.row_bytes);
+  uint4* vc = reinterpret_cast<uint4*>(static_cast<char*>(p.v_cache) +
+                                       (unit * p.N_max + (size_t)(n - 1)) * p.row_bytes);
+  for (int i = threadIdx.x; i < pieces; i += blockDim.x) {
+    kc[i] = kn[i];
+    vc[i] = vn[i];
+  }
+}
+
+}  // namespace
+
+cudaError_t launch_append_kv(const AppendParams& p, cudaStream_t st) {
+  const cudaError_t e =
+      launch_pdl(append_kv_kernel, dim3((unsigned)(p.B * p.Hkv)), dim3(64), 0, st, p);
   if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }

@@ -199,6 +199,23 @@ def decode_stack(q, k_caches, v_caches, seqlens, head_roles, k, *, k_per_seq=Non
     return out, idx_final, idx_layers
 
 
+def append_kv(k_new, v_new, k_cache, v_cache, seqlens, stream=None):
+    """The current token's K/V rows [B,Hkv,d] into the caches [B,Hkv,N_max,d] at
+    row seqlens[b] - 1 (in place).  Returns (k_cache, v_cache)."""
+    B, Hkv, N_max, d = k_cache.shape
+    dt = k_cache.dtype
+    _need_cuda("k_cache", k_cache, dt, (B, Hkv, N_max, d))
+    _need_cuda("v_cache", v_cache, dt, (B, Hkv, N_max, d))
+    _need_cuda("k_new", k_new, dt, (B, Hkv, d))
+    _need_cuda("v_new", v_new, dt, (B, Hkv, d))
+    _need_cuda("seqlens", seqlens, torch.int32, (B,))
+    sh = make_shape(B, Hkv, Hkv, d, N_max, 1, dt)
+    st = N.load().lychee_append_kv(ctypes.byref(sh), _ptr(k_new), _ptr(v_new), _ptr(k_cache),
+                                   _ptr(v_cache), _ptr(seqlens), _stream_handle(stream))
+    _check(st, "lychee_append_kv")
+    return k_cache, v_cache
+
+
 def check_device_error(workspace, stream=None):
     """Synchronise, read and clear the device error word.  Returns (status, bits)."""
     _need_cuda("workspace", workspace, torch.uint8)

@@ -186,6 +186,24 @@ LYCHEE_API lychee_status lychee_decode_stack(const lychee_shape* s, int32_t L, c
                                   int32_t* idx_layers, void* workspace, size_t workspace_bytes,
                                   void* stream);
 
+/* The step before a layer's attention in a decode step: the current token's
+ * key and value rows go into the caches at row n_b - 1 of their sequence (the
+ * calls above read rows j < n_b, the current token included).  The rows are
+ * copied bit for bit; the method's pages describe decoding over a KV cache
+ * that holds the current token but give no rule of their own for the append.
+ *   k_new, v_new      device [B, Hkv, d]         dtype
+ *   k_cache, v_cache  device [B, Hkv, N_max, d]  dtype
+ *   seqlens           device [B] int32; a sequence whose n_b is outside
+ *                     [1, N_max] is left untouched
+ *   stream            cudaStream_t
+ * Only s->B, Hkv, d, N_max, dtype are used (the rest must still form a valid
+ * shape).  Allocates nothing; graph-capturable.  The attention output `out`
+ * [B, Hq, d] of the calls above is, byte for byte, the row-major [B, Hq * d]
+ * matrix an output projection reads: no re-layout step is needed. */
+LYCHEE_API lychee_status lychee_append_kv(const lychee_shape* s, const void* k_new,
+                                          const void* v_new, void* k_cache, void* v_cache,
+                                          const int32_t* seqlens, void* stream);
+
 /* Synchronises `stream`, reads the device error word of `workspace` and clears
  * it.  Returns LYCHEE_OK, LYCHEE_ERR_BAD_INDEX, LYCHEE_ERR_TIMEOUT or
  * LYCHEE_ERR_CUDA.  If detail is not NULL it receives the raw flag bits

@@ -122,6 +122,19 @@ def block_select(s: np.ndarray, kb: int, block: int, cap: int) -> np.ndarray:
     return out
 
 
+def append_kv(k_new, v_new, K, V, seqlens):
+    """The decode step's cache append, written out: copies of K and V [B,Hkv,N,d]
+    with row n_b - 1 of every sequence set to the new rows k_new / v_new
+    [B,Hkv,d]; a sequence with n_b outside [1, N] is left as it is."""
+    K2, V2 = np.array(K, copy=True), np.array(V, copy=True)
+    for b in range(K.shape[0]):
+        n = int(seqlens[b])
+        if 1 <= n <= K.shape[2]:
+            K2[b, :, n - 1] = k_new[b]
+            V2[b, :, n - 1] = v_new[b]
+    return K2, V2
+
+
 def attention_weights(q: np.ndarray, Kg: np.ndarray) -> np.ndarray:
     """A = softmax(q Kg^T / sqrt(d)) for one query head over all rows of Kg [n, d]."""
     dt = _dtype_code(q)

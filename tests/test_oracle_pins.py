@@ -566,3 +566,36 @@ def test_sparse_set_ends_at_first_minus_one():
     bad[0, 1, 9] = 40   # an entry after the end of the set
     with pytest.raises(oracle.OracleError):
         oracle.hybrid_layer(q, K, V, seq, role, bad, 12)
+
+
+# ---- the cache append before a step ------------------------------------------
+
+def test_append_then_layer_is_attention_over_the_extended_cache():
+    """After the append, the oracle's all-retrieval layer over n rows equals
+    torch fp64 softmax(q [K_old; k_new]^T / sqrt(d)) [V_old; v_new]: the new row
+    is the current token the layer reads, and nothing else moved."""
+    g = rng(500)
+    B, Hq, Hkv, d, N = 2, 4, 2, 16, 50
+    q = g.standard_normal((B, Hq, d)).astype(np.float32)
+    K = g.standard_normal((B, Hkv, N, d)).astype(np.float32)
+    V = g.standard_normal((B, Hkv, N, d)).astype(np.float32)
+    kn = g.standard_normal((B, Hkv, d)).astype(np.float32)
+    vn = g.standard_normal((B, Hkv, d)).astype(np.float32)
+    seq = np.array([37, 50], np.int32)
+    K2, V2 = oracle.append_kv(kn, vn, K, V, seq)
+    out, _, _ = oracle.hybrid_layer(q, K2, V2, seq, np.full(Hq, R, np.uint8),
+                                    np.full((B, Hq, 4), -1, np.int32), 4)
+    for b in range(B):
+        n = int(seq[b])
+        for h in range(Hq):
+            gk = h // (Hq // Hkv)
+            Kx = torch.from_numpy(np.concatenate([K[b, gk, :n - 1], kn[b, gk][None]])).double()
+            Vx = torch.from_numpy(np.concatenate([V[b, gk, :n - 1], vn[b, gk][None]])).double()
+            a = torch.softmax(torch.from_numpy(q[b, h]).double() @ Kx.T / math.sqrt(d), 0)
+            assert np.allclose(out[b, h], (a @ Vx).numpy(), rtol=0, atol=1e-12)
+    # rows other than n_b - 1 are untouched; out-of-range lengths change nothing
+    mask = np.ones(N, bool)
+    mask[36] = False
+    assert np.array_equal(K2[0][:, mask], K[0][:, mask])
+    K3, V3 = oracle.append_kv(kn, vn, K, V, np.array([0, 51], np.int32))
+    assert np.array_equal(K3, K) and np.array_equal(V3, V)
