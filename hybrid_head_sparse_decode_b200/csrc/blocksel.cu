@@ -227,7 +227,7 @@ __device__ __forceinline__ void block_select_body(const BlockSelParams& p, int p
 // combine of every head on the next ncomb (the kCombineSplit CTAs of a head are
 // one cluster).
 template <typename T, int D>
-__global__ void __launch_bounds__(kSelThreads, 1)
+__global__ void __launch_bounds__(kSelThreads, D >= 128 ? 2 : 1)
     block_select_combine_kernel(const __grid_constant__ BlockSelParams p,
                                 const __grid_constant__ CombineParams cp, int nsel) {
   static_assert(kSelThreads == kCombThreads, "one block size for both roles");

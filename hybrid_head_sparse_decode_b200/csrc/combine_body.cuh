@@ -23,7 +23,7 @@ __device__ __forceinline__ void store_out<float>(float* p, float v) {
   *p = v;
 }
 
-constexpr int kBatch = 4;
+constexpr int kBatch = 5;
 
 // Merge one state (e = (m, l), a = four elements of acc) into running sums.
 __device__ __forceinline__ void absorb(float2 e, float4 a, float sl, float& m, float& l,
