@@ -181,13 +181,13 @@ def describe(name, prob):
         return {"workload": name, "layers": L, "B": B, "Hq": Hq, "Hkv": Hkv, "d": d,
                 "N": N, "seqlens": [int(x) for x in prob.seqlens.cpu()], "k": prob.k,
                 "retrieval_heads": int(prob.roles.sum()), "layer0": "all retrieval",
-                "io_dtype": "bf16",
+                "io_dtype": "bf16", "accumulate": "fp32",
                 "l2": "no flush: each step reads %.1f GB of K/V (> 126 MB L2)" % (
                     2 * L * B * Hkv * N * d * 2 / 1e9)}
     B, Hq, Hkv, d, N = prob.shape
     return {"workload": name, "layers": 1, "B": B, "Hq": Hq, "Hkv": Hkv, "d": d, "N": N,
             "k": prob.k, "retrieval_heads": int(prob.role.sum()), "io_dtype": "bf16",
-            "l2": "flushed between steps by writing a 256 MB buffer"}
+            "accumulate": "fp32", "l2": "flushed between steps by writing a 256 MB buffer"}
 
 
 def union_rows(prob, idx_layers):
@@ -362,7 +362,7 @@ def run_lychee(args, rank, world, device):
         "metric": METRIC, "value": round(us_step_job, 3), "unit": UNIT, "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_step, 5),
         "higher_is_better": False, "scaling": "weak", "vs_baseline": None,
-        "dtype": "fp32", "data": "synthetic (seeded; planted high-affinity keys)",
+        "dtype": "bf16", "data": "synthetic (seeded; planted high-affinity keys)",
         "config": dict(describe(args.workload, prob),
                        select="argsTopK" if blk <= 1 else f"blocks of {blk}"),
         "us_per_layer": round(ms_step * 1e3 / L, 3),
