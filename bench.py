@@ -190,6 +190,12 @@ def describe(name, prob):
             "accumulate": "fp32", "l2": "flushed between steps by writing a 256 MB buffer"}
 
 
+def nearest_rank(sorted_xs, q):
+    """The q-quantile of a sorted list by the nearest-rank rule."""
+    n = len(sorted_xs)
+    return sorted_xs[min(n - 1, max(0, math.ceil(q * n) - 1))]
+
+
 def union_rows(prob, idx_layers):
     """Rows the method must read per layer and group: n_b for a group holding a
     retrieval head, |union of the heads' incoming sets| for a sparse-only group.
@@ -290,6 +296,15 @@ def run_lychee(args, rank, world, device):
         for _ in range(args.steps):
             step()
         torch.cuda.synchronize()
+    # per-step spread: an event after every step of another pass of the same steps
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps + 1)]
+    torch.cuda.synchronize()
+    ev[0].record(stream)
+    for i in range(args.steps):
+        step()
+        ev[i + 1].record(stream)
+    torch.cuda.synchronize()
+    per_step = sorted(ev[i].elapsed_time(ev[i + 1]) for i in range(args.steps))
     ms_total = max_over_ranks(ms_total, world, device)
     ms_step = ms_total / args.steps
     recs = prof.records
@@ -366,6 +381,10 @@ def run_lychee(args, rank, world, device):
         "config": dict(describe(args.workload, prob),
                        select="argsTopK" if blk <= 1 else f"blocks of {blk}"),
         "us_per_layer": round(ms_step * 1e3 / L, 3),
+        "step_ms_spread": {"p10": round(nearest_rank(per_step, 0.1), 5),
+                           "median": round(nearest_rank(per_step, 0.5), 5),
+                           "p90": round(nearest_rank(per_step, 0.9), 5),
+                           "steps": len(per_step), "rank": rank},
         "step_hbm_gbs_union": round(sum(union_bytes) / (ms_step * 1e-3) / 1e9, 1),
         "step_hbm_gbs_literal": round(sum(literal_bytes) / (ms_step * 1e-3) / 1e9, 1),
         "bytes_per_step": {"union": sum(union_bytes), "literal": sum(literal_bytes),

@@ -69,3 +69,12 @@ def test_single_rank_needs_no_process_group():
     import bench
     assert bench.max_over_ranks(3.25, 1, torch.device("cpu")) == 3.25
     assert bench.job_us_per_step(3.25, 1) == pytest.approx(3250.0)
+
+
+def test_step_spread_uses_nearest_rank():
+    sys.path.insert(0, ROOT)
+    import bench
+    xs = sorted([5.0, 1.0, 2.0, 3.0, 4.0, 6.0, 7.0, 8.0, 9.0, 10.0])
+    assert (bench.nearest_rank(xs, 0.1), bench.nearest_rank(xs, 0.5),
+            bench.nearest_rank(xs, 0.9)) == (1.0, 5.0, 9.0)
+    assert bench.nearest_rank([3.0], 0.9) == 3.0
