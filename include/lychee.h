@@ -22,9 +22,13 @@
  *     k_b = min(k_per_seq[b] (or k when k_per_seq is NULL), k, n_b).
  *   - argsTopK ranks positions by larger logit first and, on equal logits, by
  *     lower position; the returned set is in ascending position order.
- *   - Element types: LYCHEE_BF16 (16-bit bfloat16) or LYCHEE_FP32.  Arithmetic
- *     is fp32 with fp32 accumulation; outputs are rounded to the input type
- *     (round to nearest even).
+ *   - Element types: LYCHEE_BF16 (16-bit bfloat16) or LYCHEE_FP32.  With fp32
+ *     caches all arithmetic is fp32.  With bf16 caches the products q.K and
+ *     p.V run on the tensor cores with bf16 operands and fp32 accumulation:
+ *     the logits are exact bf16 products summed in fp32, and the softmax
+ *     weights p are rounded to bf16 for p.V, with the normaliser summing the
+ *     same rounded weights.  Softmax, top-k and combine are fp32.  Outputs are
+ *     rounded to the input type (round to nearest even).
  *   - Ownership: the caller owns every buffer.  The library allocates no
  *     memory, never synchronises inside a call, and launches only on `stream`
  *     (a cudaStream_t; NULL = the legacy default stream), so a call can be
@@ -38,6 +42,14 @@
  *     trap: the offending entry is skipped or clamped, a flag is set in the
  *     workspace, and lychee_check_device_error() reports it.
  *   - Device pointers must be 16-byte aligned (q, caches, out, workspace).
+ *   - Threads and devices: the first call of each kernel configuration in a
+ *     process sets that kernel's attributes (dynamic shared memory, cluster
+ *     size) on the current device and remembers that it did, with no lock.
+ *     Make the first call of each configuration from one host thread, and use
+ *     one device per process: a second device in the same process is not
+ *     set up, and its launches may be refused (LYCHEE_ERR_CUDA).
+ *     After the first calls, calls on different streams with their own
+ *     workspaces may come from any thread.
  */
 #ifndef LYCHEE_H
 #define LYCHEE_H
