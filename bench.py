@@ -219,7 +219,7 @@ def union_rows(prob, idx_layers):
                     mark = torch.zeros(n, dtype=torch.bool, device=dev)
                     for h in hs:
                         row = idx_layers[l - 1, b, h, :kb].long()
-                        mark[row] = True
+                        mark[row[row >= 0]] = True   # a set ends at its first -1
                     u += int(mark.sum())
                     lit += kb
         union.append(u)

@@ -78,3 +78,50 @@ def test_step_spread_uses_nearest_rank():
     assert (bench.nearest_rank(xs, 0.1), bench.nearest_rank(xs, 0.5),
             bench.nearest_rank(xs, 0.9)) == (1.0, 5.0, 9.0)
     assert bench.nearest_rank([3.0], 0.9) == 3.0
+
+
+def test_union_rows_counts_each_group_row_once():
+    """The roofline's algorithmic bytes: n_b rows for a group with a retrieval
+    head, the size of the union of the heads' sets otherwise (sets end at their
+    first -1), counted here by brute force over Python sets."""
+    sys.path.insert(0, ROOT)
+    import bench
+    from types import SimpleNamespace
+    g = torch.Generator().manual_seed(7)
+    L, B, Hq, Hkv, d, N, k = 3, 2, 8, 2, 64, 40, 12
+    G = Hq // Hkv
+    seqlens = torch.tensor([40, 23], dtype=torch.int32)
+    kb = [12, 6]
+    roles = torch.zeros(L, Hq, dtype=torch.uint8)
+    roles[0] = 1
+    roles[1, 5] = 1                      # layer 1: group 1 dense, group 0 sparse-only
+    idx = torch.full((L, B, Hq, k), -1, dtype=torch.int32)
+    for l in range(L):
+        for b in range(B):
+            for h in range(Hq):
+                m = kb[b] - (h % 3)      # some sets end early, at their first -1
+                pos = torch.randperm(int(seqlens[b]), generator=g)[:m].sort().values
+                idx[l, b, h, :m] = pos.int()
+    prob = SimpleNamespace(shape=(L, B, Hq, Hkv, d, N), roles=roles, seqlens=seqlens,
+                           meta={"kb": kb})
+    union, literal, dense = bench.union_rows(prob, idx)
+    for l in range(L):
+        want_u = want_l = 0
+        for b in range(B):
+            n = int(seqlens[b])
+            for grp in range(Hkv):
+                hs = range(grp * G, grp * G + G)
+                if any(int(roles[l, h]) for h in hs):
+                    want_u += n
+                    want_l += n
+                else:
+                    rows = set()
+                    for h in hs:
+                        for x in idx[l - 1, b, h].tolist():
+                            if x < 0:
+                                break
+                            rows.add(x)
+                    want_u += len(rows)
+                    want_l += kb[b]
+        assert union[l] == want_u and literal[l] == want_l
+        assert dense[l] == Hkv * int(seqlens.sum())
