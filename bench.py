@@ -190,6 +190,10 @@ def describe(name, prob):
             "accumulate": "fp32", "l2": "flushed between steps by writing a 256 MB buffer"}
 
 
+def select_name(block):
+    return "argsTopK" if block <= 1 else f"blocks of {block}"
+
+
 def nearest_rank(sorted_xs, q):
     """The q-quantile of a sorted list by the nearest-rank rule."""
     n = len(sorted_xs)
@@ -379,7 +383,7 @@ def run_lychee(args, rank, world, device):
         "higher_is_better": False, "scaling": "weak", "vs_baseline": None,
         "dtype": "bf16", "data": "synthetic (seeded; planted high-affinity keys)",
         "config": dict(describe(args.workload, prob),
-                       select="argsTopK" if blk <= 1 else f"blocks of {blk}"),
+                       select=select_name(blk)),
         "us_per_layer": round(ms_step * 1e3 / L, 3),
         "step_ms_spread": {"p10": round(nearest_rank(per_step, 0.1), 5),
                            "median": round(nearest_rank(per_step, 0.5), 5),
@@ -409,9 +413,9 @@ def run_lychee(args, rank, world, device):
 
 
 # ---------------------------------------------------------------- the oracle arm
-def oracle_chain_time(prob, layers, nthreads):
-    """Time the oracle's own chain over the given leading layers of the stack;
-    returns per-layer seconds."""
+def oracle_chain_time(prob, layers, nthreads, block=0):
+    """Time the oracle's own chain over the given leading layers of the stack
+    (block > 1: block-granular selection); returns per-layer seconds."""
     import numpy as np
 
     import oracle
@@ -429,7 +433,8 @@ def oracle_chain_time(prob, layers, nthreads):
         q, K, V = bits(prob.q[l]), bits(prob.k_caches[l]), bits(prob.v_caches[l])
         t = time.perf_counter()
         _, idx, _ = oracle.hybrid_layer(q, K, V, seqlens, prob.roles[l].numpy(), idx, prob.k,
-                                        k_per_seq=kps, nthreads=nthreads)
+                                        k_per_seq=kps, nthreads=nthreads,
+                                        block=max(1, block))
         times.append(time.perf_counter() - t)
     return times
 
@@ -441,13 +446,13 @@ def scale_to_step(times, L):
     return times[0] + sum(rest) / len(rest) * (L - 1)
 
 
-def cpu_baseline(prob, sample_layers=8):
+def cpu_baseline(prob, sample_layers=8, block=0):
     import oracle
     oracle.build()
     L = prob.shape[0]
     nthreads = os.cpu_count() or 1
     B, Hq = prob.shape[1], prob.shape[2]
-    times = oracle_chain_time(prob, min(sample_layers, L), nthreads)
+    times = oracle_chain_time(prob, min(sample_layers, L), nthreads, block)
     est = scale_to_step(times, L)
     return {"value": round(est * 1e6, 1), "unit": UNIT, "cores": min(nthreads, B * Hq),
             "kind": "oracle",
@@ -470,10 +475,10 @@ def run_reference(args, rank, world):
     nthreads = os.cpu_count() or 1
     layers = 2
     for _ in range(args.warmup if args.warmup < 3 else 1):
-        oracle_chain_time(prob, 1, nthreads)
+        oracle_chain_time(prob, 1, nthreads, args.block)
     per = []
     for _ in range(args.steps):
-        per.append(scale_to_step(oracle_chain_time(prob, layers, nthreads), L))
+        per.append(scale_to_step(oracle_chain_time(prob, layers, nthreads, args.block), L))
     us = statistics.median(per) * 1e6
     B, Hq = prob.shape[1], prob.shape[2]
     cb = {"value": round(us, 1), "unit": UNIT, "cores": min(nthreads, B * Hq), "kind": "oracle",
@@ -483,7 +488,8 @@ def run_reference(args, rank, world):
             "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": round(us / 1e3, 3), "higher_is_better": False, "scaling": "weak",
             "vs_baseline": None, "dtype": "f64", "data": "synthetic (seeded)",
-            "config": describe(args.workload, prob), "cpu_baseline": cb,
+            "config": dict(describe(args.workload, prob), select=select_name(args.block)),
+            "cpu_baseline": cb,
             "e2e": {"value": round(us, 1), "unit": UNIT, "h2d_bytes_per_step": 0,
                     "d2h_bytes_per_step": 0}}
 
@@ -524,7 +530,7 @@ def main():
     res, prob, _ = run_lychee(args, rank, world, device)
     if rank == 0:
         if world == 1 and not args.no_cpu_baseline:
-            res["cpu_baseline"] = cpu_baseline(prob)
+            res["cpu_baseline"] = cpu_baseline(prob, block=args.block)
         print(json.dumps(res), flush=True)
     if world > 1:
         torch.distributed.barrier()

@@ -125,3 +125,14 @@ def test_union_rows_counts_each_group_row_once():
                     want_l += kb[b]
         assert union[l] == want_u and literal[l] == want_l
         assert dense[l] == Hkv * int(seqlens.sum())
+
+
+@pytest.mark.parametrize("block", [0, 32])
+def test_reference_arm_on_rank0_prints_the_contract_keys(block):
+    sys.path.insert(0, ROOT)
+    import bench
+    args = argparse.Namespace(workload="qwen3_stack_256x2", steps=2, warmup=0, block=block)
+    res = bench.run_reference(args, 0, 1)
+    assert res["impl"] == "reference" and res["value"] > 0 and not res["higher_is_better"]
+    assert res["e2e"]["value"] == res["value"] and res["cpu_baseline"]["kind"] == "oracle"
+    assert res["config"]["select"] == ("argsTopK" if block == 0 else "blocks of 32")
