@@ -136,3 +136,12 @@ def test_reference_arm_on_rank0_prints_the_contract_keys(block):
     assert res["impl"] == "reference" and res["value"] > 0 and not res["higher_is_better"]
     assert res["e2e"]["value"] == res["value"] and res["cpu_baseline"]["kind"] == "oracle"
     assert res["config"]["select"] == ("argsTopK" if block == 0 else "blocks of 32")
+
+
+def test_cpu_baseline_leg_runs_on_host_tensors():
+    sys.path.insert(0, ROOT)
+    import bench
+    prob = bench.make_workload("qwen3_stack_256x3", torch.device("cpu"))
+    cb = bench.cpu_baseline(prob, sample_layers=2, block=32)
+    assert cb["kind"] == "oracle" and cb["value"] > 0 and cb["cores"] >= 1
+    assert "layers 0..1" in cb["sample"]
