@@ -233,8 +233,9 @@ LYCHEE_API int32_t lychee_version(void);
  * events recorded on its launch stream, up to max_launches launches (later
  * launches run unrecorded).  lychee_profile_end synchronises on the recorded
  * events and writes, for the first min(n, capacity) launches, the kind
- * (0 attention, 1 top-k, 2 combine, 3 set->bitmap, 4 bitmap->set, 5 top-k and
- * combine in one launch) and the
+ * (0 attention, 1 top-k, 2 combine, 3 set->bitmap, 4 bitmap->set, 5 the
+ * retrieval heads' selection -- argsTopK, or the block selection when
+ * s->block > 1 -- and the combine in one launch) and the
  * elapsed milliseconds; *n_out receives n.  Process-global state: one profiling
  * session at a time.  Events are created on the current device on first use
  * and kept for reuse. */
