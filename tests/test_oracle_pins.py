@@ -493,6 +493,13 @@ def test_block_select_properties(seed):
     _block_props(s, kb, blk, sel)
 
 
+def test_block_select_golden():
+    fx = json.load(open(os.path.join(GOLDEN, "block_select_small.json")))
+    for c in fx["cases"]:
+        got = oracle.block_select(np.array(c["s"]), c["kb"], c["block"], c["cap"])
+        assert got.tolist() == c["expect"], c
+
+
 def test_block_select_of_one_position_blocks_is_token_topk():
     g = rng(77)
     for n in (1, 5, 33, 200):
