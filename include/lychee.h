@@ -132,7 +132,9 @@ LYCHEE_API lychee_status lychee_workspace_offsets(const lychee_shape* s, size_t*
  *   idx_in    device [B, Hq, k] int32; rows of sparse heads are read (their
  *             entries before the first -1, at most k_b of them, strictly
  *             ascending, in [0, n_b)); may be NULL only when every head is a
- *             retrieval head
+ *             retrieval head.  A block-granular set may hold more than k_b
+ *             positions (k_b < block); this call reads only its first k_b,
+ *             whereas lychee_decode_stack hands every set on whole
  *   out       device [B, Hq, d] dtype
  *   idx_out   device [B, Hq, k] int32: retrieval heads get argsTopK of their
  *             logits, or their block-granular set (s->block), ascending, -1

@@ -30,8 +30,9 @@
  *   - GQA: query head h reads KV head floor(h / G), G = Hq / Hkv.
  *   - A sparse head reads its own layer's K/V at the inherited positions; only
  *     the index set is shared between layers.
- *   - A set row ends at its first -1 (at most k_b entries are read), so a set
- *     may hold fewer than k_b positions; a head with an empty set outputs 0.
+ *   - A set row ends at its first -1 (or at the row capacity k); a sparse head
+ *     attends over all of it, which may be fewer than k_b positions, or more
+ *     (a block-granular set when k_b < B).  A head with an empty set outputs 0.
  *   - Block-granular selection (the block-sparse decoding kernel of the same
  *     page; the block-level maximum scores and the k/B top blocks of the
  *     HySparse page, B = 64): a block's score is the largest logit among its
@@ -232,33 +233,34 @@ done:
   return rc;
 }
 
-/* Sparse attention over S: its entries before the first -1, at most kb of them
- * (distinct and in [0, n); a non-negative entry after a -1 is an error).  An
+/* Sparse attention over the whole set S it was handed (method step (4)): the
+ * row's entries before its first -1, within the row capacity cap (distinct and
+ * in [0, n); a non-negative entry after a -1 is an error).  The budget k_b does
+ * not bound the set: a block-granular set may hold more than k_b positions.  An
  * empty set gives out = 0.  idx_out (may be NULL) receives S unchanged (all cap
  * entries). */
 static int sparse_head(const void *q, size_t q_off, const void *K, const void *V,
-                       size_t kv_off, int n, int d, int dt, const int32_t *S, int kb,
-                       int cap, double *out, int32_t *idx_out) {
-  if (kb < 1) return OR_EARG;
-  int kv = 0;
-  while (kv < kb && S[kv] >= 0) ++kv;
-  for (int t = kv; t < kb; ++t)
+                       size_t kv_off, int n, int d, int dt, const int32_t *S, int cap,
+                       double *out, int32_t *idx_out) {
+  if (cap < 1) return OR_EARG;
+  int m = 0;
+  while (m < cap && S[m] >= 0) ++m;
+  for (int t = m; t < cap; ++t)
     if (S[t] >= 0) return OR_EINDEX;
-  if (kv == 0) {
+  if (m == 0) {
     for (int i = 0; i < d; ++i) out[i] = 0.0;
     if (idx_out) memcpy(idx_out, S, sizeof(int32_t) * (size_t)cap);
     return OR_OK;
   }
-  kb = kv;
   unsigned char *seen = (unsigned char *)calloc((size_t)n, 1);
-  double *s = (double *)malloc(sizeof(double) * (size_t)kb);
-  double *p = (double *)malloc(sizeof(double) * (size_t)kb);
+  double *s = (double *)malloc(sizeof(double) * (size_t)m);
+  double *p = (double *)malloc(sizeof(double) * (size_t)m);
   int rc = OR_OK;
   if (!seen || !s || !p) {
     rc = OR_ENOMEM;
     goto done;
   }
-  for (int t = 0; t < kb; ++t) {
+  for (int t = 0; t < m; ++t) {
     int32_t j = S[t];
     if (j < 0 || j >= n || seen[j]) {
       rc = OR_EINDEX;
@@ -266,9 +268,9 @@ static int sparse_head(const void *q, size_t q_off, const void *K, const void *V
     }
     seen[j] = 1;
   }
-  logits_rows(q, q_off, K, kv_off, d, dt, S, kb, s);
-  double z = softmax_unnormalised(s, kb, p);
-  weighted_values(p, z, V, kv_off, d, dt, S, kb, out);
+  logits_rows(q, q_off, K, kv_off, d, dt, S, m, s);
+  double z = softmax_unnormalised(s, m, p);
+  weighted_values(p, z, V, kv_off, d, dt, S, m, out);
   if (idx_out) memcpy(idx_out, S, sizeof(int32_t) * (size_t)cap);
 done:
   free(seen);
@@ -299,7 +301,8 @@ static int check_shape(int B, int Hq, int Hkv, int d, int N_max, int k, int dt) 
  *   seqlens  [B]                    1 <= n_b <= N_max
  *   k_per_seq[B] or NULL            k_b = min(k_per_seq[b] or k, n_b)
  *   role     [Hq]                   1 = retrieval, 0 = sparse
- *   idx_in   [B, Hq, k]             rows of sparse heads are read (first k_b entries)
+ *   idx_in   [B, Hq, k]             rows of sparse heads are read (entries before the
+ *                                   first -1, up to k)
  *   out      [B, Hq, d]   double
  *   logits   [B, Hq, N_max] double or NULL: s_j of retrieval heads for j < n_b
  *   idx_out  [B, Hq, k]             retrieval: top-k set; sparse: idx_in row copied
@@ -339,7 +342,7 @@ int oracle_hybrid_layer(int B, int Hq, int Hkv, int d, int N_max, int k, int dt,
       if (!idx_in) {
         r = OR_EARG;
       } else {
-        r = sparse_head(q, q_off, K, V, kv_off, n, d, dt, idx_in + row * (size_t)k, kb, k,
+        r = sparse_head(q, q_off, K, V, kv_off, n, d, dt, idx_in + row * (size_t)k, k,
                         out + row * (size_t)d, idx_out ? idx_out + row * (size_t)k : NULL);
       }
     }

@@ -575,6 +575,63 @@ def test_sparse_set_ends_at_first_minus_one():
         oracle.hybrid_layer(q, K, V, seq, role, bad, 12)
 
 
+def _torch_attn_over(qv, Kg, Vg, rows):
+    """torch fp64 softmax(q K[S]^T / sqrt(d)) V[S] over the given positions."""
+    Kx = torch.from_numpy(Kg[rows].astype(np.float64))
+    Vx = torch.from_numpy(Vg[rows].astype(np.float64))
+    qx = torch.from_numpy(qv.astype(np.float64))
+    w = torch.softmax(Kx @ qx / math.sqrt(qv.size), dim=0)
+    return (w @ Vx).numpy()
+
+
+def test_sparse_head_attends_over_the_whole_handed_set():
+    """Step (4): a sparse head attends over every position of the set it was
+    handed, even when the set holds more than the budget k_b (block sets when
+    k_b < B); the budget bounds what a retrieval head selects, not what a
+    sparse head reads."""
+    g = rng(11)
+    B, Hq, Hkv, d, N, k = 1, 2, 1, 16, 64, 20
+    q = g.standard_normal((B, Hq, d)).astype(np.float32)
+    K = g.standard_normal((B, Hkv, N, d)).astype(np.float32)
+    V = g.standard_normal((B, Hkv, N, d)).astype(np.float32)
+    rows = np.sort(g.choice(N, 15, replace=False)).astype(np.int32)
+    idx = np.full((B, Hq, k), -1, np.int32)
+    idx[0, 1, :15] = rows
+    out, idx_out, _ = oracle.hybrid_layer(q, K, V, np.array([N], np.int32),
+                                          np.array([R, S], np.uint8), idx, k,
+                                          k_per_seq=np.array([4], np.int32))
+    np.testing.assert_allclose(out[0, 1], _torch_attn_over(q[0, 1], K[0, 0], V[0, 0], rows),
+                               rtol=0, atol=1e-12)
+    assert np.array_equal(idx_out[0, 1], idx[0, 1])
+
+
+def test_block_stack_short_sequence_hands_on_the_whole_block():
+    """A block-mode stack where k_b < B: layer 0's retrieval head keeps one whole
+    block (B positions, more than k_b), and the same-position sparse head of
+    layer 1 attends over all of that block."""
+    g = rng(12)
+    L, B, Hq, Hkv, d, N, blk = 2, 1, 2, 1, 16, 96, 32
+    n, k = 90, 32
+    q = g.standard_normal((L, B, Hq, d)).astype(np.float32)
+    Ks = [g.standard_normal((B, Hkv, N, d)).astype(np.float32) for _ in range(L)]
+    Vs = [g.standard_normal((B, Hkv, N, d)).astype(np.float32) for _ in range(L)]
+    roles = np.array([[R, R], [R, S]], np.uint8)
+    kps = np.array([5], np.int32)                      # k_b = 5 < B = 32
+    out, _, layers = oracle.stack(q, Ks, Vs, np.array([n], np.int32), roles, k,
+                                  k_per_seq=kps, want_layers=True, block=blk)
+    S1 = layers[0, 0, 1]
+    m = int((S1 >= 0).sum())
+    assert m == blk and np.all(S1[m:] == -1)            # one whole block, not 5 positions
+    c = int(S1[0]) // blk
+    assert S1[:m].tolist() == list(range(c * blk, c * blk + blk))
+    s0 = (Ks[0][0, 0, :n].astype(np.float64) @ q[0, 0, 1].astype(np.float64)) / math.sqrt(d)
+    assert all(s0[c * blk:(c + 1) * blk].max() >= s0[o * blk:min(n, o * blk + blk)].max()
+               for o in range(-(-n // blk)))
+    np.testing.assert_allclose(out[1, 0, 1],
+                               _torch_attn_over(q[1, 0, 1], Ks[1][0, 0], Vs[1][0, 0], S1[:m]),
+                               rtol=0, atol=1e-12)
+
+
 # ---- the cache append before a step ------------------------------------------
 
 def test_append_then_layer_is_attention_over_the_extended_cache():
