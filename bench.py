@@ -222,8 +222,10 @@ def union_rows(prob, idx_layers):
                 else:
                     mark = torch.zeros(n, dtype=torch.bool, device=dev)
                     for h in hs:
-                        row = idx_layers[l - 1, b, h, :kb].long()
-                        mark[row[row >= 0]] = True   # a set ends at its first -1
+                        # the whole set the head was handed: entries before the
+                        # first -1 (a block set may hold more than k_b)
+                        row = idx_layers[l - 1, b, h].long()
+                        mark[row[row >= 0]] = True
                     u += int(mark.sum())
                     lit += kb
         union.append(u)

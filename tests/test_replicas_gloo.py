@@ -99,7 +99,8 @@ def test_union_rows_counts_each_group_row_once():
     for l in range(L):
         for b in range(B):
             for h in range(Hq):
-                m = kb[b] - (h % 3)      # some sets end early, at their first -1
+                # some sets end early at their first -1, one holds more than k_b
+                m = kb[b] - (h % 3) if h != 6 else min(k, int(seqlens[b]))
                 pos = torch.randperm(int(seqlens[b]), generator=g)[:m].sort().values
                 idx[l, b, h, :m] = pos.int()
     prob = SimpleNamespace(shape=(L, B, Hq, Hkv, d, N), roles=roles, seqlens=seqlens,
