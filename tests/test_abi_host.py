@@ -128,6 +128,35 @@ def test_stack_rejects_bad_arguments_on_host(lib):
     assert call_stack(lib, s, 2, [1] * 4 + [0] * 4, ws_bytes=256) == N.ERR_WORKSPACE
 
 
+def test_append_rejects_bad_arguments_on_host(lib):
+    s = shape()
+    ok = [FAKE] * 5
+    for i in range(5):                                   # every pointer is required
+        args = list(ok)
+        args[i] = None
+        assert lib.lychee_append_kv(ctypes.byref(s), *args, None) == N.ERR_INVALID_ARG
+    args = list(ok)
+    args[2] = FAKE + 8                                   # a cache not 16-byte aligned
+    assert lib.lychee_append_kv(ctypes.byref(s), *args, None) == N.ERR_INVALID_ARG
+    assert lib.lychee_append_kv(None, *ok, None) == N.ERR_INVALID_ARG
+    assert lib.lychee_append_kv(ctypes.byref(shape(d=96)), *ok, None) == N.ERR_UNSUPPORTED
+
+
+def test_noalloc_refuses_shapes_beyond_its_scratch_on_host(lib):
+    """The static-scratch layer call checks the shape and the scratch size
+    before it looks the scratch up on a device."""
+    def call(sh):
+        r = (ctypes.c_uint8 * sh.Hq)(*([1] * sh.Hq))
+        return lib.lychee_hybrid_decode_attn_noalloc(
+            ctypes.byref(sh), FAKE, FAKE, FAKE, FAKE, None, ctypes.cast(r, ctypes.c_void_p),
+            None, FAKE, FAKE, None, None)
+    big = N.Shape(2, 32, 8, 128, 131072, N.BF16, 39321, 0)
+    assert lib.lychee_workspace_size(ctypes.byref(big)) > N.NOALLOC_SCRATCH_BYTES
+    assert call(big) == N.ERR_WORKSPACE
+    assert call(shape(Hq=6, Hkv=4)) == N.ERR_INVALID_ARG
+    assert call(shape(d=96)) == N.ERR_UNSUPPORTED
+
+
 def test_status_strings(lib):
     for st in range(7):
         assert lib.lychee_status_string(st)
