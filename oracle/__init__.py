@@ -4,8 +4,10 @@ TEST INFRASTRUCTURE ONLY.  Only ``tests/``, ``__graft_entry__.smoke()`` and the
 ``cpu_baseline`` / ``--impl reference`` legs of ``bench.py`` may import this
 package.  The CUDA library never calls it and shares no code with it.
 
-The arithmetic lives in ``lychee_oracle.c`` (plain C, fp64); this module only
-compiles it with gcc and marshals numpy arrays through ctypes.  The method it
+The attention, selection and stack arithmetic lives in ``lychee_oracle.c``
+(plain C, fp64); this module only compiles it with gcc and marshals numpy
+arrays through ctypes.  The head roles from HardKuma gate parameters (method
+steps (2) and (7)) are in ``hardkuma.py`` (numpy / scipy, fp64).  The method it
 follows is the seven-step description on the page "LycheeDecode: Accelerating
 Long-Context LLM Inference via Hybrid-Head Sparse Decoding"
 (paper.rainbus.top/paper/2602.04541): steps (1), (3), (4) and (7).
