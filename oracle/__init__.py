@@ -7,7 +7,9 @@ package.  The CUDA library never calls it and shares no code with it.
 The attention, selection and stack arithmetic lives in ``lychee_oracle.c``
 (plain C, fp64); this module only compiles it with gcc and marshals numpy
 arrays through ctypes.  The head roles from HardKuma gate parameters (method
-steps (2) and (7)) are in ``hardkuma.py`` (numpy / scipy, fp64).  The method it
+steps (2) and (7)) are in ``hardkuma.py`` (numpy / scipy, fp64), and the
+sliding-window branch of sparse heads with its sigmoid gate (the HySparse
+page's methodology) in ``swa.py`` (numpy, fp64).  The method it
 follows is the seven-step description on the page "LycheeDecode: Accelerating
 Long-Context LLM Inference via Hybrid-Head Sparse Decoding"
 (paper.rainbus.top/paper/2602.04541): steps (1), (3), (4) and (7).
