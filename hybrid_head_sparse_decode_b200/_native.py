@@ -32,10 +32,11 @@ ROLE_RETRIEVAL = 1
 # LYCHEE_NOALLOC_SCRATCH_BYTES of include/lychee.h
 NOALLOC_SCRATCH_BYTES = 64 << 20
 
-EXPORTED = ("lychee_workspace_size", "lychee_workspace_offsets", "lychee_hybrid_decode_attn",
+EXPORTED = ("lychee_workspace_size", "lychee_layer_workspace_size", "lychee_workspace_offsets", "lychee_hybrid_decode_attn",
             "lychee_hybrid_decode_attn_noalloc", "lychee_decode_stack",
             "lychee_check_device_error", "lychee_status_string", "lychee_version",
-            "lychee_profile_begin", "lychee_profile_end", "lychee_append_kv")
+            "lychee_profile_begin", "lychee_profile_end", "lychee_append_kv",
+            "lychee_hardkuma_roles", "lychee_hybrid_decode_attn_swa", "lychee_decode_stack_swa")
 
 
 class Shape(ctypes.Structure):
@@ -69,6 +70,8 @@ def load(path: str | None = None):
         sp = ctypes.POINTER(Shape)
         lib.lychee_workspace_size.argtypes = [sp]
         lib.lychee_workspace_size.restype = ctypes.c_size_t
+        lib.lychee_layer_workspace_size.argtypes = [sp]
+        lib.lychee_layer_workspace_size.restype = ctypes.c_size_t
         lib.lychee_workspace_offsets.argtypes = [sp, ctypes.POINTER(ctypes.c_size_t),
                                                  ctypes.POINTER(ctypes.c_size_t),
                                                  ctypes.POINTER(i32)]
@@ -79,8 +82,17 @@ def load(path: str | None = None):
         lib.lychee_hybrid_decode_attn_noalloc.restype = ctypes.c_int
         lib.lychee_decode_stack.argtypes = [sp, i32] + [vp] * 10 + [ctypes.c_size_t, vp]
         lib.lychee_decode_stack.restype = ctypes.c_int
+        lib.lychee_hybrid_decode_attn_swa.argtypes = [sp] + [vp] * 9 + [i32] + [vp] * 4 + [
+            ctypes.c_size_t, vp]
+        lib.lychee_hybrid_decode_attn_swa.restype = ctypes.c_int
+        lib.lychee_decode_stack_swa.argtypes = [sp, i32] + [vp] * 8 + [i32] + [vp] * 5 + [
+            ctypes.c_size_t, vp]
+        lib.lychee_decode_stack_swa.restype = ctypes.c_int
         lib.lychee_append_kv.argtypes = [sp] + [vp] * 6
         lib.lychee_append_kv.restype = ctypes.c_int
+        lib.lychee_hardkuma_roles.argtypes = [vp, vp, i32, i32, ctypes.c_double, ctypes.c_double,
+                                              i32, vp, vp, vp, vp]
+        lib.lychee_hardkuma_roles.restype = ctypes.c_int
         lib.lychee_check_device_error.argtypes = [vp, vp, u32p]
         lib.lychee_check_device_error.restype = ctypes.c_int
         lib.lychee_status_string.argtypes = [ctypes.c_int]

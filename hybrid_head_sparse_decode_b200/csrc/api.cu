@@ -21,8 +21,17 @@ namespace {
 
 constexpr int kVersion = 100;   // 0.1.0
 
+// Workspace regions.  The single-layer call uses the first set of logits and
+// partial states and ends at `layer_total`; the stack alternates two logits
+// regions and three partial-state regions between consecutive layers (layer l
+// uses logits l % 2 and partials l % 3), so that a layer's attention can run
+// while the previous layer's selection reads its logits and the layer before
+// that is still being combined.
+constexpr int kLogitBufs = 2;
+constexpr int kPartBufs = 3;
 struct Layout {
-  size_t logits, part_ml, part_acc, part_n, bitmaps, total;
+  size_t logits[kLogitBufs], part_ml[kPartBufs], part_acc[kPartBufs], part_n[kPartBufs];
+  size_t bitmaps, layer_total, total;
   int nchunk, nwords;
 };
 
@@ -56,17 +65,29 @@ Layout layout_of(const lychee_shape* s) {
   L.nchunk = (s->N_max + kChunkMin - 1) / kChunkMin;   // room for the shortest chunk
   L.nwords = (s->N_max + 31) / 32;
   const size_t bh = (size_t)s->B * s->Hq;
+  const size_t logits_b = align256(bh * s->N_max * 4);
+  const size_t ml_b = align256(bh * L.nchunk * kPartSlots * 2 * 4);
+  const size_t acc_b = align256(bh * L.nchunk * kPartSlots * s->d * 4);
+  const size_t n_b = align256(bh * L.nchunk * 4);
   size_t off = sizeof(WsHeader);
-  L.logits = off;
-  off += align256(bh * s->N_max * 4);
-  L.part_ml = off;
-  off += align256(bh * L.nchunk * kPartSlots * 2 * 4);
-  L.part_acc = off;
-  off += align256(bh * L.nchunk * kPartSlots * s->d * 4);
-  L.part_n = off;
-  off += align256(bh * L.nchunk * 4);
-  L.bitmaps = off;
-  off += align256(bh * L.nwords * 4);
+  auto take = [&](size_t bytes) {
+    const size_t o = off;
+    off += bytes;
+    return o;
+  };
+  // the single-layer call's regions first
+  L.logits[0] = take(logits_b);
+  L.part_ml[0] = take(ml_b);
+  L.part_acc[0] = take(acc_b);
+  L.part_n[0] = take(n_b);
+  L.bitmaps = take(align256(bh * L.nwords * 4));
+  L.layer_total = off;
+  for (int i = 1; i < kLogitBufs; ++i) L.logits[i] = take(logits_b);
+  for (int i = 1; i < kPartBufs; ++i) {
+    L.part_ml[i] = take(ml_b);
+    L.part_acc[i] = take(acc_b);
+    L.part_n[i] = take(n_b);
+  }
   L.total = off;
   return L;
 }
@@ -130,6 +151,29 @@ bool tma_gathers_disabled() {
     return v && v[0] == '1';
   }();
   return off;
+}
+
+// Failure-path testing of the attention kernel's bounded waits, read once from
+// the environment: LYCHEE_TEST_WAIT_LIMIT_MS=<ms> shortens the limit after
+// which its pipeline waits give up (default 2 s), and
+// LYCHEE_TEST_WITHHOLD_ITEM=1 makes every CTA's builder withhold the
+// announcement of its first work item, so that the waits on that item run out:
+// the call then reports LYCHEE_ERR_TIMEOUT through lychee_check_device_error
+// and every kernel returns.  Neither is meant for use outside tests.
+uint64_t attn_wait_limit_ns() {
+  static const uint64_t ns = [] {
+    const char* v = std::getenv("LYCHEE_TEST_WAIT_LIMIT_MS");
+    const long ms = v ? std::strtol(v, nullptr, 10) : 0;
+    return ms > 0 ? (uint64_t)ms * 1000000ull : kWaitLimitNs;
+  }();
+  return ns;
+}
+bool attn_withhold_first_item() {
+  static const bool on = [] {
+    const char* v = std::getenv("LYCHEE_TEST_WITHHOLD_ITEM");
+    return v && v[0] == '1';
+  }();
+  return on;
 }
 
 // The cache [B, Hkv, N_max, d] as rows of d elements, box one row high and one
@@ -218,20 +262,84 @@ int pick_chunk(const lychee_shape* s, int sms) {
   return best;
 }
 
+// How one layer's launches are placed in a call.
+struct LayerPlan {
+  int lbuf = 0, pbuf = 0;      // logits / partial-state regions of this layer
+  bool build_bits = false;     // single layer: incoming index rows -> bitmaps first
+  bool write_bits = false;     // stack: the retrieval heads' sets go to the bitmaps
+  bool fused_combine = true;   // single layer: the combine shares the selection launch
+  const uint8_t* prev_role = nullptr;   // stack: the previous layer's roles (null: none)
+  int tail_pbuf = -1;          // stack: partial region of the previous layer, combined
+  void* tail_out = nullptr;    //   by this layer's attention CTAs into tail_out
+  WindowParams win{};          // this layer's window branch (single layer; k null: none)
+  WindowParams tail_win{};     // the previous layer's window branch (stack)
+};
+
+// The window branch of one layer: its ring caches, gate logits and roles.
+WindowParams window_of(const lychee_shape* s, const void* q, const void* k, const void* v,
+                       int window, const float* gate, const uint8_t* role) {
+  WindowParams w{};
+  if (!k) return w;
+  w.q = q;
+  w.k = k;
+  w.v = v;
+  w.gate = gate;
+  w.window = window;
+  w.Hkv = s->Hkv;
+  fill_roles(w.role, role, s->Hq);
+  return w;
+}
+
+// Host checks of a window branch's arguments (k non-null means "on").
+lychee_status check_window(const void* k, const void* v, int window, const float* gate) {
+  if (!k) return LYCHEE_OK;
+  if (!v || !gate || window < 1 || window > kMaxWindow) return LYCHEE_ERR_INVALID_ARG;
+  if (!aligned(k, 16) || !aligned(v, 16) || !aligned(gate, 4)) return LYCHEE_ERR_INVALID_ARG;
+  return LYCHEE_OK;
+}
+
+// KV groups in the order the attention kernel takes them: first the groups
+// whose sparse heads' sets are final when the kernel starts, then the groups
+// holding a sparse head whose set the previous layer's selection is still
+// writing (its head was a retrieval head there).  Returns the count of the first.
+int group_order(const uint8_t* role, const uint8_t* prev_role, int Hq, int Hkv, uint8_t* order) {
+  const int G = Hq / Hkv;
+  int n = 0;
+  auto dependent = [&](int g) {
+    if (!prev_role) return false;
+    for (int t = 0; t < G; ++t) {
+      const int h = g * G + t;
+      if (role[h] == LYCHEE_ROLE_SPARSE && prev_role[h] == LYCHEE_ROLE_RETRIEVAL) return true;
+    }
+    return false;
+  };
+  for (int g = 0; g < Hkv; ++g)
+    if (!dependent(g)) order[n++] = (uint8_t)g;
+  const int n_indep = n;
+  for (int g = 0; g < Hkv; ++g)
+    if (dependent(g)) order[n++] = (uint8_t)g;
+  return n_indep;
+}
+
 // One layer's launches.  bitmaps carry the sets of sparse heads in and (when
-// write_bits) the sets of retrieval heads out.
+// plan.write_bits) the sets of retrieval heads out.  The single-layer call
+// (build_bits, fused_combine) waits for the previous kernel before the first
+// work item; in a stack the attention kernel starts on the groups whose sets
+// are final while the previous layer's selection still runs, combines the
+// layer before in its tail, and the selection launch holds no combine.
 lychee_status run_layer(const Ctx& c, const void* q, const void* kc, const void* vc,
                         const int32_t* seqlens, const int32_t* k_per_seq, const uint8_t* role,
-                        const int32_t* idx_in, void* out, int32_t* idx_out, bool build_bits,
-                        bool write_bits) {
+                        const int32_t* idx_in, void* out, int32_t* idx_out,
+                        const LayerPlan& plan) {
   const lychee_shape* s = c.s;
   const int Hq = s->Hq, G = Hq / s->Hkv;
   uint32_t* err = &c.hdr()->err;
-  uint32_t* counter = &c.hdr()->counters[0];
-  float* logits = reinterpret_cast<float*>(c.ws + c.L.logits);
-  float* part_ml = reinterpret_cast<float*>(c.ws + c.L.part_ml);
-  float* part_acc = reinterpret_cast<float*>(c.ws + c.L.part_acc);
-  int32_t* part_n = reinterpret_cast<int32_t*>(c.ws + c.L.part_n);
+  // work / exit / tail counters of the attention launch, alternating by layer
+  uint32_t* ctr = &c.hdr()->counters[4 * (plan.lbuf & 1)];
+  float* logits = reinterpret_cast<float*>(c.ws + c.L.logits[plan.lbuf]);
+  float* part_ml = reinterpret_cast<float*>(c.ws + c.L.part_ml[plan.pbuf]);
+  float* part_acc = reinterpret_cast<float*>(c.ws + c.L.part_acc[plan.pbuf]);
+  int32_t* part_n = reinterpret_cast<int32_t*>(c.ws + c.L.part_n[plan.pbuf]);
   uint32_t* bitmaps = reinterpret_cast<uint32_t*>(c.ws + c.L.bitmaps);
   uint8_t rheads[kMaxHq], sheads[kMaxHq];
   int nr = 0, ns = 0;
@@ -240,7 +348,7 @@ lychee_status run_layer(const Ctx& c, const void* q, const void* kc, const void*
     else sheads[ns++] = (uint8_t)h;
   }
   cudaError_t e = cudaSuccess;
-  if (build_bits && ns > 0) {
+  if (plan.build_bits && ns > 0) {
     BuildBitsParams bp{};
     bp.idx_in = idx_in;
     bp.idx_out = idx_out;
@@ -264,8 +372,9 @@ lychee_status run_layer(const Ctx& c, const void* q, const void* kc, const void*
   ap.part_n = part_n;
   ap.k_per_seq = k_per_seq;
   ap.err = err;
-  ap.counter = counter;
-  ap.exits = &c.hdr()->counters[1];
+  ap.counter = ctr;
+  ap.exits = ctr + 1;
+  ap.t_counter = ctr + 2;
   ap.B = s->B; ap.Hq = Hq; ap.Hkv = s->Hkv; ap.N_max = s->N_max;
   ap.nwords = c.L.nwords; ap.nchunk = c.L.nchunk;
   ap.chunk = pick_chunk(s, c.sms);
@@ -273,21 +382,39 @@ lychee_status run_layer(const Ctx& c, const void* q, const void* kc, const void*
   ap.n_items = s->B * s->Hkv * ap.nchunk_run;
   ap.scale_log2 = (float)(1.4426950408889634 / std::sqrt((double)s->d));
   fill_roles(ap.role, role, Hq);
+  if (plan.build_bits) {
+    // every group waits: the bitmaps come from the launch just before
+    for (int g = 0; g < s->Hkv; ++g) ap.gorder[g] = (uint8_t)g;
+    ap.n_indep = 0;
+  } else {
+    ap.n_indep = group_order(role, plan.prev_role, Hq, s->Hkv, ap.gorder);
+  }
+  if (plan.tail_pbuf >= 0) {
+    ap.t_part_ml = reinterpret_cast<const float*>(c.ws + c.L.part_ml[plan.tail_pbuf]);
+    ap.t_part_acc = reinterpret_cast<const float*>(c.ws + c.L.part_acc[plan.tail_pbuf]);
+    ap.t_part_n = reinterpret_cast<const int32_t*>(c.ws + c.L.part_n[plan.tail_pbuf]);
+    ap.t_out = plan.tail_out;
+    ap.t_heads = s->B * Hq;
+    ap.t_win = plan.tail_win;
+  }
+  ap.wait_ns = attn_wait_limit_ns();
+  ap.withhold_first = attn_withhold_first_item() ? 1 : 0;
   ap.gather_tma = !tma_gathers_disabled() && encode_row_map(&ap.tmk, kc, s) &&
                    encode_row_map(&ap.tmv, vc, s) ? 1 : 0;
   e = timed(kKindAttn, c.st, [&] { return launch_attn(ap, s->dtype, s->d, G, c.sms, c.st); });
   if (e != cudaSuccess) return LYCHEE_ERR_CUDA;
-  // top-k of the retrieval heads and the combine of every head: independent
-  // (logits vs partial states), so one launch does both
+  // the retrieval heads' selection; in the single-layer call the same launch
+  // combines every head (logits vs partial states: disjoint inputs and outputs)
   TopkParams tp{};
   tp.logits = logits;
   tp.seqlens = seqlens;
   tp.k_per_seq = k_per_seq;
-  tp.bitmaps = write_bits ? bitmaps : nullptr;
+  tp.bitmaps = plan.write_bits ? bitmaps : nullptr;
   tp.idx_out = idx_out;
   tp.err = err;
   tp.B = s->B; tp.Hq = Hq; tp.N_max = s->N_max; tp.nwords = c.L.nwords; tp.k = s->k;
   tp.nheads = nr;
+  tp.sms = c.sms;
   std::memcpy(tp.heads, rheads, nr);
   CombineParams cp{};
   cp.part_ml = part_ml;
@@ -296,11 +423,13 @@ lychee_status run_layer(const Ctx& c, const void* q, const void* kc, const void*
   cp.seqlens = seqlens;
   cp.out = out;
   cp.err = err;
-  cp.B = s->B; cp.Hq = Hq; cp.N_max = s->N_max; cp.nchunk = c.L.nchunk;
+  cp.B = plan.fused_combine ? s->B : 0;   // B = 0: no combine CTAs
+  cp.Hq = Hq; cp.N_max = s->N_max; cp.nchunk = c.L.nchunk;
   cp.chunk = ap.chunk;
   cp.scale_log2 = ap.scale_log2;
+  cp.win = plan.win;
+  if (nr == 0 && !plan.fused_combine) return LYCHEE_OK;
   if (s->block > 1 && nr > 0) {
-    // block-granular selection and the combine in one launch
     BlockSelParams bp{};
     bp.logits = logits;
     bp.seqlens = seqlens;
@@ -312,15 +441,35 @@ lychee_status run_layer(const Ctx& c, const void* q, const void* kc, const void*
     bp.nheads = nr;
     bp.block = s->block;
     std::memcpy(bp.heads, rheads, nr);
-    e = timed(kKindTopkCombine, c.st,
+    e = timed(plan.fused_combine ? kKindTopkCombine : kKindTopk, c.st,
               [&] { return launch_block_select_combine(bp, cp, s->dtype, s->d, c.st); });
     if (e != cudaSuccess) return LYCHEE_ERR_CUDA;
     return LYCHEE_OK;
   }
-  e = timed(nr > 0 ? kKindTopkCombine : kKindCombine, c.st,
+  e = timed(nr == 0 ? kKindCombine : (plan.fused_combine ? kKindTopkCombine : kKindTopk), c.st,
             [&] { return launch_topk_combine(tp, cp, s->dtype, s->d, c.st); });
   if (e != cudaSuccess) return LYCHEE_ERR_CUDA;
   return LYCHEE_OK;
+}
+
+// The combine of one layer on its own launch (the stack's last layer).
+lychee_status combine_layer(const Ctx& c, int pbuf, const int32_t* seqlens, void* out,
+                            const WindowParams& win) {
+  const lychee_shape* s = c.s;
+  CombineParams cp{};
+  cp.part_ml = reinterpret_cast<const float*>(c.ws + c.L.part_ml[pbuf]);
+  cp.part_acc = reinterpret_cast<const float*>(c.ws + c.L.part_acc[pbuf]);
+  cp.part_n = reinterpret_cast<const int32_t*>(c.ws + c.L.part_n[pbuf]);
+  cp.seqlens = seqlens;
+  cp.out = out;
+  cp.err = &c.hdr()->err;
+  cp.B = s->B; cp.Hq = s->Hq; cp.N_max = s->N_max; cp.nchunk = c.L.nchunk;
+  cp.chunk = pick_chunk(s, c.sms);
+  cp.scale_log2 = (float)(1.4426950408889634 / std::sqrt((double)s->d));
+  cp.win = win;
+  const cudaError_t e =
+      timed(kKindCombine, c.st, [&] { return launch_combine(cp, s->dtype, s->d, c.st); });
+  return e == cudaSuccess ? LYCHEE_OK : LYCHEE_ERR_CUDA;
 }
 
 lychee_status export_sets(const Ctx& c, const int32_t* seqlens, int32_t* idx) {
@@ -342,23 +491,31 @@ size_t lychee_workspace_size(const lychee_shape* s) {
   return layout_of(s).total;
 }
 
+size_t lychee_layer_workspace_size(const lychee_shape* s) {
+  if (check_shape(s) != LYCHEE_OK) return 0;
+  return layout_of(s).layer_total;
+}
+
 lychee_status lychee_workspace_offsets(const lychee_shape* s, size_t* logits_off,
                                       size_t* bitmaps_off, int32_t* nwords) {
   if (check_shape(s) != LYCHEE_OK || !logits_off || !bitmaps_off || !nwords)
     return LYCHEE_ERR_INVALID_ARG;
   const Layout L = layout_of(s);
-  *logits_off = L.logits;
+  *logits_off = L.logits[0];
   *bitmaps_off = L.bitmaps;
   *nwords = L.nwords;
   return LYCHEE_OK;
 }
 
-lychee_status lychee_hybrid_decode_attn(const lychee_shape* s, const void* q,
-                                        const void* k_cache, const void* v_cache,
-                                        const int32_t* seqlens, const int32_t* k_per_seq,
-                                        const uint8_t* head_role, const int32_t* idx_in,
-                                        void* out, int32_t* idx_out, void* workspace,
-                                        size_t workspace_bytes, void* stream) {
+}  // extern "C"
+
+namespace {
+
+lychee_status layer_impl(const lychee_shape* s, const void* q, const void* k_cache,
+                         const void* v_cache, const int32_t* seqlens, const int32_t* k_per_seq,
+                         const uint8_t* head_role, const int32_t* idx_in, const void* swa_k,
+                         const void* swa_v, int32_t window, const float* gate, void* out,
+                         int32_t* idx_out, void* workspace, size_t workspace_bytes, void* stream) {
   lychee_status st = check_shape(s);
   if (st != LYCHEE_OK) return st;
   int ns = 0;
@@ -367,31 +524,41 @@ lychee_status lychee_hybrid_decode_attn(const lychee_shape* s, const void* q,
   if (ns > 0 && !idx_in) return LYCHEE_ERR_INVALID_ARG;
   if (!aligned(q, 16) || !aligned(k_cache, 16) || !aligned(v_cache, 16) || !aligned(out, 16))
     return LYCHEE_ERR_INVALID_ARG;
+  if ((st = check_window(swa_k, swa_v, window, gate)) != LYCHEE_OK) return st;
   const Layout L = layout_of(s);
-  if (!workspace || workspace_bytes < L.total || !aligned(workspace, 256))
+  if (!workspace || workspace_bytes < L.layer_total || !aligned(workspace, 256))
     return LYCHEE_ERR_WORKSPACE;
   Ctx c{s, L, static_cast<unsigned char*>(workspace), static_cast<cudaStream_t>(stream), 0};
   if ((c.sms = num_sms_current()) <= 0) return LYCHEE_ERR_CUDA;
-  if (cudaMemsetAsync(workspace, 0, L.logits, c.st) != cudaSuccess) return LYCHEE_ERR_CUDA;
+  if (cudaMemsetAsync(workspace, 0, sizeof(WsHeader), c.st) != cudaSuccess) return LYCHEE_ERR_CUDA;
+  LayerPlan plan;
+  plan.build_bits = true;
+  plan.win = window_of(s, q, swa_k, swa_v, window, gate, head_role);
   return run_layer(c, q, k_cache, v_cache, seqlens, k_per_seq, head_role, ns > 0 ? idx_in : nullptr,
-                   out, idx_out, /*build_bits=*/true, /*write_bits=*/false);
+                   out, idx_out, plan);
 }
 
-lychee_status lychee_decode_stack(const lychee_shape* s, int32_t L, const void* q,
-                                  const void* const* k_caches, const void* const* v_caches,
-                                  const int32_t* seqlens, const int32_t* k_per_seq,
-                                  const uint8_t* head_role, void* out, int32_t* idx_final,
-                                  int32_t* idx_layers, void* workspace, size_t workspace_bytes,
-                                  void* stream) {
+lychee_status stack_impl(const lychee_shape* s, int32_t L, const void* q,
+                         const void* const* k_caches, const void* const* v_caches,
+                         const int32_t* seqlens, const int32_t* k_per_seq,
+                         const uint8_t* head_role, const void* const* swa_k,
+                         const void* const* swa_v, int32_t window, const float* gate, void* out,
+                         int32_t* idx_final, int32_t* idx_layers, void* workspace,
+                         size_t workspace_bytes, void* stream) {
   lychee_status st = check_shape(s);
   if (st != LYCHEE_OK) return st;
   if (L < 1 || !q || !k_caches || !v_caches || !seqlens || !head_role || !out || !idx_final)
     return LYCHEE_ERR_INVALID_ARG;
   if (!aligned(q, 16) || !aligned(out, 16)) return LYCHEE_ERR_INVALID_ARG;
+  if (swa_k && (!swa_v || !gate)) return LYCHEE_ERR_INVALID_ARG;
   for (int l = 0; l < L; ++l) {
     if ((st = check_roles(head_role + (size_t)l * s->Hq, s->Hq, nullptr)) != LYCHEE_OK) return st;
     if (!k_caches[l] || !v_caches[l] || !aligned(k_caches[l], 16) || !aligned(v_caches[l], 16))
       return LYCHEE_ERR_INVALID_ARG;
+    if (swa_k) {
+      if (!swa_k[l] || !swa_v[l]) return LYCHEE_ERR_INVALID_ARG;
+      if ((st = check_window(swa_k[l], swa_v[l], window, gate)) != LYCHEE_OK) return st;
+    }
   }
   for (int h = 0; h < s->Hq; ++h)
     if (head_role[h] != LYCHEE_ROLE_RETRIEVAL) return LYCHEE_ERR_INVALID_ARG;
@@ -400,22 +567,89 @@ lychee_status lychee_decode_stack(const lychee_shape* s, int32_t L, const void* 
     return LYCHEE_ERR_WORKSPACE;
   Ctx c{s, lay, static_cast<unsigned char*>(workspace), static_cast<cudaStream_t>(stream), 0};
   if ((c.sms = num_sms_current()) <= 0) return LYCHEE_ERR_CUDA;
-  if (cudaMemsetAsync(workspace, 0, lay.logits, c.st) != cudaSuccess) return LYCHEE_ERR_CUDA;
+  if (cudaMemsetAsync(workspace, 0, sizeof(WsHeader), c.st) != cudaSuccess) return LYCHEE_ERR_CUDA;
   const size_t layer_elems = (size_t)s->B * s->Hq * s->d;
   const size_t esz = elem_size(s);
+  auto q_of = [&](int l) { return static_cast<const char*>(q) + (size_t)l * layer_elems * esz; };
+  auto out_of = [&](int l) { return static_cast<char*>(out) + (size_t)l * layer_elems * esz; };
+  auto win_of = [&](int l) {
+    return swa_k ? window_of(s, q_of(l), swa_k[l], swa_v[l], window,
+                             gate + (size_t)l * s->B * s->Hq, head_role + (size_t)l * s->Hq)
+                 : WindowParams{};
+  };
   for (int l = 0; l < L; ++l) {
-    const char* ql = static_cast<const char*>(q) + (size_t)l * layer_elems * esz;
-    char* ol = static_cast<char*>(out) + (size_t)l * layer_elems * esz;
-    st = run_layer(c, ql, k_caches[l], v_caches[l], seqlens, k_per_seq,
-                   head_role + (size_t)l * s->Hq, nullptr, ol, nullptr, /*build_bits=*/false,
-                   /*write_bits=*/true);
+    LayerPlan plan;
+    plan.lbuf = l % kLogitBufs;
+    plan.pbuf = l % kPartBufs;
+    plan.write_bits = true;
+    plan.fused_combine = false;
+    if (l > 0) {
+      plan.prev_role = head_role + (size_t)(l - 1) * s->Hq;
+      plan.tail_pbuf = (l - 1) % kPartBufs;
+      plan.tail_out = out_of(l - 1);
+      plan.tail_win = win_of(l - 1);
+    }
+    st = run_layer(c, q_of(l), k_caches[l], v_caches[l], seqlens, k_per_seq,
+                   head_role + (size_t)l * s->Hq, nullptr, nullptr, nullptr, plan);
     if (st != LYCHEE_OK) return st;
     if (idx_layers) {
       st = export_sets(c, seqlens, idx_layers + (size_t)l * s->B * s->Hq * s->k);
       if (st != LYCHEE_OK) return st;
     }
   }
+  // the last layer's output (every other layer was combined by the next one)
+  st = combine_layer(c, (L - 1) % kPartBufs, seqlens, out_of(L - 1), win_of(L - 1));
+  if (st != LYCHEE_OK) return st;
   return export_sets(c, seqlens, idx_final);
+}
+
+}  // namespace
+
+extern "C" {
+
+lychee_status lychee_hybrid_decode_attn(const lychee_shape* s, const void* q,
+                                        const void* k_cache, const void* v_cache,
+                                        const int32_t* seqlens, const int32_t* k_per_seq,
+                                        const uint8_t* head_role, const int32_t* idx_in,
+                                        void* out, int32_t* idx_out, void* workspace,
+                                        size_t workspace_bytes, void* stream) {
+  return layer_impl(s, q, k_cache, v_cache, seqlens, k_per_seq, head_role, idx_in, nullptr,
+                    nullptr, 0, nullptr, out, idx_out, workspace, workspace_bytes, stream);
+}
+
+lychee_status lychee_hybrid_decode_attn_swa(const lychee_shape* s, const void* q,
+                                            const void* k_cache, const void* v_cache,
+                                            const int32_t* seqlens, const int32_t* k_per_seq,
+                                            const uint8_t* head_role, const int32_t* idx_in,
+                                            const void* swa_k, const void* swa_v, int32_t window,
+                                            const float* gate, void* out, int32_t* idx_out,
+                                            void* workspace, size_t workspace_bytes,
+                                            void* stream) {
+  if (!swa_k) return LYCHEE_ERR_INVALID_ARG;
+  return layer_impl(s, q, k_cache, v_cache, seqlens, k_per_seq, head_role, idx_in, swa_k, swa_v,
+                    window, gate, out, idx_out, workspace, workspace_bytes, stream);
+}
+
+lychee_status lychee_decode_stack(const lychee_shape* s, int32_t L, const void* q,
+                                  const void* const* k_caches, const void* const* v_caches,
+                                  const int32_t* seqlens, const int32_t* k_per_seq,
+                                  const uint8_t* head_role, void* out, int32_t* idx_final,
+                                  int32_t* idx_layers, void* workspace, size_t workspace_bytes,
+                                  void* stream) {
+  return stack_impl(s, L, q, k_caches, v_caches, seqlens, k_per_seq, head_role, nullptr, nullptr,
+                    0, nullptr, out, idx_final, idx_layers, workspace, workspace_bytes, stream);
+}
+
+lychee_status lychee_decode_stack_swa(const lychee_shape* s, int32_t L, const void* q,
+                                      const void* const* k_caches, const void* const* v_caches,
+                                      const int32_t* seqlens, const int32_t* k_per_seq,
+                                      const uint8_t* head_role, const void* const* swa_k,
+                                      const void* const* swa_v, int32_t window, const float* gate,
+                                      void* out, int32_t* idx_final, int32_t* idx_layers,
+                                      void* workspace, size_t workspace_bytes, void* stream) {
+  if (!swa_k) return LYCHEE_ERR_INVALID_ARG;
+  return stack_impl(s, L, q, k_caches, v_caches, seqlens, k_per_seq, head_role, swa_k, swa_v,
+                    window, gate, out, idx_final, idx_layers, workspace, workspace_bytes, stream);
 }
 
 lychee_status lychee_append_kv(const lychee_shape* s, const void* k_new, const void* v_new,
@@ -437,6 +671,33 @@ lychee_status lychee_append_kv(const lychee_shape* s, const void* k_new, const v
   p.row_bytes = s->d * (int)elem_size(s);
   return launch_append_kv(p, static_cast<cudaStream_t>(stream)) == cudaSuccess ? LYCHEE_OK
                                                                                : LYCHEE_ERR_CUDA;
+}
+
+lychee_status lychee_hardkuma_roles(const double* alpha, const double* beta, int32_t L,
+                                    int32_t Hq, double p, double q, int32_t layer0_retrieval,
+                                    uint8_t* head_role, double* expected_z, double* expected_l0,
+                                    void* stream) {
+  if (!alpha || !beta || !head_role || L < 1 || Hq < 1) return LYCHEE_ERR_INVALID_ARG;
+  if ((long long)L * Hq >= (1LL << 31)) return LYCHEE_ERR_UNSUPPORTED;
+  if (!(p < 0.0) || !(q > 1.0) || !std::isfinite(p) || !std::isfinite(q))
+    return LYCHEE_ERR_INVALID_ARG;
+  if (!aligned(alpha, 8) || !aligned(beta, 8) || !aligned(expected_z, 8) ||
+      !aligned(expected_l0, 8))
+    return LYCHEE_ERR_INVALID_ARG;
+  RolesParams rp{};
+  rp.alpha = alpha;
+  rp.beta = beta;
+  rp.role = head_role;
+  rp.expected_z = expected_z;
+  rp.expected_l0 = expected_l0;
+  rp.p = p;
+  rp.q = q;
+  rp.L = L;
+  rp.Hq = Hq;
+  rp.layer0_retrieval = layer0_retrieval ? 1 : 0;
+  return launch_hardkuma_roles(rp, static_cast<cudaStream_t>(stream)) == cudaSuccess
+             ? LYCHEE_OK
+             : LYCHEE_ERR_CUDA;
 }
 
 lychee_status lychee_check_device_error(void* workspace, void* stream, uint32_t* detail) {

@@ -54,6 +54,7 @@
 // written to the workspace for the top-k kernel.
 #include <type_traits>
 
+#include "combine_body.cuh"
 #include "common.cuh"
 #include "kernels.h"
 
@@ -201,15 +202,26 @@ struct AttnCfg {
   static constexpr int SMEM = OFF_BAR + NBAR * 8 + 128;   // + alignment slack
 };
 
-// Item decode shared by the builder: item -> (b, c, g).  With a compact item
-// space (B <= kMaxBatchCompact) items enumerate only chunks below n_b, chunk
-// major over the concatenated sequences, KV group fastest; cum[b] holds the
-// number of chunks of sequences before b.  Otherwise every (b, c < nchunk, g)
-// is an item and chunks beyond n_b are skipped.
+// Item decode shared by the builder: item -> (b, c, g).  Items come in two
+// classes: first those of the groups gorder[0 .. n_indep), then those of the
+// other groups; within a class chunk by chunk, group fastest.  With a compact
+// item space (B <= kMaxBatchCompact) the chunks are only those below n_b,
+// chunk major over the concatenated sequences; cum[b] holds the number of
+// chunks of sequences before b.  Otherwise every (b, c < nchunk) is a chunk and
+// those beyond n_b are skipped.
 __device__ __forceinline__ void decode_item(int item, bool compact, const int* cum, int B,
-                                            int Hkv, int nchunk, int& b, int& c, int& g) {
-  g = item % Hkv;
-  const int cg = item / Hkv;
+                                            int Hkv, int nchunk, int n_indep, int ncg,
+                                            const uint8_t* gorder, int& b, int& c, int& g) {
+  int gi, cg;
+  if (item < ncg * n_indep) {
+    gi = item % n_indep;
+    cg = item / n_indep;
+  } else {
+    const int r = item - ncg * n_indep, nd = Hkv - n_indep;
+    gi = n_indep + r % nd;
+    cg = r / nd;
+  }
+  g = gorder[gi];
   if (compact) {
     int lo = 0, hi = B;  // largest b with cum[b] <= cg
     while (hi - lo > 1) {
@@ -285,6 +297,95 @@ template <typename T, int D, int G, int NW, int NP, int TT, int STAGES>
 __device__ __forceinline__ void consumer_loop_mma(const AttnParams& p, unsigned char* smem,
                                                   uint64_t* full, uint64_t* empty, uint64_t* freeb);
 
+// The tail of a stack layer's attention kernel: the combine of the previous
+// layer (its partial states are complete once the previous kernel of the stream
+// has), with its sparse heads' window branch when it has one (combine_body.cuh),
+// run by every CTA that has no attention item left.  Work items are whole
+// (sequence, head) pairs taken from a counter.  Each of the CTA's NSL slots (a
+// warp, or half a warp for d = 64) merges the states of every NSL-th chunk,
+// eight states in flight, into running sums (combine_body.cuh: absorb); the
+// slots are then merged in a fixed order and the head's output is written.  The
+// order of the merges does not depend on scheduling.
+template <typename T, int D, int NT>
+__device__ __forceinline__ void tail_combine(const AttnParams& p, unsigned char* smem) {
+  constexpr int LPR = D / 4;             // lanes per state row
+  constexpr int SPW = 32 / LPR;          // state rows per warp
+  constexpr int NSL = (NT / 32) * SPW;   // slots
+  constexpr int RS = D + 4;              // slot row in shared memory: acc[D], m, l
+  static_assert(NT >= D, "one thread per output element");
+  float* red = reinterpret_cast<float*>(smem);
+  int* s_item = reinterpret_cast<int*>(smem + NSL * RS * 4);
+  float* wsm = reinterpret_cast<float*>(smem + NSL * RS * 4 + 16);   // window branch scratch
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int slot = warp * SPW + lane / LPR, col = (lane % LPR) * 4;
+  const float sl = p.scale_log2;
+  for (;;) {
+    if (threadIdx.x == 0) *s_item = (int)atomicAdd(p.t_counter, 1u);
+    __syncthreads();
+    const int bh = *s_item;
+    if (bh >= p.t_heads) break;
+    const int b = bh / p.Hq;
+    const int n = min(max(__ldg(&p.seqlens[b]), 1), p.N_max);
+    const int nc = (n + p.chunk - 1) / p.chunk;
+    const int32_t* pn = p.t_part_n + (size_t)bh * p.nchunk;
+    const float2* ml = reinterpret_cast<const float2*>(p.t_part_ml) + (size_t)bh * p.nchunk * kPartSlots;
+    const float* pa = p.t_part_acc + (size_t)bh * p.nchunk * kPartSlots * D;
+    float m = -INFINITY, l = 0.f;
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+    // chunks slot, slot + NSL, ...: two at a time, four states of each in flight
+    for (int ca = slot; ca < nc; ca += 2 * NSL) {
+      const int cb = ca + NSL;
+      const int na = min(max(__ldcg(pn + ca), 0), kPartSlots);
+      const int nb = cb < nc ? min(max(__ldcg(pn + cb), 0), kPartSlots) : 0;
+      for (int s0 = 0; s0 < max(na, nb); s0 += 4) {
+        float2 e[8];
+        float4 a[8];
+#pragma unroll
+        for (int q = 0; q < 8; ++q) {
+          const int c = q < 4 ? ca : cb, st = s0 + (q & 3);
+          e[q] = make_float2(-INFINITY, 0.f);
+          a[q] = make_float4(0.f, 0.f, 0.f, 0.f);
+          if (st < (q < 4 ? na : nb)) {
+            const size_t si = (size_t)c * kPartSlots + st;
+            e[q] = __ldcg(ml + si);
+            a[q] = __ldcg(reinterpret_cast<const float4*>(pa + si * D + col));
+          }
+        }
+#pragma unroll
+        for (int q = 0; q < 8; ++q) absorb(e[q], a[q], sl, m, l, acc);
+      }
+    }
+    float* row = red + slot * RS;
+    *reinterpret_cast<float4*>(row + col) = acc;
+    if (col == 0) {
+      row[D] = m;
+      row[D + 1] = l;
+    }
+    __syncthreads();
+    // a sparse head's window branch (every thread; fused below)
+    const bool win = window_on(p.t_win, bh % p.Hq);
+    float ow = 0.f;
+    if (win) ow = window_out<T, D>(p.t_win, bh, p.Hq, n, sl, wsm);
+    if (threadIdx.x < D) {
+      float M = -INFINITY;
+      for (int s2 = 0; s2 < NSL; ++s2) M = fmaxf(M, red[s2 * RS + D]);
+      float A = 0.f, Lsum = 0.f;
+      if (M != -INFINITY) {
+        for (int s2 = 0; s2 < NSL; ++s2) {
+          const float ms = red[s2 * RS + D];
+          const float w = ms == -INFINITY ? 0.f : fast_exp2((ms - M) * sl);
+          A = fmaf(w, red[s2 * RS + threadIdx.x], A);
+          Lsum = fmaf(w, red[s2 * RS + D + 1], Lsum);
+        }
+      }
+      float o = Lsum > 0.f ? A / Lsum : 0.f;
+      if (win) o = gate_fuse(o, ow, p.t_win.gate[bh]);
+      store_out<T>(reinterpret_cast<T*>(p.t_out) + (size_t)bh * D + threadIdx.x, o);
+    }
+    __syncthreads();   // the slot rows and the item slot are rewritten next
+  }
+}
+
 template <typename T, int D, int G, int NW, int NP, int TT, int STAGES>
 __global__ void __launch_bounds__((NW + NP) * 32, 1)
     attn_kernel(const __grid_constant__ AttnParams p) {
@@ -306,8 +407,12 @@ __global__ void __launch_bounds__((NW + NP) * 32, 1)
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int Hq = p.Hq, Hkv = p.Hkv, N_max = p.N_max, B = p.B;
   const bool compact = B <= kMaxBatchCompact;
-  pdl_launch_dependents();
-  pdl_wait();
+  // Programmatic dependent launch: no warp waits for the previous kernel of the
+  // stream at the start.  The builder alone waits for it, before it reads the
+  // first set that kernel may still be writing (the groups past n_indep) and at
+  // the latest once it has claimed its last item; only then does it let the
+  // next kernel launch.  So when every CTA has let the next kernel go, the
+  // previous kernel has completed, and the layer before it too.
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
       mbar_init(&full[s], NS);
@@ -349,22 +454,46 @@ __global__ void __launch_bounds__((NW + NP) * 32, 1)
   }
   if (warp == NW + 1) {
     // ------------------------------------------------------------ builder
-    const int n_items = compact ? cum[B] * Hkv : p.n_items;
+    const int ncg = compact ? cum[B] : B * p.nchunk_run;   // (sequence, chunk) pairs
+    const int n_items = ncg * Hkv;
+    const int first_dep = ncg * p.n_indep;                   // first item of a waiting group
+    bool waited = false, released = false;                   // warp-uniform
+    auto wait_prev = [&]() {
+      if (!waited) {
+        pdl_wait();
+        waited = true;
+      }
+    };
     // claim an item (lane 0) and load what building its row list needs
     auto claim = [&]() -> int { return lane == 0 ? (int)atomicAdd(p.counter, 1u) : 0; };
     auto prefetch = [&](int item, int& nraw, uint32_t (&w)[G]) {
       nraw = 1;
 #pragma unroll
       for (int t = 0; t < G; ++t) w[t] = 0u;
-      if (item >= n_items) return;
+      if (item >= n_items) {
+        // this CTA takes no further item
+        wait_prev();
+        if (!released) {
+          pdl_launch_dependents();
+          released = true;
+        }
+        return;
+      }
+      if (item >= first_dep) wait_prev();
       int b, c, g;
-      decode_item(item, compact, cum, B, Hkv, p.nchunk_run, b, c, g);
+      decode_item(item, compact, cum, B, Hkv, p.nchunk_run, p.n_indep, ncg, p.gorder, b, c, g);
       nraw = __ldg(&p.seqlens[b]);
       const int word = c * (p.chunk / 32) + lane;
       if (lane < p.chunk / 32 && word < p.nwords) {
+        // sparse heads' words only (a retrieval head reads every row), through
+        // L2: in a stack the previous kernel may have rewritten these rows
+        // while this kernel ran
         const size_t wbase = (size_t)(b * Hq + g * G) * p.nwords + word;
 #pragma unroll
-        for (int t = 0; t < G; ++t) w[t] = __ldg(&p.bitmaps[wbase + (size_t)t * p.nwords]);
+        for (int t = 0; t < G; ++t) {
+          const int h = g * G + t;
+          if (!((p.role[h >> 5] >> (h & 31)) & 1u)) w[t] = __ldcg(&p.bitmaps[wbase + (size_t)t * p.nwords]);
+        }
       }
     };
     if (blockIdx.x == 0) {
@@ -380,7 +509,7 @@ __global__ void __launch_bounds__((NW + NP) * 32, 1)
     int claimed = claim();
     for (uint32_t it = 0;; ++it) {
       const int buf = it & 1;
-      if (!mbar_wait(&freeb[buf], ((it >> 1) & 1u) ^ 1u, p.err)) break;
+      if (!mbar_wait(&freeb[buf], ((it >> 1) & 1u) ^ 1u, p.err, p.wait_ns)) break;
       unsigned char* ib = smem + C::OFF_ITEM + buf * C::IBUF;
       int* desc = reinterpret_cast<int*>(ib);
       uint8_t* asg = ib + C::IB_ASG;
@@ -392,7 +521,7 @@ __global__ void __launch_bounds__((NW + NP) * 32, 1)
           total = -1;
           break;
         }
-        decode_item(cur, compact, cum, B, Hkv, p.nchunk_run, b, c, g);
+        decode_item(cur, compact, cum, B, Hkv, p.nchunk_run, p.n_indep, ncg, p.gorder, b, c, g);
         const int n = min(max(cur_n, 1), N_max);
         p0 = c * p.chunk;
         const int h0 = g * G;
@@ -514,9 +643,13 @@ __global__ void __launch_bounds__((NW + NP) * 32, 1)
         desc[5] = (int)rmask;
       }
       __syncwarp();
-      if (lane == 0) mbar_arrive(&ready[buf]);
+      // (test only: with p.withhold_first the first item is never announced,
+      // so every wait that depends on it runs out after p.wait_ns)
+      if (lane == 0 && !(p.withhold_first && it == 0)) mbar_arrive(&ready[buf]);
       if (total < 0) break;
     }
+    wait_prev();   // (a wait that gave up leaves the loop early)
+    if (!released) pdl_launch_dependents();
   } else if (warp >= NW) {
     // ------------------------------------------------------ streaming warps
     const int sw = warp == NW ? 0 : warp - NW - 1;   // 0: publishes tiles, bulk copies
@@ -526,7 +659,7 @@ __global__ void __launch_bounds__((NW + NP) * 32, 1)
     bool ok = true;
     for (uint32_t it = 0;; ++it) {
       const int buf = it & 1;
-      if (!mbar_wait(&ready[buf], (it >> 1) & 1u, p.err)) break;
+      if (!mbar_wait(&ready[buf], (it >> 1) & 1u, p.err, p.wait_ns)) break;
       const unsigned char* ib = smem + C::OFF_ITEM + buf * C::IBUF;
       const int* desc = reinterpret_cast<const int*>(ib);
       const int32_t* lpos = reinterpret_cast<const int32_t*>(ib + C::IB_LPOS);
@@ -542,7 +675,7 @@ __global__ void __launch_bounds__((NW + NP) * 32, 1)
       const int ntile = total <= 0 ? 1 : (total + TT - 1) / TT;
       for (int tt = 0; tt < ntile; ++tt) {
         const int t0 = tt * TT;
-        if (!mbar_wait(&empty[s], ph ^ 1u, p.err)) {
+        if (!mbar_wait(&empty[s], ph ^ 1u, p.err, p.wait_ns)) {
           ok = false;
           break;
         }
@@ -646,12 +779,25 @@ __global__ void __launch_bounds__((NW + NP) * 32, 1)
     if constexpr (C::MMA) consumer_loop_mma<T, D, G, NW, NP, TT, STAGES>(p, smem, full, empty, freeb);
     else consumer_loop<T, D, G, NW, NP, TT, STAGES>(p, smem, full, empty, freeb);
   }
-  // ---- the last CTA to leave resets the launch counters for the next launch
   __syncthreads();
+  if (p.t_heads > 0) {
+    if constexpr (!C::MMA && ILP > 1 && LYCHEE_ATTN_REGSPLIT) {
+      // back to the launch's registers per thread in every warp
+      if (warp >= NW) asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(128));
+      else asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(128));
+    }
+    pdl_wait();   // the previous layer's partial states are complete
+    static_assert((C::NT / 32) * (32 / (D / 4)) * (D + 4) * 4 + 16 + window_smem_floats<D>() * 4 <=
+                      C::OFF_INFO,
+                  "the tail's shared memory fits the (drained) ring");
+    tail_combine<T, D, C::NT>(p, smem);
+  }
+  // ---- the last CTA to leave resets the launch counters for the next launch
   if (threadIdx.x == 0) {
     __threadfence();
     if (atomicAdd(p.exits, 1u) == gridDim.x - 1) {
       *p.counter = 0u;
+      *p.t_counter = 0u;
       *p.exits = 0u;
       __threadfence();
     }
@@ -695,7 +841,7 @@ __device__ __forceinline__ void consumer_loop(const AttnParams& p, unsigned char
 
   uint32_t s = 0, ph = 0;
   for (;;) {
-    if (!mbar_wait(&full[s], ph, p.err)) break;
+    if (!mbar_wait(&full[s], ph, p.err, p.wait_ns)) break;
     const int4 i0 = info[2 * s], i1 = info[2 * s + 1];
     const int flags = i1.x;
     if (flags & kTerm) break;
@@ -968,7 +1114,7 @@ __device__ __forceinline__ void consumer_loop_mma(const AttnParams& p, unsigned 
 
   uint32_t s = 0, ph = 0;
   for (;;) {
-    if (!mbar_wait(&full[s], ph, p.err)) break;
+    if (!mbar_wait(&full[s], ph, p.err, p.wait_ns)) break;
     const int4 i0 = info[2 * s], i1 = info[2 * s + 1];
     const int flags = i1.x;
     if (flags & kTerm) break;
@@ -1151,8 +1297,8 @@ template <typename T, int D, int G, int NW, int NP, int TT, int STAGES>
 cudaError_t launch_attn_t(const AttnParams& p, int num_sms, cudaStream_t st) {
   using C = AttnCfg<T, D, G, NW, NP, TT, STAGES>;
   auto kfn = attn_kernel<T, D, G, NW, NP, TT, STAGES>;
-  static bool attr_set = false;  // per instantiation; set once per process
-  if (!attr_set) {
+  static PerDeviceOnce attrs;   // per instantiation and device
+  const cudaError_t ea = attrs.run([&]() -> cudaError_t {
     cudaError_t e =
         cudaFuncSetAttribute(kfn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)C::SMEM);
     if (e != cudaSuccess) return e;
@@ -1163,8 +1309,9 @@ cudaError_t launch_attn_t(const AttnParams& p, int num_sms, cudaStream_t st) {
       if (e != cudaSuccess) return e;
       if (fa.numRegs != 128) return cudaErrorInvalidConfiguration;
     }
-    attr_set = true;
-  }
+    return cudaSuccess;
+  });
+  if (ea != cudaSuccess) return ea;
   const int grid = max(1, min(num_sms, p.n_items));
   const cudaError_t e = launch_pdl(kfn, dim3(grid), dim3(C::NT), (size_t)C::SMEM, st, p);
   if (e != cudaSuccess) return e;

@@ -245,13 +245,12 @@ __global__ void __launch_bounds__(kSelThreads, D >= 128 ? 2 : 1)
 template <typename T, int D>
 cudaError_t launch_bsc(const BlockSelParams& p, const CombineParams& cp, cudaStream_t st) {
   auto kfn = block_select_combine_kernel<T, D>;
-  static bool attr = false;
-  if (!attr) {
-    const cudaError_t e = cudaFuncSetAttribute(kfn, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                               (int)kBlockSelSmemMax);
-    if (e != cudaSuccess) return e;
-    attr = true;
-  }
+  static PerDeviceOnce attrs;   // per instantiation and device
+  const cudaError_t ea = attrs.run([&] {
+    return cudaFuncSetAttribute(kfn, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                (int)kBlockSelSmemMax);
+  });
+  if (ea != cudaSuccess) return ea;
   const int nsel = p.B * p.nheads * kSelCtas;
   const int ncomb = cp.B * cp.Hq * kCombineSplit;
   size_t smem = block_select_smem(p.N_max, p.block);

@@ -25,6 +25,124 @@ __device__ __forceinline__ void store_out<float>(float* p, float v) {
 
 constexpr int kBatch = 5;
 
+// ---- the sliding-window branch of a sparse head -------------------------------------
+// Page "HySparse: A Hybrid Sparse Attention Architecture with Oracle Token
+// Selection and KV Cache Sharing" (paperlayer.ai/abs/2602.03560v1),
+// Methodology: a sparse layer fuses its sparse branch with a local
+// sliding-window branch (window 128, its own cache) through sigmoid gating.
+// Here the window branch of sparse head h attends to the min(window, n_b) rows
+// in use of its KV group's window ring (position j lives in row j % window; the
+// order of the rows does not matter to softmax), and the head's output is
+// s * O_sparse + (1 - s) * O_window with s = sigmoid(gate logit).
+
+// Shared memory of window_out, in floats: q, the row scores, two reduction slots.
+template <int D>
+constexpr int window_smem_floats() {
+  return D + kMaxWindow + 32;
+}
+
+template <typename T>
+__device__ __forceinline__ float elem_to_float(const T* p, int i);
+template <>
+__device__ __forceinline__ float elem_to_float<__nv_bfloat16>(const __nv_bfloat16* p, int i) {
+  return __bfloat162float(p[i]);
+}
+template <>
+__device__ __forceinline__ float elem_to_float<float>(const float* p, int i) {
+  return p[i];
+}
+
+// Dot product of the fp32 vector sq[0 .. D) with row r (16-byte loads).
+template <typename T, int D>
+__device__ __forceinline__ float dot_row(const float* sq, const T* r) {
+  const uint4* v = reinterpret_cast<const uint4*>(r);
+  float acc = 0.f;
+  if constexpr (sizeof(T) == 2) {
+#pragma unroll 4
+    for (int c = 0; c < D / 8; ++c) {
+      const uint4 w = __ldg(v + c);
+      const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const float2 f = bf16x2_to_float2(ws[e]);
+        acc = fmaf(sq[8 * c + 2 * e], f.x, acc);
+        acc = fmaf(sq[8 * c + 2 * e + 1], f.y, acc);
+      }
+    }
+  } else {
+#pragma unroll 4
+    for (int c = 0; c < D / 4; ++c) {
+      const uint4 w = __ldg(v + c);
+      acc = fmaf(sq[4 * c], __uint_as_float(w.x), acc);
+      acc = fmaf(sq[4 * c + 1], __uint_as_float(w.y), acc);
+      acc = fmaf(sq[4 * c + 2], __uint_as_float(w.z), acc);
+      acc = fmaf(sq[4 * c + 3], __uint_as_float(w.w), acc);
+    }
+  }
+  return acc;
+}
+
+// Whether head h of a layer gets the window branch.
+__device__ __forceinline__ bool window_on(const WindowParams& w, int h) {
+  return w.k != nullptr && !((w.role[h >> 5] >> (h & 31)) & 1u);
+}
+
+// The window branch's output element threadIdx.x (< D) of head bh = b * Hq + h
+// with n_b = n, computed by every thread of the CTA (a call the whole CTA makes
+// together); sm: window_smem_floats<D>() floats of shared memory.  Scores are
+// fp32 sums of exact products, the softmax and the weighted sum fp32, in a
+// fixed order.
+template <typename T, int D>
+__device__ __forceinline__ float window_out(const WindowParams& w, int bh, int Hq, int n,
+                                            float sl, float* sm) {
+  float* sq = sm;
+  float* ss = sm + D;
+  float* red = ss + kMaxWindow;
+  const int b = bh / Hq, h = bh % Hq, g = h / (Hq / w.Hkv);
+  const T* qr = reinterpret_cast<const T*>(w.q) + (size_t)bh * D;
+  const size_t ring = ((size_t)b * w.Hkv + g) * (size_t)w.window * D;
+  const T* K = reinterpret_cast<const T*>(w.k) + ring;
+  const T* V = reinterpret_cast<const T*>(w.v) + ring;
+  const int rows = min(min(w.window, n), kMaxWindow);
+  const int tid = threadIdx.x, lane = tid & 31;
+  for (int i = tid; i < D; i += blockDim.x) sq[i] = elem_to_float<T>(qr, i);
+  __syncthreads();
+  for (int r = tid; r < rows; r += blockDim.x) ss[r] = dot_row<T, D>(sq, K + (size_t)r * D);
+  __syncthreads();
+  if (tid < 32) {
+    float m = -INFINITY;
+    for (int r = lane; r < rows; r += 32) m = fmaxf(m, ss[r]);
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+    if (lane == 0) red[0] = m;
+  }
+  __syncthreads();
+  const float m = red[0];
+  for (int r = tid; r < rows; r += blockDim.x) ss[r] = fast_exp2((ss[r] - m) * sl);
+  __syncthreads();
+  if (tid < 32) {
+    float l = 0.f;
+    for (int r = lane; r < rows; r += 32) l += ss[r];
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) l += __shfl_xor_sync(0xffffffffu, l, o);
+    if (lane == 0) red[1] = l;
+  }
+  __syncthreads();
+  float o = 0.f;
+  if (tid < D) {
+    for (int r = 0; r < rows; ++r) o = fmaf(ss[r], elem_to_float<T>(V + (size_t)r * D, tid), o);
+    o /= red[1];
+  }
+  __syncthreads();   // sm is reused by the caller
+  return o;
+}
+
+// s * o_sparse + (1 - s) * o_window with s = sigmoid(g).
+__device__ __forceinline__ float gate_fuse(float o_sparse, float o_window, float g) {
+  const float s = 1.f / (1.f + expf(-g));
+  return s * o_sparse + (1.f - s) * o_window;
+}
+
 // Merge one state (e = (m, l), a = four elements of acc) into running sums.
 __device__ __forceinline__ void absorb(float2 e, float4 a, float sl, float& m, float& l,
                                        float4& acc) {
@@ -54,6 +172,7 @@ constexpr int kCombineSplit = 8;   // combine CTAs per (sequence, head): one gro
 //   recv  [kCombineSplit][D + 4] floats: the head's CTA states (leader CTA only)
 //   red   [NS][D + 4] floats: this CTA's slot states, then its own state
 //   slist [kCombThreads * kPartSlots] u16: the states of a block of chunks, in order
+//         (then, in the leader, the window branch's scratch)
 //   wsum  [kCombWarps + 1] ints
 template <int D>
 struct CombineSmem {
@@ -65,6 +184,8 @@ struct CombineSmem {
   static constexpr size_t kWsum = kSlist + (size_t)kCombThreads * kPartSlots * 2;
   static constexpr size_t kBytes = kWsum + (kCombWarps + 1) * 4;
   static_assert(kRed % 16 == 0 && kSlist % 16 == 0 && (RS * 4) % 16 == 0, "16-byte rows");
+  static_assert((size_t)kCombThreads * kPartSlots * 2 >= (size_t)window_smem_floats<D>() * 4,
+                "the window branch's scratch fits the state list");
 };
 template <int D>
 constexpr size_t combine_smem_bytes() {
@@ -199,6 +320,11 @@ __device__ __forceinline__ void combine_body(const CombineParams& p, int cta, un
   }
   __syncthreads();
   cluster_wait();   // every leader's barrier is set up
+  // the head's window branch (leader only; while the other states travel)
+  const int hh = bh % p.Hq;
+  const bool win = sp == 0 && window_on(p.win, hh);
+  float ow = 0.f;
+  if (win) ow = window_out<T, D>(p.win, bh, p.Hq, n, sl, reinterpret_cast<float*>(slist));
   const uint32_t leader = cluster_ctarank() - (uint32_t)sp;
   if (sp != 0) {
     // send the state to row sp of the leader's receive rows
@@ -228,7 +354,9 @@ __device__ __forceinline__ void combine_body(const CombineParams& p, int cta, un
         Lsum = fmaf(w, recv[k * RS + D + 1], Lsum);
       }
     }
-    store_out<T>(reinterpret_cast<T*>(p.out) + (size_t)bh * D + tid, Lsum > 0.f ? A / Lsum : 0.f);
+    float o = Lsum > 0.f ? A / Lsum : 0.f;
+    if (win) o = gate_fuse(o, ow, p.win.gate[bh]);
+    store_out<T>(reinterpret_cast<T*>(p.out) + (size_t)bh * D + tid, o);
   }
   cluster_wait();   // no CTA leaves while a state may still be on its way to it
 }

@@ -11,6 +11,8 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <atomic>
+
 namespace lychee {
 
 // ---- device error word (workspace header) ---------------------------------
@@ -33,6 +35,7 @@ constexpr int kChunk = 960;           // positions per attention work item, at m
 constexpr int kChunkMin = 768;        // ... and at least (the host picks one per launch)
 constexpr int kPartSlots = 12;        // partial states per (sequence, head, chunk): one per warp
 constexpr int kMaxHq = 128;           // query heads supported
+constexpr int kMaxWindow = 1024;      // rows of a sparse head's sliding-window ring, at most
 constexpr uint64_t kWaitLimitNs = 2000000000ull;   // 2 s: a wait this long is a fault
 
 __device__ __forceinline__ uint64_t globaltimer() {
@@ -88,12 +91,13 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity,
 }
 
 // Wait for the phase with the given parity to complete.  Gives up after
-// kWaitLimitNs, sets kErrTimeout and returns false; the caller then leaves.
-__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, uint32_t* err) {
+// limit_ns, sets kErrTimeout and returns false; the caller then leaves.
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, uint32_t* err,
+                                          uint64_t limit_ns = kWaitLimitNs) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = globaltimer();
   while (!mbar_try_wait(bar, parity)) {
-    if (globaltimer() - t0 > kWaitLimitNs) {
+    if (globaltimer() - t0 > limit_ns) {
       flag_error(err, kErrTimeout);
       return false;
     }
@@ -225,6 +229,31 @@ __device__ __forceinline__ uint32_t float_to_key(float f) {
 __device__ __forceinline__ float2 bf16x2_to_float2(uint32_t w) {
   return make_float2(__uint_as_float(w << 16), __uint_as_float(w & 0xffff0000u));
 }
+
+// ---- per-device one-time host work ----------------------------------------------
+// Kernel attributes (dynamic shared memory, cluster sizes) are per device.  A
+// PerDeviceOnce remembers, per device ordinal below 64, that its work succeeded
+// on that device; callers from several host threads may both run it the first
+// time (the work is idempotent), never neither.  Devices 64 and up repeat the
+// work on every call.
+class PerDeviceOnce {
+ public:
+  template <typename F>
+  cudaError_t run(F&& work) {
+    int dev = 0;
+    const cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (dev < 0 || dev >= 64) return work();
+    const uint64_t bit = 1ull << dev;
+    if (done_.load(std::memory_order_acquire) & bit) return cudaSuccess;
+    const cudaError_t w = work();
+    if (w == cudaSuccess) done_.fetch_or(bit, std::memory_order_acq_rel);
+    return w;
+  }
+
+ private:
+  std::atomic<uint64_t> done_{0};
+};
 
 // Launch with programmatic stream serialization (see pdl_wait above).
 template <typename... KArgs, typename... Args>

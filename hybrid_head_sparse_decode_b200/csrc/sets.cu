@@ -20,19 +20,23 @@ constexpr int kEntriesPerCta = 4 * kThreads;   // set entries one build_bits CTA
 // writer, so the row needs no clearing pass and no atomics: the thread holding
 // the first entry of a word ORs that word's entries (at most 32, contiguous in
 // the ascending row) and also writes the empty words between the previous
-// entry's word and its own; the first and last entries cover the words before
-// and after the set.  A set ends at its first -1 (at most k_b entries are
-// read); that entry clears the words after the last member.  An entry outside
-// [0, n_b), not strictly above its predecessor, or after the end of the set
-// sets kErrBadIndex; the row is then not a set and its bitmap is unspecified,
-// but every store still stays inside the row.
+// entry's word and its own.  A set ends at its first -1 (or at the row's k-th
+// entry; the budget k_b does not bound what a sparse head reads).  The empty
+// words before the first member and after the last one can be thousands; the
+// CTA holding that entry clears them together after its entries.  An entry
+// outside [0, n_b), not strictly above its predecessor, or after the end of the
+// set sets kErrBadIndex; the row is then not a set and its bitmap is
+// unspecified, but every store still stays inside the row.
 __global__ void __launch_bounds__(kThreads) build_bits_kernel(const __grid_constant__ BuildBitsParams p) {
   pdl_launch_dependents();
   pdl_wait();
+  // word ranges this CTA clears together: [0] before the first member, [1]
+  // after the last (each written by the one thread that finds it)
+  __shared__ int s_lo[2], s_hi[2];
+  if (threadIdx.x < 2) s_lo[threadIdx.x] = s_hi[threadIdx.x] = 0;
+  __syncthreads();
   const int b = blockIdx.y / p.nheads, h = p.heads[blockIdx.y % p.nheads];
   const int n = min(max(p.seqlens[b], 1), p.N_max);
-  int kb = p.k_per_seq ? p.k_per_seq[b] : p.k;
-  kb = min(min(max(kb, 1), p.k), n);
   const size_t bh = (size_t)b * p.Hq + h;
   uint32_t* row = p.bitmaps + bh * p.nwords;
   const int words = (n + 31) >> 5;
@@ -44,13 +48,14 @@ __global__ void __launch_bounds__(kThreads) build_bits_kernel(const __grid_const
     if (t >= p.k) break;
     const int j = idx[t];
     if (p.idx_out) p.idx_out[bh * p.k + t] = j;
-    if (t >= kb) continue;
     const int prev = t > 0 ? idx[t - 1] : -1;
     if (j < 0) {
-      // the set ends at its first -1: that entry clears the words after the
-      // last member (all of them for an empty set)
-      if (t == 0 || prev >= 0)
-        for (int g = t == 0 ? 0 : (prev >> 5) + 1; g < words; ++g) row[g] = 0u;
+      // the set ends at its first -1: the words after the last member (all of
+      // them for an empty set) are cleared below
+      if (t == 0 || prev >= 0) {
+        s_lo[1] = t == 0 ? 0 : (prev >> 5) + 1;
+        s_hi[1] = words;
+      }
       continue;
     }
     if (t > 0 && prev < 0) {   // a member after the end of the set
@@ -65,17 +70,28 @@ __global__ void __launch_bounds__(kThreads) build_bits_kernel(const __grid_const
     const int pw = prev >> 5;   // -1 for the first entry (arithmetic shift)
     if (w != pw) {
       uint32_t bits = 1u << (j & 31);
-      for (int u = t + 1; u < kb; ++u) {
+      for (int u = t + 1; u < p.k; ++u) {
         const int ju = idx[u];
         if ((ju >> 5) != w || ju <= j) break;
         bits |= 1u << (ju & 31);
       }
       row[w] = bits;
-      for (int g = max(pw + 1, 0); g < w; ++g) row[g] = 0u;
+      if (pw < 0) {            // the first member: the words before it, below
+        s_lo[0] = 0;
+        s_hi[0] = w;
+      } else {
+        for (int g = pw + 1; g < w; ++g) row[g] = 0u;
+      }
     }
-    if (t == kb - 1)
-      for (int g = w + 1; g < words; ++g) row[g] = 0u;
+    if (t == p.k - 1) {        // a full row: the words after its last member
+      s_lo[1] = w + 1;
+      s_hi[1] = words;
+    }
   }
+  __syncthreads();
+#pragma unroll
+  for (int e = 0; e < 2; ++e)
+    for (int g = s_lo[e] + threadIdx.x; g < s_hi[e]; g += kThreads) row[g] = 0u;
 }
 
 // Bitmaps -> index rows for every head: ascending positions, -1 padded to k.

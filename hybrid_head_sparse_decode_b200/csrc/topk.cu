@@ -17,6 +17,7 @@
 // Softmax is strictly increasing, so selecting on logits selects the same set as
 // selecting on attention weights.
 #include <algorithm>
+#include <mutex>
 
 #include "cluster.cuh"
 #include "combine_body.cuh"
@@ -325,16 +326,6 @@ __device__ __forceinline__ void topk_body(const TopkParams& p, int keys_cap, int
   cluster_wait();    // no CTA leaves while a histogram may still be on its way to it
 }
 
-template <int C>
-__global__ void __launch_bounds__(kThreads, 2)
-    topk_kernel(const __grid_constant__ TopkParams p, int keys_cap, int wpc_cap) {
-  extern __shared__ __align__(16) uint32_t dsm[];
-  pdl_launch_dependents();
-  topk_prologue<C>(dsm);
-  pdl_wait();
-  topk_body<C>(p, keys_cap, wpc_cap, blockIdx.x, dsm);
-}
-
 // Top-k of the retrieval heads and the combine of all heads in one launch: the
 // first ntopk CTAs (whole clusters) select, the next ncomb CTAs combine (each
 // head's kCombineSplit CTAs are one group of a cluster, since C is a multiple
@@ -394,52 +385,63 @@ void fill_config(cudaLaunchConfig_t& cfg, cudaLaunchAttribute* at, unsigned grid
   cfg.numAttrs = 2;
 }
 
-template <int C>
-cudaError_t set_attributes() {
-  static bool done = false;
-  if (done) return cudaSuccess;
-  cudaError_t e = cudaFuncSetAttribute(topk_kernel<C>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       (int)kSmemBudget);
-  if (e == cudaSuccess && C > 8)
-    e = cudaFuncSetAttribute(topk_kernel<C>, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
-  if (e == cudaSuccess) done = true;
-  return e;
+// Dynamic shared memory and (C = 16) the non-portable cluster size of the
+// fused kernel, once per device.
+template <int C, typename T, int D>
+cudaError_t set_tc_attributes() {
+  static PerDeviceOnce attrs;
+  return attrs.run([] {
+    auto kfn = topk_combine_kernel<C, T, D>;
+    cudaError_t e =
+        cudaFuncSetAttribute(kfn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemBudget);
+    if (e == cudaSuccess && C > 8)
+      e = cudaFuncSetAttribute(kfn, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+    return e;
+  });
 }
 
-template <int C>
-cudaError_t launch_c(const TopkParams& p, cudaStream_t st) {
-  const Geometry<C> g(p.N_max);
-  if (!g.ok) return cudaErrorInvalidValue;
-  cudaError_t e = set_attributes<C>();
-  if (e != cudaSuccess) return e;
-  cudaLaunchConfig_t cfg;
-  cudaLaunchAttribute at[2];
-  fill_config<C>(cfg, at, (unsigned)(C * p.B * p.nheads), g.smem, st);
-  e = cudaLaunchKernelEx(&cfg, topk_kernel<C>, p, g.keys_cap, g.wpc_cap);
-  if (e != cudaSuccess) return e;
-  return cudaGetLastError();
+// Shared memory of one CTA of the fused launch: the larger of its two roles'.
+template <int C, int D>
+size_t tc_smem(const Geometry<C>& g) {
+  return std::max(g.smem, combine_smem_bytes<D>());
 }
 
-// Whether clusters of 16 CTAs with this geometry can be resident (queried once
-// per process for the first N_max seen, and again if a larger one fails).
+// Whether clusters of 16 CTAs of the fused kernel, with the shared memory it is
+// launched with for rows of N_max logits, can be resident on the current
+// device.  Remembered per device for the largest N_max asked so far, and asked
+// again for a larger one.
+template <typename T, int D>
 bool cluster16_ok(int N_max, cudaStream_t st) {
-  static int known_n = -1;
-  static bool known_ok = false;
-  if (known_n >= N_max) return known_ok;
+  static std::mutex mu;
+  static int known_n[64];
+  static bool known_ok[64];
+  static bool init = false;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) {
+    cudaGetLastError();
+    return false;
+  }
+  std::lock_guard<std::mutex> lock(mu);
+  if (!init) {
+    for (int i = 0; i < 64; ++i) known_n[i] = -1;
+    init = true;
+  }
+  if (known_n[dev] >= N_max) return known_ok[dev];
   const Geometry<16> g(N_max);
-  bool ok = g.ok && set_attributes<16>() == cudaSuccess;
+  bool ok = g.ok && set_tc_attributes<16, T, D>() == cudaSuccess;
   if (ok) {
     cudaLaunchConfig_t cfg;
     cudaLaunchAttribute at[2];
-    fill_config<16>(cfg, at, 16u, g.smem, st);
+    fill_config<16>(cfg, at, 16u, tc_smem<16, D>(g), st);
     cfg.numAttrs = 1;   // the occupancy query needs only the cluster shape
     int nclusters = 0;
-    ok = cudaOccupancyMaxActiveClusters(&nclusters, topk_kernel<16>, &cfg) == cudaSuccess &&
+    ok = cudaOccupancyMaxActiveClusters(&nclusters, topk_combine_kernel<16, T, D>, &cfg) ==
+             cudaSuccess &&
          nclusters >= 1;
   }
   cudaGetLastError();   // a refused query leaves no sticky error
-  known_n = N_max;
-  known_ok = ok;
+  known_n[dev] = N_max;
+  known_ok[dev] = ok;
   return ok;
 }
 
@@ -448,18 +450,13 @@ cudaError_t launch_tc(const TopkParams& p, const CombineParams& cp, cudaStream_t
   static_assert(kThreads == kCombThreads, "one block size for both roles");
   const Geometry<C> g(p.N_max);
   if (!g.ok) return cudaErrorInvalidValue;
-  static bool done = false;
   auto kfn = topk_combine_kernel<C, T, D>;
-  if (!done) {
-    cudaError_t e = cudaFuncSetAttribute(kfn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemBudget);
-    if (e == cudaSuccess && C > 8) e = cudaFuncSetAttribute(kfn, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
-    if (e != cudaSuccess) return e;
-    done = true;
-  }
+  const cudaError_t ea = set_tc_attributes<C, T, D>();
+  if (ea != cudaSuccess) return ea;
   const int ntopk = C * p.B * p.nheads;
-  const int ncomb = cp.B * cp.Hq * kCombineSplit;
+  const int ncomb = cp.B * cp.Hq * kCombineSplit;   // 0: selection only
   const int grid = (ntopk + ncomb + C - 1) / C * C;
-  const size_t smem = std::max(g.smem, combine_smem_bytes<D>());
+  const size_t smem = tc_smem<C, D>(g);
   cudaLaunchConfig_t cfg;
   cudaLaunchAttribute at[2];
   fill_config<C>(cfg, at, (unsigned)grid, smem, st);
@@ -470,7 +467,13 @@ cudaError_t launch_tc(const TopkParams& p, const CombineParams& cp, cudaStream_t
 
 template <typename T, int D>
 cudaError_t launch_tc_d(const TopkParams& p, const CombineParams& cp, cudaStream_t st) {
-  return cluster16_ok(p.N_max, st) ? launch_tc<16, T, D>(p, cp, st) : launch_tc<8, T, D>(p, cp, st);
+  // 16 CTAs per head when the GPU can hold such clusters and the heads' CTAs
+  // fit one wave (two CTAs per SM); else 8, so that many heads (a layer of
+  // retrieval heads) are selected in one wave instead of two
+  const long long ctas16 = 16LL * p.B * p.nheads;
+  const bool one_wave = p.sms <= 0 || ctas16 <= 2LL * p.sms;
+  return one_wave && cluster16_ok<T, D>(p.N_max, st) ? launch_tc<16, T, D>(p, cp, st)
+                                                     : launch_tc<8, T, D>(p, cp, st);
 }
 
 }  // namespace
@@ -483,11 +486,6 @@ cudaError_t launch_topk_combine(const TopkParams& p, const CombineParams& cp, in
   if (dtype == 1 && D == 128) return launch_tc_d<float, 128>(p, cp, st);
   if (dtype == 1 && D == 64) return launch_tc_d<float, 64>(p, cp, st);
   return cudaErrorInvalidValue;
-}
-
-cudaError_t launch_topk(const TopkParams& p, cudaStream_t st) {
-  if (p.nheads <= 0) return cudaSuccess;
-  return cluster16_ok(p.N_max, st) ? launch_c<16>(p, st) : launch_c<8>(p, st);
 }
 
 }  // namespace lychee

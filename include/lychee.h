@@ -42,14 +42,13 @@
  *     trap: the offending entry is skipped or clamped, a flag is set in the
  *     workspace, and lychee_check_device_error() reports it.
  *   - Device pointers must be 16-byte aligned (q, caches, out, workspace).
- *   - Threads and devices: the first call of each kernel configuration in a
- *     process sets that kernel's attributes (dynamic shared memory, cluster
- *     size) on the current device and remembers that it did, with no lock.
- *     Make the first call of each configuration from one host thread, and use
- *     one device per process: a second device in the same process is not
- *     set up, and its launches may be refused (LYCHEE_ERR_CUDA).
- *     After the first calls, calls on different streams with their own
- *     workspaces may come from any thread.
+ *   - Threads and devices: every call launches on the current device (the
+ *     pointers it is given must live there).  The first call of each kernel
+ *     configuration on a device sets that kernel's attributes (dynamic shared
+ *     memory, cluster size) there and records it per device (atomically, for
+ *     device ordinals below 64; higher ordinals set them on every call), so
+ *     calls on several devices and from several host threads are fine as long
+ *     as calls sharing a workspace are ordered on one stream.
  */
 #ifndef LYCHEE_H
 #define LYCHEE_H
@@ -71,7 +70,7 @@ typedef enum {
   LYCHEE_OK = 0,
   LYCHEE_ERR_INVALID_ARG = 1, /* NULL pointer, bad shape, bad role value, misalignment */
   LYCHEE_ERR_UNSUPPORTED = 2, /* shape outside what the kernels are built for      */
-  LYCHEE_ERR_WORKSPACE = 3,   /* workspace NULL or smaller than lychee_workspace_size */
+  LYCHEE_ERR_WORKSPACE = 3,   /* workspace NULL, misaligned or too small for the call */
   LYCHEE_ERR_CUDA = 4,        /* a CUDA runtime call or launch failed               */
   LYCHEE_ERR_BAD_INDEX = 5,   /* device-side: bad incoming index / length / budget  */
   LYCHEE_ERR_TIMEOUT = 6      /* device-side: a pipeline wait gave up (never expected) */
@@ -105,18 +104,25 @@ typedef struct {
   int32_t block;  /* 0/1: token-level argsTopK; else positions per selected block */
 } lychee_shape;
 
-/* Bytes of device workspace that lychee_hybrid_decode_attn and
- * lychee_decode_stack need for shape *s (the same figure for both, any L).
- * Returns 0 if *s is invalid.  The workspace holds fp32 logits of retrieval
- * heads ([B, Hq, N_max], the raw dot products q.k, not divided by sqrt(d)),
- * split partials, one membership bitmap per head position ([B, Hq,
- * ceil(N_max/32)] uint32, bit j of word w = position 32w+j is in S), a work
- * counter and the device error word. */
+/* Bytes of device workspace that serve both lychee_hybrid_decode_attn and
+ * lychee_decode_stack for shape *s (any L).  Returns 0 if *s is invalid.  The
+ * workspace holds fp32 logits of retrieval heads ([B, Hq, N_max], the raw dot
+ * products q.k, not divided by sqrt(d)), split partials, one membership bitmap
+ * per head position ([B, Hq, ceil(N_max/32)] uint32, bit j of word w =
+ * position 32w+j is in S), work counters and the device error word.  The
+ * stack keeps two logits regions and three partial-state regions, so that a
+ * layer's attention overlaps the previous layer's selection and combine. */
 LYCHEE_API size_t lychee_workspace_size(const lychee_shape* s);
 
+/* Bytes of device workspace that lychee_hybrid_decode_attn alone needs for
+ * shape *s: the leading part of lychee_workspace_size(s) (one logits region,
+ * one partial-state region, the bitmaps).  Returns 0 if *s is invalid. */
+LYCHEE_API size_t lychee_layer_workspace_size(const lychee_shape* s);
+
 /* Byte offsets, inside a workspace for shape *s, of the fp32 logits region
- * [B, Hq, N_max] (raw q.k of the retrieval heads of the most recent layer,
- * positions j < n_b) and of the membership-bitmap region [B, Hq, nwords]
+ * [B, Hq, N_max] (raw q.k of the retrieval heads of the most recent
+ * lychee_hybrid_decode_attn call, positions j < n_b; the stack alternates
+ * between this region and another) and of the membership-bitmap region [B, Hq, nwords]
  * (nwords = ceil(N_max / 32)); *nwords receives nwords.  For inspection and
  * tests.  Returns LYCHEE_ERR_INVALID_ARG for an invalid shape or NULL output. */
 LYCHEE_API lychee_status lychee_workspace_offsets(const lychee_shape* s, size_t* logits_off,
@@ -139,7 +145,7 @@ LYCHEE_API lychee_status lychee_workspace_offsets(const lychee_shape* s, size_t*
  *   idx_out   device [B, Hq, k] int32: retrieval heads get argsTopK of their
  *             logits, or their block-granular set (s->block), ascending, -1
  *             padded; sparse heads get their idx_in row copied bit for bit
- *   workspace device, >= lychee_workspace_size(s) bytes, 256-byte aligned
+ *   workspace device, >= lychee_layer_workspace_size(s) bytes, 256-byte aligned
  *   stream    cudaStream_t
  * The call overwrites the whole workspace header, so device errors reported by
  * lychee_check_device_error() refer to the most recent call on that workspace. */
@@ -151,8 +157,8 @@ LYCHEE_API lychee_status lychee_hybrid_decode_attn(const lychee_shape* s, const 
                                         size_t workspace_bytes, void* stream);
 
 /* Size of the static device scratch behind lychee_hybrid_decode_attn_noalloc:
- * 64 MiB per device, enough for a layer whose lychee_workspace_size() is at
- * most that (e.g. B = 1, Hq = 32, d = 128, N_max = 131072 needs about 49 MiB). */
+ * 64 MiB per device, enough for a layer whose lychee_layer_workspace_size() is
+ * at most that (e.g. B = 1, Hq = 32, d = 128, N_max = 131072 needs about 49 MiB). */
 #define LYCHEE_NOALLOC_SCRATCH_BYTES (64u << 20)
 
 /* lychee_hybrid_decode_attn without a caller-owned workspace and without any
@@ -166,13 +172,16 @@ LYCHEE_API lychee_status lychee_hybrid_decode_attn(const lychee_shape* s, const 
  *   device_error device uint32 or NULL: receives, in stream order, the device
  *                error bits of this call (as lychee_check_device_error's detail)
  * Returns LYCHEE_ERR_WORKSPACE, before touching the GPU, when
- * lychee_workspace_size(s) exceeds LYCHEE_NOALLOC_SCRATCH_BYTES; the shape and
+ * lychee_layer_workspace_size(s) exceeds LYCHEE_NOALLOC_SCRATCH_BYTES; the shape and
  * argument errors of lychee_hybrid_decode_attn otherwise; LYCHEE_ERR_CUDA if the
  * scratch address cannot be looked up.
- * All calls on one device share the scratch: calls whose executions overlap
- * (other streams, host threads) race on it, so serialise them.  The first call
- * on each device looks the scratch address up (cudaGetSymbolAddress); make it
- * before any stream capture. */
+ * All calls in one CUDA context (one per device and process) share the
+ * scratch: calls whose executions overlap (other streams, host threads) race on
+ * it, so serialise them.  The first call on each device looks the scratch
+ * address up (cudaGetSymbolAddress); make it before any stream capture.  The
+ * address is remembered per device together with the context it was looked up
+ * in, and looked up again when the device's current context has changed (after
+ * cudaDeviceReset, say). */
 LYCHEE_API lychee_status lychee_hybrid_decode_attn_noalloc(const lychee_shape* s, const void* q,
                                         const void* k_cache, const void* v_cache,
                                         const int32_t* seqlens, const int32_t* k_per_seq,
@@ -200,6 +209,46 @@ LYCHEE_API lychee_status lychee_decode_stack(const lychee_shape* s, int32_t L, c
                                   int32_t* idx_layers, void* workspace, size_t workspace_bytes,
                                   void* stream);
 
+/* lychee_hybrid_decode_attn with a sliding-window branch on every sparse head,
+ * fused with its sparse branch by a sigmoid gate (page "HySparse: A Hybrid
+ * Sparse Attention Architecture with Oracle Token Selection and KV Cache
+ * Sharing", paperlayer.ai/abs/2602.03560v1, Methodology: sparse layers combine
+ * the sparse branch with a local sliding-window branch -- window 128, its own
+ * cache -- through sigmoid gating).  For a sparse head h of KV group g:
+ *   O_window = softmax(q_h . K_w^T / sqrt(d)) V_w over the min(window, n_b)
+ *              rows in use of the group's window ring,
+ *   out_h    = s * O_sparse + (1 - s) * O_window,  s = 1 / (1 + exp(-gate[b, h])).
+ * Retrieval heads are unchanged.  Extra arguments (the rest as in
+ * lychee_hybrid_decode_attn, whose results this gives for retrieval heads and
+ * for sets, bit for bit):
+ *   swa_k, swa_v device [B, Hkv, window, d] dtype, 16-byte aligned: the window
+ *                ring of each sequence and KV group, position j in row
+ *                j % window (rows 0 .. min(window, n_b) - 1 are read)
+ *   window       1 .. 1024 (the page's choice is 128)
+ *   gate         device [B, Hq] fp32 gate logits (read for sparse heads)
+ * Arithmetic: fp32 scores of exact products, fp32 softmax and sums. */
+LYCHEE_API lychee_status lychee_hybrid_decode_attn_swa(const lychee_shape* s, const void* q,
+                                        const void* k_cache, const void* v_cache,
+                                        const int32_t* seqlens, const int32_t* k_per_seq,
+                                        const uint8_t* head_role, const int32_t* idx_in,
+                                        const void* swa_k, const void* swa_v, int32_t window,
+                                        const float* gate, void* out, int32_t* idx_out,
+                                        void* workspace, size_t workspace_bytes, void* stream);
+
+/* lychee_decode_stack with the sliding-window branch of
+ * lychee_hybrid_decode_attn_swa on the sparse heads of every layer.
+ *   swa_k, swa_v HOST arrays of L device pointers, each [B, Hkv, window, d]
+ *   window       1 .. 1024
+ *   gate         device [L, B, Hq] fp32 gate logits
+ * The sets handed between layers do not depend on the window branch. */
+LYCHEE_API lychee_status lychee_decode_stack_swa(const lychee_shape* s, int32_t L, const void* q,
+                                  const void* const* k_caches, const void* const* v_caches,
+                                  const int32_t* seqlens, const int32_t* k_per_seq,
+                                  const uint8_t* head_role, const void* const* swa_k,
+                                  const void* const* swa_v, int32_t window, const float* gate,
+                                  void* out, int32_t* idx_final, int32_t* idx_layers,
+                                  void* workspace, size_t workspace_bytes, void* stream);
+
 /* The step before a layer's attention in a decode step: the current token's
  * key and value rows go into the caches at row n_b - 1 of their sequence (the
  * calls above read rows j < n_b, the current token included).  The rows are
@@ -217,6 +266,32 @@ LYCHEE_API lychee_status lychee_decode_stack(const lychee_shape* s, int32_t L, c
 LYCHEE_API lychee_status lychee_append_kv(const lychee_shape* s, const void* k_new,
                                           const void* v_new, void* k_cache, void* v_cache,
                                           const int32_t* seqlens, void* stream);
+
+/* Head roles from HardKuma gate parameters (method steps (1), (2), (7) and the
+ * closed-form expected L0 norm of the same page's novelty paragraph).  The gate
+ * of head h in layer l is z ~ HardKuma(alpha, beta): K ~ Kumaraswamy(alpha,
+ * beta) on (0, 1) with CDF F(x) = 1 - (1 - x^alpha)^beta, stretched to
+ * p + (q - p) K and rectified to [0, 1].  A head is a retrieval head when
+ * E[z] > 0.5; with layer0_retrieval, layer 0 is all retrieval whatever its
+ * parameters.  The expected L0 norm is the sum over the gated heads (every head
+ * but layer 0's when layer0_retrieval) of P(z != 0) = 1 - F(-p / (q - p)).
+ * Computed in fp64; E[z] by the integral (q - p) * integral_a^b (1 - k^alpha)^beta dk,
+ * a = -p/(q-p), b = (1-p)/(q-p), with composite Simpson's rule (2048 panels).
+ *   alpha, beta  device [L, Hq] double, finite and > 0 (a head with other values
+ *                gets E[z] = NaN and the sparse role, and makes the L0 sum NaN)
+ *   p, q         stretch limits, p < 0 and q > 1 (the HardKuma distribution's
+ *                usual choice is p = -0.1, q = 1.1; the pages give none)
+ *   head_role    device [L, Hq] uint8 out: LYCHEE_ROLE_RETRIEVAL / _SPARSE, the
+ *                form lychee_decode_stack takes (after a copy to the host)
+ *   expected_z   device [L, Hq] double out, or NULL
+ *   expected_l0  device [1] double out, or NULL
+ * Returns LYCHEE_ERR_INVALID_ARG for NULL inputs, L or Hq below 1, p >= 0,
+ * q <= 1 or pointers not 8-byte aligned; allocates nothing; one launch. */
+LYCHEE_API lychee_status lychee_hardkuma_roles(const double* alpha, const double* beta, int32_t L,
+                                               int32_t Hq, double p, double q,
+                                               int32_t layer0_retrieval, uint8_t* head_role,
+                                               double* expected_z, double* expected_l0,
+                                               void* stream);
 
 /* Synchronises `stream`, reads the device error word of `workspace` and clears
  * it.  Returns LYCHEE_OK, LYCHEE_ERR_BAD_INDEX, LYCHEE_ERR_TIMEOUT or

@@ -42,14 +42,21 @@ def shape(B=1, Hq=4, Hkv=2, d=128, N_max=1024, dtype=N.BF16, k=307):
 def test_workspace_size_valid_and_invalid(lib):
     s = shape()
     n = lib.lychee_workspace_size(ctypes.byref(s))
-    # header + logits + partials + bitmaps, each 256-byte aligned
-    assert n >= 256 + 1 * 4 * 1024 * 4 + 4 * 1 * (2 + 128) * 4 + 4 * 32 * 4
-    assert n % 256 == 0
+    m = lib.lychee_layer_workspace_size(ctypes.byref(s))
+    # the layer call: header + logits + partials + bitmaps, each 256-byte aligned
+    logits = 1 * 4 * 1024 * 4
+    partials = 4 * 2 * 12 * (2 + 128) * 4      # [B, Hq, nchunk = ceil(1024 / 768), 12 slots]
+    assert m >= 256 + logits + partials + 4 * 32 * 4
+    # the stack: a second logits region and two more partial-state regions
+    assert n >= m + logits + 2 * partials
+    assert n % 256 == 0 and m % 256 == 0
     bad = [shape(Hq=6, Hkv=4), shape(d=96), shape(k=0), shape(k=2000), shape(Hq=48, Hkv=3),
            shape(dtype=7), shape(B=0), shape(N_max=(1 << 24) + 1)]
     for b in bad:
         assert lib.lychee_workspace_size(ctypes.byref(b)) == 0
+        assert lib.lychee_layer_workspace_size(ctypes.byref(b)) == 0
     assert lib.lychee_workspace_size(None) == 0
+    assert lib.lychee_layer_workspace_size(None) == 0
 
 
 def test_block_selection_shapes(lib):
@@ -78,9 +85,9 @@ def test_workspace_offsets(lib):
     assert lib.lychee_workspace_offsets(ctypes.byref(s), ctypes.byref(lo), ctypes.byref(bo),
                                         ctypes.byref(nw)) == N.OK
     assert lo.value == 256 and nw.value == (5000 + 31) // 32
-    total = lib.lychee_workspace_size(ctypes.byref(s))
+    total = lib.lychee_layer_workspace_size(ctypes.byref(s))
     assert lo.value + 2 * 8 * 5000 * 4 <= bo.value
-    assert bo.value + 2 * 8 * nw.value * 4 <= total
+    assert bo.value + 2 * 8 * nw.value * 4 <= total <= lib.lychee_workspace_size(ctypes.byref(s))
 
 
 FAKE = 0x10000   # 16-byte aligned, never dereferenced: every call below fails on the host
@@ -151,7 +158,7 @@ def test_noalloc_refuses_shapes_beyond_its_scratch_on_host(lib):
             ctypes.byref(sh), FAKE, FAKE, FAKE, FAKE, None, ctypes.cast(r, ctypes.c_void_p),
             None, FAKE, FAKE, None, None)
     big = N.Shape(2, 32, 8, 128, 131072, N.BF16, 39321, 0)
-    assert lib.lychee_workspace_size(ctypes.byref(big)) > N.NOALLOC_SCRATCH_BYTES
+    assert lib.lychee_layer_workspace_size(ctypes.byref(big)) > N.NOALLOC_SCRATCH_BYTES
     assert call(big) == N.ERR_WORKSPACE
     assert call(shape(Hq=6, Hkv=4)) == N.ERR_INVALID_ARG
     assert call(shape(d=96)) == N.ERR_UNSUPPORTED
@@ -174,3 +181,47 @@ def test_binding_refuses_cpu_tensors(lib):
 def test_missing_library_fails_loudly(tmp_path):
     with pytest.raises(RuntimeError, match="not found"):
         N.load(str(tmp_path / "liblychee.so"))
+
+
+def test_hardkuma_roles_rejects_bad_arguments_on_host(lib):
+    def call(alpha=FAKE, beta=FAKE, L=2, Hq=4, p=-0.1, q=1.1, role=FAKE, ez=None, l0=None):
+        return lib.lychee_hardkuma_roles(alpha, beta, L, Hq, p, q, 1, role, ez, l0, None)
+    assert call(alpha=None) == N.ERR_INVALID_ARG
+    assert call(beta=None) == N.ERR_INVALID_ARG
+    assert call(role=None) == N.ERR_INVALID_ARG
+    assert call(L=0) == N.ERR_INVALID_ARG and call(Hq=0) == N.ERR_INVALID_ARG
+    assert call(p=0.0) == N.ERR_INVALID_ARG and call(q=1.0) == N.ERR_INVALID_ARG
+    assert call(p=float("nan")) == N.ERR_INVALID_ARG and call(q=float("inf")) == N.ERR_INVALID_ARG
+    assert call(ez=FAKE + 4) == N.ERR_INVALID_ARG
+    assert call(L=1 << 16, Hq=1 << 15) == N.ERR_UNSUPPORTED
+
+
+def test_window_branch_calls_reject_bad_arguments_on_host(lib):
+    s = shape()
+    r = (ctypes.c_uint8 * 4)(*[1, 0, 1, 0])
+    rp = ctypes.cast(r, ctypes.c_void_p)
+
+    def layer(swa_k=FAKE, swa_v=FAKE, window=128, gate=FAKE):
+        return lib.lychee_hybrid_decode_attn_swa(ctypes.byref(s), FAKE, FAKE, FAKE, FAKE, None, rp,
+                                                 FAKE, swa_k, swa_v, window, gate, FAKE, FAKE,
+                                                 FAKE, ctypes.c_size_t(1 << 40), None)
+    assert layer(swa_k=None) == N.ERR_INVALID_ARG
+    assert layer(swa_v=None) == N.ERR_INVALID_ARG and layer(gate=None) == N.ERR_INVALID_ARG
+    assert layer(window=0) == N.ERR_INVALID_ARG and layer(window=1025) == N.ERR_INVALID_ARG
+    assert layer(swa_k=FAKE + 8) == N.ERR_INVALID_ARG and layer(gate=FAKE + 2) == N.ERR_INVALID_ARG
+    L = 2
+    roles = (ctypes.c_uint8 * 8)(*[1, 1, 1, 1, 1, 0, 1, 0])
+    caches = (ctypes.c_void_p * L)(FAKE, FAKE)
+    rings = (ctypes.c_void_p * L)(FAKE, FAKE)
+    holes = (ctypes.c_void_p * L)(FAKE, None)
+
+    def stack(swa_k=rings, swa_v=rings, window=128, gate=FAKE):
+        return lib.lychee_decode_stack_swa(
+            ctypes.byref(s), L, FAKE, ctypes.cast(caches, ctypes.c_void_p),
+            ctypes.cast(caches, ctypes.c_void_p), FAKE, None, ctypes.cast(roles, ctypes.c_void_p),
+            None if swa_k is None else ctypes.cast(swa_k, ctypes.c_void_p),
+            None if swa_v is None else ctypes.cast(swa_v, ctypes.c_void_p), window, gate, FAKE,
+            FAKE, None, FAKE, ctypes.c_size_t(1 << 40), None)
+    assert stack(swa_k=None) == N.ERR_INVALID_ARG and stack(swa_v=None) == N.ERR_INVALID_ARG
+    assert stack(gate=None) == N.ERR_INVALID_ARG and stack(window=2000) == N.ERR_INVALID_ARG
+    assert stack(swa_k=holes) == N.ERR_INVALID_ARG

@@ -137,12 +137,14 @@ def test_reference_arm_on_rank0_prints_the_contract_keys(block):
     assert res["impl"] == "reference" and res["value"] > 0 and not res["higher_is_better"]
     assert res["e2e"]["value"] == res["value"] and res["cpu_baseline"]["kind"] == "oracle"
     assert res["config"]["select"] == ("argsTopK" if block == 0 else "blocks of 32")
+    assert "all 2 layers" in res["cpu_baseline"]["sample"]
 
 
 def test_cpu_baseline_leg_runs_on_host_tensors():
     sys.path.insert(0, ROOT)
     import bench
     prob = bench.make_workload("qwen3_stack_256x3", torch.device("cpu"))
-    cb = bench.cpu_baseline(prob, sample_layers=2, block=32)
+    cb = bench.cpu_baseline(prob, block=32, single_layers=2)
     assert cb["kind"] == "oracle" and cb["value"] > 0 and cb["cores"] >= 1
-    assert "layers 0..1" in cb["sample"]
+    assert "all 3 layers" in cb["sample"] and cb["cpu_model"]
+    assert cb["single_thread"]["cores"] == 1 and "layers 0..1" in cb["single_thread"]["sample"]

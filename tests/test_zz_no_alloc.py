@@ -33,7 +33,7 @@ def test_scratch_size_matches_header():
 def test_oversize_layer_refused_on_host(lib):
     # B = 2, Hq = 32, N_max = 131072: ~86 MiB of scratch > 64 MiB
     s = N.Shape(2, 32, 8, 128, 131072, N.BF16, 39321)
-    assert lib.lychee_workspace_size(ctypes.byref(s)) > N.NOALLOC_SCRATCH_BYTES
+    assert lib.lychee_layer_workspace_size(ctypes.byref(s)) > N.NOALLOC_SCRATCH_BYTES
     roles = (ctypes.c_uint8 * 32)(*([1] * 32))
     st = lib.lychee_hybrid_decode_attn_noalloc(
         ctypes.byref(s), FAKE, FAKE, FAKE, FAKE, None, ctypes.cast(roles, ctypes.c_void_p), None,
@@ -98,3 +98,43 @@ def test_noalloc_binding_refuses_oversize_layer():
     sl = torch.full((2,), 131072, dtype=torch.int32, device=DEV)
     with pytest.raises(ValueError, match="static scratch"):
         ops.hybrid_decode_attn_noalloc(q, kv, kv, sl, [1] * 32, None, 39321)
+
+
+@pytest.mark.gpu
+def test_noalloc_same_shape_state_does_not_leak():
+    """Three calls of one shape in a row on the shared scratch, where head 1
+    flips from sparse to retrieval and back and the sparse heads' incoming sets
+    change between the calls: each equals the workspace call bit for bit, so
+    nothing a call leaves in the scratch (bitmaps, partial states, logits,
+    counters) reaches the next; and the device's free memory, as the driver
+    reports it, does not move across the calls (after one warm-up call, which
+    may load the library's device code)."""
+    import dataclasses
+    a = inputs.make_layer(1, 8, 2, 128, 6000, roles=[1, 0, 0, 0, 0, 1, 0, 0], seed=35,
+                          k_frac=0.3, n_planted=8)
+    other = inputs.make_layer(1, 8, 2, 128, 6000, roles=[1, 0, 0, 0, 0, 1, 0, 0], seed=36,
+                              k_frac=0.3)
+    role_b = a.role.clone()
+    role_b[1] = 1
+    b = dataclasses.replace(a, role=role_b, idx_in=other.idx_in)
+    q, kc, vc = a.q.to(DEV), a.k_cache.to(DEV), a.v_cache.to(DEV)
+    sl, kps = a.seqlens.to(DEV), a.k_per_seq.to(DEV)
+    refs = []
+    for prob in (a, b, a):
+        refs.append(ops.hybrid_decode_attn(q, kc, vc, sl, prob.role, prob.idx_in.to(DEV), a.k,
+                                           k_per_seq=kps))
+    outs = [(torch.empty_like(r[0]), torch.empty_like(r[1])) for r in refs]
+    err = torch.zeros(1, dtype=torch.int32, device=DEV)
+    idx_dev = [prob.idx_in.to(DEV) for prob in (a, b, a)]
+    ops.hybrid_decode_attn_noalloc(q, kc, vc, sl, a.role, idx_dev[0], a.k, k_per_seq=kps,
+                                   out=outs[0][0], idx_out=outs[0][1], device_error=err)
+    torch.cuda.synchronize()
+    free0 = torch.cuda.mem_get_info()[0]
+    for prob, idx, (o, i) in zip((a, b, a), idx_dev, outs):
+        ops.hybrid_decode_attn_noalloc(q, kc, vc, sl, prob.role, idx, a.k, k_per_seq=kps,
+                                       out=o, idx_out=i, device_error=err)
+        torch.cuda.synchronize()
+        assert int(err.item()) == 0
+    assert torch.cuda.mem_get_info()[0] == free0
+    for (o, i), (ro, ri) in zip(outs, refs):
+        assert torch.equal(o, ro) and torch.equal(i, ri)
