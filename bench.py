@@ -343,6 +343,49 @@ def run_lychee(args, rank, world, device):
     d1.record(stream)
     torch.cuda.synchronize()
     dense_ms = d0.elapsed_time(d1) / dsteps
+    # its per-kernel split (events around every launch, which serialise it)
+    dprof = ops.Profile(max_launches=dsteps * (4 * L + 2) + 16)
+    torch.cuda.synchronize()
+    with dprof:
+        for _ in range(dsteps):
+            step(dense_roles, dense_out)
+        torch.cuda.synchronize()
+    dkinds = {}
+    for k, ms in dprof.records:
+        dkinds[k] = dkinds.get(k, 0.0) + ms / dsteps
+
+    # the step before the attention of a decode step, timed on its own: the
+    # current token's K/V rows into every layer's cache (the rows already there,
+    # so the caches do not change)
+    b_idx = torch.arange(B, device=device)
+    last = (prob.seqlens.long() - 1)
+    k_new = [kc[b_idx, :, last].contiguous() for kc in prob.k_caches]
+    v_new = [vc[b_idx, :, last].contiguous() for vc in prob.v_caches]
+
+    def append_all():
+        for l in range(L):
+            ops.append_kv(k_new[l], v_new[l], prob.k_caches[l], prob.v_caches[l], prob.seqlens)
+
+    for _ in range(2):
+        append_all()
+    # replayed from a CUDA graph, so that the host's per-call work is not timed
+    gstream = torch.cuda.Stream()
+    graph = torch.cuda.CUDAGraph()
+    torch.cuda.synchronize()
+    with torch.cuda.stream(gstream):
+        with torch.cuda.graph(graph, stream=gstream):
+            append_all()
+    for _ in range(2):
+        graph.replay()
+    a0, a1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    a0.record(stream)
+    for _ in range(args.steps):
+        graph.replay()
+    a1.record(stream)
+    torch.cuda.synchronize()
+    append_ms = a0.elapsed_time(a1) / args.steps
+    del graph
 
     # end to end through the public call with host buffers: q (and the per-sequence
     # lengths and budgets) copied in from pinned memory, out and the final sets read
@@ -416,9 +459,14 @@ def run_lychee(args, rank, world, device):
         "kernels_ms_per_step": {k: round(v[1] / args.steps, 4) for k, v in kinds.items()},
         "dense_comparator": {"ms_per_step": round(dense_ms, 4),
                              "hbm_gbs": round(sum(dense_bytes) / (dense_ms * 1e-3) / 1e9, 1),
-                             "speedup_hybrid_vs_dense": round(dense_ms / ms_step, 3)},
+                             "speedup_hybrid_vs_dense": round(dense_ms / ms_step, 3),
+                             "kernels_ms_per_step": {k: round(v, 4) for k, v in dkinds.items()}},
         "e2e": {"value": round(job_us_per_step(e_ms / args.steps, world), 3), "unit": UNIT,
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+        "append_kv": {"ms_per_step": round(append_ms, 4), "launches_per_step": L,
+                      "note": "the current token's K/V rows into all layers' caches, one launch "
+                              "per layer, replayed from a CUDA graph; the step above starts from "
+                              "caches that hold them"},
         "gpu_launches": sum(v[0] for v in kinds.values()),
         "clocks": sampler.summary(),
     }

@@ -197,3 +197,16 @@ def test_sparse_row_copies_without_tensor_maps():
            os.path.join(here, "test_gpu_layer.py") + "::test_deterministic_bitwise"]
     r = subprocess.run(cmd, env=env, capture_output=True, text=True, timeout=900)
     assert r.returncode == 0, r.stdout[-3000:] + r.stderr[-3000:]
+
+
+def test_large_batch_item_space():
+    """More than 1024 sequences: the attention kernel enumerates every (sequence,
+    chunk) pair and skips chunks past n_b instead of keeping per-sequence chunk
+    counts in shared memory.  Ragged short sequences, both head roles."""
+    B = 1100
+    g = torch.Generator().manual_seed(1101)
+    seqlens = torch.randint(1, 41, (B,), generator=g).tolist()
+    prob = inputs.make_layer(B, 4, 2, 128, 40, roles=[1, 0, 0, 1], seed=1102, seqlens=seqlens,
+                             k_fixed=12, idx_mode="random")
+    err, rep = check_layer(prob)
+    assert rep.exact + rep.near_tie == 2 * B

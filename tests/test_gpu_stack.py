@@ -207,3 +207,20 @@ def test_stack_layer_outputs_match_single_layer_calls():
         err = (o1.float() - out[l].float()).abs().max().item()
         assert err <= 2e-2, (l, err)
         assert torch.equal(i1, lay[l]), l
+
+
+def test_stack_large_batch_item_space():
+    """A stack over more than 1024 sequences (the attention kernel's
+    non-compact item space, with the groups waiting for the previous layer's
+    sets taken last): every layer teacher-forced against the oracle."""
+    B = 1100
+    g = torch.Generator().manual_seed(4401)
+    seqlens = torch.randint(1, 65, (B,), generator=g).tolist()
+    prob = inputs.make_stack(3, B, 4, 2, 128, 64, seed=4402, seqlens=seqlens, k_fixed=20,
+                             n_extra_retrieval=3)
+    out, idx_final, idx_layers = run_stack(prob)
+    rep = SetReport()
+    for l in range(3):
+        teacher_forced_layer(prob, l, out, idx_layers, rep)
+    assert not rep.failures, rep.failures[:5]
+    assert torch.equal(idx_final, idx_layers[-1])
