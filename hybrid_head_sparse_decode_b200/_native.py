@@ -35,7 +35,8 @@ NOALLOC_SCRATCH_BYTES = 64 << 20
 EXPORTED = ("lychee_workspace_size", "lychee_layer_workspace_size", "lychee_workspace_offsets", "lychee_hybrid_decode_attn",
             "lychee_hybrid_decode_attn_noalloc", "lychee_decode_stack",
             "lychee_check_device_error", "lychee_status_string", "lychee_version",
-            "lychee_profile_begin", "lychee_profile_end", "lychee_append_kv",
+            "lychee_profile_begin", "lychee_profile_spans_begin", "lychee_profile_end",
+            "lychee_append_kv",
             "lychee_hardkuma_roles", "lychee_hybrid_decode_attn_swa", "lychee_decode_stack_swa")
 
 
@@ -101,6 +102,8 @@ def load(path: str | None = None):
         lib.lychee_version.restype = i32
         lib.lychee_profile_begin.argtypes = [i32]
         lib.lychee_profile_begin.restype = ctypes.c_int
+        lib.lychee_profile_spans_begin.argtypes = [i32]
+        lib.lychee_profile_spans_begin.restype = ctypes.c_int
         lib.lychee_profile_end.argtypes = [i32, vp, vp, ctypes.POINTER(i32)]
         lib.lychee_profile_end.restype = ctypes.c_int
         if path is None:

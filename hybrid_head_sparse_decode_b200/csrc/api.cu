@@ -197,9 +197,13 @@ bool encode_row_map(CUtensorMap* m, const void* base, const lychee_shape* s) {
 }
 
 // ---- optional launch profiler ----------------------------------------------------
+// Per-launch mode: two events around every launch.  Span mode: two events per
+// stack call, before its first attention launch and after its last one, and
+// none in between, so that the layers still overlap.
 struct Profiler {
   std::mutex mu;
   bool on = false;
+  bool spans = false;
   int cap = 0, n = 0;
   std::vector<cudaEvent_t> ev;
   std::vector<int32_t> kinds;
@@ -212,14 +216,33 @@ enum {
   kKindCombine = 2,
   kKindBuildBits = 3,
   kKindExport = 4,
-  kKindTopkCombine = 5
+  kKindTopkCombine = 5,
+  kKindAttnSpan = 6
 };
+
+// Span mode: open (end = false) or close (end = true) the current stack call's
+// attention span on `st`.
+void span_mark(bool end, cudaStream_t st) {
+  if (!g_prof.on || !g_prof.spans) return;
+  std::lock_guard<std::mutex> g(g_prof.mu);
+  if (!g_prof.on || !g_prof.spans) return;
+  if (!end) {
+    if (g_prof.n >= g_prof.cap) return;
+    const int i = g_prof.n++;
+    g_prof.kinds[i] = -1;   // open
+    cudaEventRecord(g_prof.ev[2 * i], st);
+  } else if (g_prof.n > 0 && g_prof.kinds[g_prof.n - 1] == -1) {
+    const int i = g_prof.n - 1;
+    g_prof.kinds[i] = kKindAttnSpan;
+    cudaEventRecord(g_prof.ev[2 * i + 1], st);
+  }
+}
 
 template <typename F>
 cudaError_t timed(int kind, cudaStream_t st, F&& launch) {
-  if (!g_prof.on) return launch();
+  if (!g_prof.on || g_prof.spans) return launch();
   std::lock_guard<std::mutex> g(g_prof.mu);
-  if (!g_prof.on || g_prof.n >= g_prof.cap) return launch();
+  if (!g_prof.on || g_prof.spans || g_prof.n >= g_prof.cap) return launch();
   const int i = g_prof.n++;
   g_prof.kinds[i] = kind;
   cudaEventRecord(g_prof.ev[2 * i], st);
@@ -271,6 +294,8 @@ struct LayerPlan {
   const uint8_t* prev_role = nullptr;   // stack: the previous layer's roles (null: none)
   int tail_pbuf = -1;          // stack: partial region of the previous layer, combined
   void* tail_out = nullptr;    //   by this layer's attention CTAs into tail_out
+  bool span_start = false;     // profiler span mode: the stack's first / last
+  bool span_end = false;       //   attention launch
   WindowParams win{};          // this layer's window branch (single layer; k null: none)
   WindowParams tail_win{};     // the previous layer's window branch (stack)
 };
@@ -401,8 +426,10 @@ lychee_status run_layer(const Ctx& c, const void* q, const void* kc, const void*
   ap.withhold_first = attn_withhold_first_item() ? 1 : 0;
   ap.gather_tma = !tma_gathers_disabled() && encode_row_map(&ap.tmk, kc, s) &&
                    encode_row_map(&ap.tmv, vc, s) ? 1 : 0;
+  if (plan.span_start) span_mark(false, c.st);
   e = timed(kKindAttn, c.st, [&] { return launch_attn(ap, s->dtype, s->d, G, c.sms, c.st); });
   if (e != cudaSuccess) return LYCHEE_ERR_CUDA;
+  if (plan.span_end) span_mark(true, c.st);
   // the retrieval heads' selection; in the single-layer call the same launch
   // combines every head (logits vs partial states: disjoint inputs and outputs)
   TopkParams tp{};
@@ -583,6 +610,8 @@ lychee_status stack_impl(const lychee_shape* s, int32_t L, const void* q,
     plan.pbuf = l % kPartBufs;
     plan.write_bits = true;
     plan.fused_combine = false;
+    plan.span_start = l == 0;
+    plan.span_end = l == L - 1;
     if (l > 0) {
       plan.prev_role = head_role + (size_t)(l - 1) * s->Hq;
       plan.tail_pbuf = (l - 1) % kPartBufs;
@@ -729,8 +758,13 @@ const char* lychee_status_string(lychee_status st) {
 
 int32_t lychee_version(void) { return kVersion; }
 
-lychee_status lychee_profile_begin(int32_t max_launches) {
-  if (max_launches < 1) return LYCHEE_ERR_INVALID_ARG;
+}  // extern "C"
+
+namespace {
+
+lychee_status profile_begin(int32_t max_records, bool spans) {
+  if (max_records < 1) return LYCHEE_ERR_INVALID_ARG;
+  const int32_t max_launches = max_records;
   std::lock_guard<std::mutex> g(g_prof.mu);
   if (g_prof.on) return LYCHEE_ERR_INVALID_ARG;
   if ((int)g_prof.ev.size() < 2 * max_launches) {
@@ -745,15 +779,29 @@ lychee_status lychee_profile_begin(int32_t max_launches) {
   g_prof.kinds.assign(max_launches, -1);
   g_prof.cap = max_launches;
   g_prof.n = 0;
+  g_prof.spans = spans;
   g_prof.on = true;
   return LYCHEE_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+lychee_status lychee_profile_begin(int32_t max_launches) {
+  return profile_begin(max_launches, false);
+}
+
+lychee_status lychee_profile_spans_begin(int32_t max_spans) {
+  return profile_begin(max_spans, true);
 }
 
 lychee_status lychee_profile_end(int32_t capacity, int32_t* kinds, float* ms, int32_t* n_out) {
   std::lock_guard<std::mutex> g(g_prof.mu);
   if (!g_prof.on) return LYCHEE_ERR_INVALID_ARG;
   g_prof.on = false;
-  const int n = g_prof.n;
+  int n = g_prof.n;
+  if (n > 0 && g_prof.kinds[n - 1] == -1) --n;   // a span left open (a failed call)
   if (n_out) *n_out = n;
   for (int i = 0; i < n && i < capacity; ++i) {
     if (cudaEventSynchronize(g_prof.ev[2 * i + 1]) != cudaSuccess) return LYCHEE_ERR_CUDA;

@@ -342,16 +342,23 @@ def workspace_views(workspace, B, Hq, Hkv, d, N_max, k, dtype):
 
 class Profile:
     """Context manager around lychee_profile_begin / lychee_profile_end.
-    After exit, ``records`` is a list of (kind, ms) per library launch."""
+    After exit, ``records`` is a list of (kind, ms) per library launch.  With
+    spans=True (lychee_profile_spans_begin) there is one ("attn_span", ms)
+    record per stack call instead, and no event between its launches."""
     KINDS = {0: "attn", 1: "topk", 2: "combine", 3: "build_bits", 4: "export",
-             5: "topk+combine"}
+             5: "topk+combine", 6: "attn_span"}
 
-    def __init__(self, max_launches=4096):
+    def __init__(self, max_launches=4096, spans=False):
         self.max_launches = int(max_launches)
+        self.spans = bool(spans)
         self.records = []
 
     def __enter__(self):
-        _check(N.load().lychee_profile_begin(self.max_launches), "lychee_profile_begin")
+        if self.spans:
+            _check(N.load().lychee_profile_spans_begin(self.max_launches),
+                   "lychee_profile_spans_begin")
+        else:
+            _check(N.load().lychee_profile_begin(self.max_launches), "lychee_profile_begin")
         return self
 
     def __exit__(self, *exc):

@@ -312,11 +312,19 @@ LYCHEE_API int32_t lychee_version(void);
  * events and writes, for the first min(n, capacity) launches, the kind
  * (0 attention, 1 top-k, 2 combine, 3 set->bitmap, 4 bitmap->set, 5 the
  * retrieval heads' selection -- argsTopK, or the block selection when
- * s->block > 1 -- and the combine in one launch) and the
+ * s->block > 1 -- and the combine in one launch; in a stack, 1 is the
+ * selection alone) and the
  * elapsed milliseconds; *n_out receives n.  Process-global state: one profiling
  * session at a time.  Events are created on the current device on first use
  * and kept for reuse. */
 LYCHEE_API lychee_status lychee_profile_begin(int32_t max_launches);
+/* Span mode of the same profiler: no events between launches (the layers of a
+ * stack still overlap), but per lychee_decode_stack(_swa) call two events, one
+ * before its first attention launch and one after its last, up to max_spans
+ * calls; lychee_profile_end reports each as kind 6 with the milliseconds
+ * between them (the time the call's attention launches take, back to back,
+ * with the selections that overlap them). */
+LYCHEE_API lychee_status lychee_profile_spans_begin(int32_t max_spans);
 LYCHEE_API lychee_status lychee_profile_end(int32_t capacity, int32_t* kinds, float* ms, int32_t* n_out);
 
 #ifdef __cplusplus

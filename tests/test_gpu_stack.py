@@ -224,3 +224,25 @@ def test_stack_large_batch_item_space():
         teacher_forced_layer(prob, l, out, idx_layers, rep)
     assert not rep.failures, rep.failures[:5]
     assert torch.equal(idx_final, idx_layers[-1])
+
+
+def test_profiler_span_mode():
+    """Span mode: one record per stack call (kind "attn_span"), none per launch;
+    per-launch mode: one record per launch, attention launches included."""
+    prob = inputs.make_stack(4, 1, 8, 2, 128, 3000, seed=4501, k_frac=0.3, n_extra_retrieval=3)
+    q = prob.q.to(DEV)
+    kc = [t.to(DEV) for t in prob.k_caches]
+    vc = [t.to(DEV) for t in prob.v_caches]
+    sl, kps = prob.seqlens.to(DEV), prob.k_per_seq.to(DEV)
+    ws = ops.alloc_workspace(1, 8, 2, 128, 3000, prob.k, q.dtype)
+    with ops.Profile(max_launches=16, spans=True) as pr:
+        for _ in range(3):
+            ops.decode_stack(q, kc, vc, sl, prob.roles, prob.k, k_per_seq=kps, workspace=ws)
+        torch.cuda.synchronize()
+    assert [k for k, _ in pr.records] == ["attn_span"] * 3
+    assert all(ms > 0 for _, ms in pr.records)
+    with ops.Profile(max_launches=256) as pl:
+        ops.decode_stack(q, kc, vc, sl, prob.roles, prob.k, k_per_seq=kps, workspace=ws)
+        torch.cuda.synchronize()
+    kinds = [k for k, _ in pl.records]
+    assert kinds.count("attn") == 4 and "attn_span" not in kinds

@@ -119,3 +119,50 @@ def test_window_arguments_are_checked():
     with pytest.raises(N.LycheeError) as e:
         ops.hybrid_decode_attn(*args, swa=(big, big, torch.zeros((1, 4), device=DEV)))
     assert e.value.status == N.ERR_INVALID_ARG
+
+
+def test_stack_with_window_branch_block_mode_and_graph_replay():
+    """Block-granular sets with the window branch: the stack captured into a
+    CUDA graph replays bit for bit, and its last layer (combined by the final
+    combine launch, not by a tail) matches the oracle."""
+    block = 64
+    prob = inputs.make_stack(4, 1, 8, 2, 128, 4000, seed=4700, k_frac=0.3, n_planted=16,
+                             n_extra_retrieval=4)
+    L, B, Hq, Hkv, d, N_max = prob.shape
+    window = 128
+    krs, vrs = zip(*[rings(B, Hkv, window, d, torch.bfloat16, 4710 + l) for l in range(L)])
+    gate = gates((L, B, Hq), 4720).to(DEV)
+    q = prob.q.to(DEV)
+    kc = [t.to(DEV) for t in prob.k_caches]
+    vc = [t.to(DEV) for t in prob.v_caches]
+    krd = [t.to(DEV) for t in krs]
+    vrd = [t.to(DEV) for t in vrs]
+    sl, kps = prob.seqlens.to(DEV), prob.k_per_seq.to(DEV)
+    ws = ops.alloc_workspace(B, Hq, Hkv, d, N_max, prob.k, q.dtype, block=block)
+    out = torch.empty((L, B, Hq, d), dtype=q.dtype, device=DEV)
+    fin = torch.empty((B, Hq, prob.k), dtype=torch.int32, device=DEV)
+    lay = torch.empty((L, B, Hq, prob.k), dtype=torch.int32, device=DEV)
+    kw = dict(k_per_seq=kps, out=out, idx_final=fin, idx_layers=lay, workspace=ws, block=block,
+              swa=(krd, vrd, gate))
+    ops.decode_stack(q, kc, vc, sl, prob.roles, prob.k, **kw)
+    torch.cuda.synchronize()
+    ref_o, ref_f, ref_l = out.clone(), fin.clone(), lay.clone()
+    s = torch.cuda.Stream()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.stream(s):
+        with torch.cuda.graph(g, stream=s):
+            ops.decode_stack(q, kc, vc, sl, prob.roles, prob.k, stream=s, **kw)
+    out.zero_()
+    fin.zero_()
+    g.replay()
+    torch.cuda.synchronize()
+    assert torch.equal(out, ref_o) and torch.equal(fin, ref_f)
+    l = L - 1
+    ref, _, _ = oracle.hybrid_layer(host_bits(prob.q[l]), host_bits(prob.k_caches[l]),
+                                    host_bits(prob.v_caches[l]), prob.seqlens.numpy(),
+                                    prob.roles[l].numpy(), ref_l[l - 1].cpu().numpy(), prob.k,
+                                    k_per_seq=prob.k_per_seq.numpy(), block=block)
+    want = oswa.layer_with_window(ref, prob.roles[l].numpy(), host_bits(prob.q[l]),
+                                  host_bits(krs[l]), host_bits(vrs[l]), prob.seqlens.numpy(),
+                                  window, gate[l].double().cpu().numpy())
+    compare_outputs(ref_o[l], want, torch.bfloat16)
