@@ -564,7 +564,11 @@ def time_layer_call(prob, steps, warmup, flush, all_retrieval):
             call()
         torch.cuda.synchronize()
     attn = sorted(ms for k, ms in prof.records if k == "attn")
-    return per, attn
+    split = {}
+    for k, ms in prof.records:
+        split.setdefault(k, []).append(ms)
+    split = {k: round(statistics.median(v) * 1e3, 2) for k, v in split.items()}
+    return per, attn, split
 
 
 def run_sweep(args, device):
@@ -581,7 +585,7 @@ def run_sweep(args, device):
             prob = inputs.sweep_layer(B, N, km, device=device, all_retrieval=False)
             dense = mode == "dense"
             u, lit = layer_rows(prob, dense)
-            per, attn = time_layer_call(prob, args.steps, args.warmup, flush, dense)
+            per, attn, split = time_layer_call(prob, args.steps, args.warmup, flush, dense)
             row_bytes = 2 * prob.shape[3] * prob.q.element_size()
             med = nearest_rank(per, 0.5)
             am = nearest_rank(attn, 0.5) if attn else float("nan")
@@ -593,7 +597,8 @@ def run_sweep(args, device):
                 "gbs_union": round(u * row_bytes / (med * 1e-3) / 1e9, 1),
                 "gbs_literal": round(lit * row_bytes / (med * 1e-3) / 1e9, 1),
                 "attn_gbs_union": round(u * row_bytes / (am * 1e-3) / 1e9, 1),
-                "attn_frac": round(u * row_bytes / (am * 1e-3) / 1e9 / peak, 4)}
+                "attn_frac": round(u * row_bytes / (am * 1e-3) / 1e9 / peak, 4),
+                "kernels_us": split}
             del prob
             torch.cuda.empty_cache()
         rec["speedup_hybrid_vs_dense"] = round(rec["dense"]["us"] / rec["hybrid"]["us"], 3)

@@ -37,6 +37,13 @@ struct Layout {
 
 size_t align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
 
+// The shortest attention work item the shape may get: kChunkMin positions, or
+// kChunkSmall when the layer's K/V rows (B * Hkv * N_max) are too few to give
+// every SM an item of kChunkMin.  The partial-state regions hold room for it.
+int chunk_lo(const lychee_shape* s) {
+  return (long long)s->B * s->Hkv * s->N_max < kSmallLayerRows ? kChunkSmall : kChunkMin;
+}
+
 lychee_status check_shape(const lychee_shape* s) {
   if (!s) return LYCHEE_ERR_INVALID_ARG;
   if (s->B < 1 || s->Hq < 1 || s->Hkv < 1 || s->d < 1 || s->N_max < 1 || s->k < 1)
@@ -49,7 +56,7 @@ lychee_status check_shape(const lychee_shape* s) {
   if (s->Hq > kMaxHq) return LYCHEE_ERR_UNSUPPORTED;
   if (s->d != 64 && s->d != 128) return LYCHEE_ERR_UNSUPPORTED;
   if (s->N_max > (1 << 24)) return LYCHEE_ERR_UNSUPPORTED;
-  const long long nchunk = (s->N_max + kChunkMin - 1) / kChunkMin;
+  const long long nchunk = (s->N_max + chunk_lo(s) - 1) / chunk_lo(s);
   if ((long long)s->B * s->Hkv * nchunk >= (1LL << 31)) return LYCHEE_ERR_UNSUPPORTED;
   if ((long long)s->B * s->Hq >= (1LL << 24)) return LYCHEE_ERR_UNSUPPORTED;
   if (s->block < 0) return LYCHEE_ERR_INVALID_ARG;
@@ -62,7 +69,7 @@ lychee_status check_shape(const lychee_shape* s) {
 
 Layout layout_of(const lychee_shape* s) {
   Layout L{};
-  L.nchunk = (s->N_max + kChunkMin - 1) / kChunkMin;   // room for the shortest chunk
+  L.nchunk = (s->N_max + chunk_lo(s) - 1) / chunk_lo(s);   // room for the shortest chunk
   L.nwords = (s->N_max + 31) / 32;
   const size_t bh = (size_t)s->B * s->Hq;
   const size_t logits_b = align256(bh * s->N_max * 4);
@@ -267,14 +274,15 @@ struct Ctx {
 };
 
 // Positions per attention work item: among the multiples of 32 in
-// [kChunkMin, kChunk], the one that minimises the work of the busiest SM for
+// [chunk_lo(s), kChunk], the one that minimises the work of the busiest SM for
 // full-length sequences, (items per SM, rounded up) x positions per item;
 // ties go to the longer chunk (fewer partial states).  Items are claimed
-// dynamically, so this only evens out the last wave.
+// dynamically, so this only evens out the last wave (and, for a small layer,
+// spreads its rows over more SMs).
 int pick_chunk(const lychee_shape* s, int sms) {
   int best = kChunk;
   long long best_cost = -1;
-  for (int cs = kChunk; cs >= kChunkMin; cs -= 32) {
+  for (int cs = kChunk; cs >= chunk_lo(s); cs -= 32) {
     const long long items = (long long)s->B * s->Hkv * ((s->N_max + cs - 1) / cs);
     const long long cost = (items + sms - 1) / sms * cs;
     if (best_cost < 0 || cost < best_cost) {

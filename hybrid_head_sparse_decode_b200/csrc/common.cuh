@@ -32,7 +32,9 @@ struct WsHeader {
 static_assert(sizeof(WsHeader) == 256, "header is 256 bytes");
 
 constexpr int kChunk = 960;           // positions per attention work item, at most (30 words)
-constexpr int kChunkMin = 768;        // ... and at least (the host picks one per launch)
+constexpr int kChunkMin = 768;        // ... and at least (the host picks one per launch),
+constexpr int kChunkSmall = 128;      // ... or this for a layer with fewer K/V rows than
+constexpr long long kSmallLayerRows = 256LL * kChunkMin;   // this (too few for every SM)
 constexpr int kPartSlots = 12;        // partial states per (sequence, head, chunk): one per warp
 constexpr int kMaxHq = 128;           // query heads supported
 constexpr int kMaxWindow = 1024;      // rows of a sparse head's sliding-window ring, at most

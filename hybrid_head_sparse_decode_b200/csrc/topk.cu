@@ -467,13 +467,16 @@ cudaError_t launch_tc(const TopkParams& p, const CombineParams& cp, cudaStream_t
 
 template <typename T, int D>
 cudaError_t launch_tc_d(const TopkParams& p, const CombineParams& cp, cudaStream_t st) {
-  // 16 CTAs per head when the GPU can hold such clusters and the heads' CTAs
-  // fit one wave (two CTAs per SM); else 8, so that many heads (a layer of
-  // retrieval heads) are selected in one wave instead of two
+  // 16 CTAs per head when the rows are long (more than 32768 logits), the GPU
+  // can hold such clusters and the heads' CTAs fit one wave (two CTAs per SM);
+  // else 8: many heads (a layer of retrieval heads) are then selected in one
+  // wave instead of two, and short rows need fewer histogram exchanges
   const long long ctas16 = 16LL * p.B * p.nheads;
   const bool one_wave = p.sms <= 0 || ctas16 <= 2LL * p.sms;
-  return one_wave && cluster16_ok<T, D>(p.N_max, st) ? launch_tc<16, T, D>(p, cp, st)
-                                                     : launch_tc<8, T, D>(p, cp, st);
+  const bool long_rows = p.N_max > 32768;
+  return long_rows && one_wave && cluster16_ok<T, D>(p.N_max, st)
+             ? launch_tc<16, T, D>(p, cp, st)
+             : launch_tc<8, T, D>(p, cp, st);
 }
 
 }  // namespace

@@ -246,3 +246,21 @@ def test_profiler_span_mode():
         torch.cuda.synchronize()
     kinds = [k for k, _ in pl.records]
     assert kinds.count("attn") == 4 and "attn_span" not in kinds
+
+
+@pytest.mark.parametrize("shape", [(8, 8, 128, torch.bfloat16), (16, 2, 128, torch.bfloat16),
+                                   (8, 2, 64, torch.bfloat16), (8, 1, 64, torch.float32)],
+                         ids=["G1", "G8", "bf16-d64", "fp32-G8-d64"])
+def test_stack_other_group_sizes(shape):
+    """The overlapped stack (tail combine, group ordering) with each attention
+    instantiation the other stack tests do not reach: one query head per KV
+    head, eight, and bf16 with d = 64; every layer teacher-forced."""
+    Hq, Hkv, d, dt = shape
+    prob = inputs.make_stack(5, 2, Hq, Hkv, d, 2500, dtype=dt, seed=4601, seqlens=[2500, 1100],
+                             k_frac=0.3, n_planted=8, n_extra_retrieval=6)
+    out, idx_final, idx_layers = run_stack(prob)
+    rep = SetReport()
+    for l in range(prob.shape[0]):
+        teacher_forced_layer(prob, l, out, idx_layers, rep)
+    assert not rep.failures, rep.failures[:5]
+    assert torch.equal(idx_final, idx_layers[-1])
