@@ -264,3 +264,27 @@ def test_stack_other_group_sizes(shape):
         teacher_forced_layer(prob, l, out, idx_layers, rep)
     assert not rep.failures, rep.failures[:5]
     assert torch.equal(idx_final, idx_layers[-1])
+
+
+def test_stack_device_errors_are_reported_not_trapped():
+    """A sequence length past N_max and a budget below 1, in a stack: the
+    kernels clamp them, flag them in the workspace and return; the next call on
+    the same workspace with good inputs reports no error."""
+    prob = inputs.make_stack(3, 2, 8, 2, 128, 1000, seed=4801, seqlens=[1000, 600], k_fixed=300,
+                             n_extra_retrieval=2)
+    L, B, Hq, Hkv, d, N_max = prob.shape
+    q = prob.q.to(DEV)
+    kc = [t.to(DEV) for t in prob.k_caches]
+    vc = [t.to(DEV) for t in prob.v_caches]
+    ws = ops.alloc_workspace(B, Hq, Hkv, d, N_max, prob.k, q.dtype)
+    bad_sl = torch.tensor([1000, 5000], dtype=torch.int32, device=DEV)
+    bad_kb = torch.tensor([300, 0], dtype=torch.int32, device=DEV)
+    out, _, _ = ops.decode_stack(q, kc, vc, bad_sl, prob.roles, prob.k, k_per_seq=bad_kb,
+                                 workspace=ws)
+    st, bits = ops.check_device_error(ws)
+    assert st == N.ERR_BAD_INDEX and bits & 2 and bits & 4, (st, bits)
+    assert torch.isfinite(out.float()).all()
+    ops.decode_stack(q, kc, vc, prob.seqlens.to(DEV), prob.roles, prob.k,
+                     k_per_seq=prob.k_per_seq.to(DEV), workspace=ws)
+    st, bits = ops.check_device_error(ws)
+    assert st == N.OK, (st, bits)
