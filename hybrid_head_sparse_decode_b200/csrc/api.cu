@@ -150,8 +150,8 @@ PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
 }
 
 // LYCHEE_NO_TMA_GATHER=1 in the environment (read once) makes every sparse row
-// gather use 16-byte copies, the path taken when no tensor map can describe the
-// cache; for testing that path.
+// gather of fp32 caches use 16-byte copies, the path taken when no tensor map
+// can describe the cache; for testing that path.
 bool tma_gathers_disabled() {
   static const bool off = [] {
     const char* v = std::getenv("LYCHEE_NO_TMA_GATHER");
@@ -200,6 +200,23 @@ bool encode_row_map(CUtensorMap* m, const void* base, const lychee_shape* s) {
       s->dtype == LYCHEE_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32;
   return enc(m, dt, 2, const_cast<void*>(base), dims, strides, box, estr,
              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// bf16 V cache [B, Hkv, N_max, d] as a 3-D tensor (d, N_max, B * Hkv), boxes 64
+// elements wide and `rows` high with a 128-byte swizzle: the form in which the
+// attention kernel's tensor-core consumers take dense V tiles.  Rows past N_max
+// read as zero.  False when the driver offers no encoder or refuses the map.
+bool encode_v_tile_map(CUtensorMap* m, const void* base, const lychee_shape* s, int rows) {
+  PFN_cuTensorMapEncodeTiled_v12000 enc = tensor_map_encoder();
+  if (!enc) return false;
+  const cuuint64_t dims[3] = {(cuuint64_t)s->d, (cuuint64_t)s->N_max,
+                              (cuuint64_t)s->B * (cuuint64_t)s->Hkv};
+  const cuuint64_t strides[2] = {(cuuint64_t)s->d * 2, (cuuint64_t)s->N_max * s->d * 2};
+  const cuuint32_t box[3] = {64u, (cuuint32_t)rows, 1u};
+  const cuuint32_t estr[3] = {1u, 1u, 1u};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box,
+             estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
@@ -380,6 +397,18 @@ lychee_status run_layer(const Ctx& c, const void* q, const void* kc, const void*
     if (role[h] == LYCHEE_ROLE_RETRIEVAL) rheads[nr++] = (uint8_t)h;
     else sheads[ns++] = (uint8_t)h;
   }
+  // the cache's tensor maps first: a map the driver refuses fails the call
+  // before anything of the layer is launched
+  AttnParams ap{};
+  if (s->dtype == LYCHEE_BF16) {
+    // dense V tiles through swizzled boxes (sparse rows: 16-byte copies)
+    if (!(encode_v_tile_map(&ap.tmv_tile, vc, s, attn_tile_rows(s->dtype, s->d)) &&
+          encode_v_tile_map(&ap.tmv_rest, vc, s, 16)))
+      return LYCHEE_ERR_CUDA;
+  } else {
+    ap.gather_tma = !tma_gathers_disabled() && encode_row_map(&ap.tmk, kc, s) &&
+                     encode_row_map(&ap.tmv, vc, s) ? 1 : 0;
+  }
   cudaError_t e = cudaSuccess;
   if (plan.build_bits && ns > 0) {
     BuildBitsParams bp{};
@@ -395,7 +424,6 @@ lychee_status run_layer(const Ctx& c, const void* q, const void* kc, const void*
     e = timed(kKindBuildBits, c.st, [&] { return launch_build_bits(bp, c.st); });
     if (e != cudaSuccess) return LYCHEE_ERR_CUDA;
   }
-  AttnParams ap{};
   ap.q = q; ap.k = kc; ap.v = vc;
   ap.seqlens = seqlens;
   ap.bitmaps = bitmaps;
@@ -432,8 +460,6 @@ lychee_status run_layer(const Ctx& c, const void* q, const void* kc, const void*
   }
   ap.wait_ns = attn_wait_limit_ns();
   ap.withhold_first = attn_withhold_first_item() ? 1 : 0;
-  ap.gather_tma = !tma_gathers_disabled() && encode_row_map(&ap.tmk, kc, s) &&
-                   encode_row_map(&ap.tmv, vc, s) ? 1 : 0;
   if (plan.span_start) span_mark(false, c.st);
   e = timed(kKindAttn, c.st, [&] { return launch_attn(ap, s->dtype, s->d, G, c.sms, c.st); });
   if (e != cudaSuccess) return LYCHEE_ERR_CUDA;

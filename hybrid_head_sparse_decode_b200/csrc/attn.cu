@@ -24,19 +24,24 @@
 //     next item is built while the current one streams and is consumed.
 //   * streaming warps move each built item through a ring of shared-memory
 //     stages in tiles of TT rows of R.  A dense tile (consecutive positions)
-//     arrives as two 1-D bulk copies (cp.async.bulk) of its K rows and V rows,
-//     issued by the first streaming warp; a sparse tile is gathered row by row
-//     over two paths at once: part of its rows as TMA tile::gather4 copies
-//     (four rows each, through a tensor map over the cache rows) issued by the
-//     first streaming warp, the rest as 16-byte cp.async by the other streaming
-//     warps (whole 32-byte sectors either way).  No copy uses multicast.
+//     arrives as a 1-D bulk copy (cp.async.bulk) of its K rows and, for bf16
+//     caches, TMA tiled loads of its V rows (one box of 64 dimensions per
+//     128-byte half row, 128-byte swizzle; fp32 caches: another 1-D bulk copy),
+//     issued by the first streaming warp.  A sparse tile is gathered row by
+//     row: for bf16 caches by 16-byte cp.async spread over every streaming
+//     warp, V rows written into the same swizzled layout; for fp32 caches over
+//     two paths at once, part of the rows as TMA tile::gather4 copies (four
+//     rows each, through a tensor map over the cache rows) issued by the first
+//     streaming warp, the rest as 16-byte cp.async by the other streaming
+//     warps.  Whole 32-byte sectors either way; no copy uses multicast.
 //   * NW consumer warps, in one of two forms.
 //     - bf16 caches (consumer_loop_mma): a warp takes whole slabs of 16 rows
 //       and serves every head of the group on them at once on the tensor cores
 //       (mma.sync m16n8k16, bf16 operands, fp32 accumulation): S^T = K q^T for
 //       the slab, scores of rows a head does not use set to -inf from the
 //       heads' membership words, an online softmax per head with a lazy
-//       maximum, O^T += V^T P with P rounded to bf16.  A row of the union
+//       maximum, O^T += V^T P with P rounded to bf16 and V^T's fragments read
+//       straight from the swizzled V tile by transposing ldmatrix.  A row of the union
 //       costs the same few instructions whichever heads use it, so the warps
 //       keep pace with HBM; the arithmetic is a skinny GEMM (at most 8 heads
 //       wide) that the warp-level MMA serves without any staging.
@@ -96,16 +101,13 @@ constexpr int ilp_of() {
 constexpr int kProdRegs = LYCHEE_ATTN_PROD_REGS;
 constexpr int kConsRegs = LYCHEE_ATTN_CONS_REGS;
 
-// Sparse tiles take two copy paths at once: the first LYCHEE_ATTN_TMA_ROWS/16 of
-// a tile's rows as TMA tile::gather4 copies issued by the first streaming warp,
-// the rest as 16-byte cp.async by the other streaming warps (each path alone
-// caps below HBM bandwidth).  0: cp.async only.
+// fp32 caches: sparse tiles take two copy paths at once, the first
+// LYCHEE_ATTN_TMA_ROWS/16 of a tile's rows as TMA tile::gather4 copies issued by
+// the first streaming warp, the rest as 16-byte cp.async by the other streaming
+// warps.  0: cp.async only (always so with bf16 caches, whose V rows land in
+// the swizzled layout).
 #ifndef LYCHEE_ATTN_TMA_ROWS
 #define LYCHEE_ATTN_TMA_ROWS 8
-#endif
-// ... with the tensor-core consumers (more streaming warps share the 16-byte copies)
-#ifndef LYCHEE_ATTN_TMA_ROWS_MMA
-#define LYCHEE_ATTN_TMA_ROWS_MMA 6
 #endif
 // bf16 caches: consumer warps contract on the tensor cores (mma.sync, see
 // consumer_loop_mma); 0: the fp32-FMA consumer for every type.
@@ -164,7 +166,15 @@ struct AttnCfg {
   static_assert(CPL >= 2 && DL % E == 0 && CPL % 2 == 0, "lane mapping");
   static_assert(TT % kPairsPerBatch == 0 && TT % 4 == 0 && TT <= 255, "tile rows");
   static constexpr bool MMA = mma_path<T>();
-  static constexpr int TMA_ROWS = MMA ? LYCHEE_ATTN_TMA_ROWS_MMA : LYCHEE_ATTN_TMA_ROWS;
+  // tensor-core consumers: V tiles in swizzled planes (below), sparse rows by
+  // 16-byte copies only
+  static constexpr bool VSW = MMA;
+  static constexpr int TMA_ROWS = MMA ? 0 : LYCHEE_ATTN_TMA_ROWS;
+  static constexpr int NPL = ROWB / 128;          // V planes (VSW): 64 dimensions each
+  static constexpr int PLANE = TT * 128;          // bytes per plane of a stage
+  static_assert(!VSW || (ROWB % 128 == 0 && TT % 16 == 0 && !LYCHEE_ATTN_RUNS),
+                "swizzled V planes: whole 128-byte half rows, 16-row boxes");
+  static constexpr int ALIGN = VSW ? 1024 : 128;  // the 128-byte swizzle repeats every 1024 bytes
   static_assert(MMA ? (G <= 8 && NW <= kPartSlots && TT % 16 == 0)
                     : (G <= NW && NW <= kPartSlots && NW <= 16),
                 "warps per head fit the partial slots; tensor-core slabs of 16 rows");
@@ -187,7 +197,7 @@ struct AttnCfg {
   static_assert(IB_LPOS % 16 == 0, "positions read four at a time");
   static constexpr int IBUF = IB_LPOS + kChunk * 4;
 
-  // shared memory layout (byte offsets from a 128-byte aligned base)
+  // shared memory layout (byte offsets from an ALIGN-byte aligned base)
   static constexpr int kStageKV = TT * ROWB;
   static constexpr int kQBytes = G * D * (int)sizeof(T);
   static constexpr int QSTRIDE = (kQBytes + 127) / 128 * 128;
@@ -199,8 +209,18 @@ struct AttnCfg {
   static constexpr int OFF_CUM = OFF_ITEM + 2 * IBUF;
   static constexpr int OFF_BAR = (OFF_CUM + (kMaxBatchCompact + 1) * 4 + 15) / 16 * 16;
   static constexpr int NBAR = 2 * STAGES + 4;     // full, empty, ready[2], freeb[2]
-  static constexpr int SMEM = OFF_BAR + NBAR * 8 + 128;   // + alignment slack
+  static constexpr int SMEM = OFF_BAR + NBAR * 8 + ALIGN;   // + alignment slack
+  static_assert(!VSW || (OFF_V % 1024 == 0 && kStageKV % 1024 == 0 && PLANE % 1024 == 0),
+                "V planes on 1024-byte boundaries");
 };
+
+// Byte offset of 16-byte piece `piece` of V row `row` in a stage with swizzled
+// V planes: plane piece / 8, the row's 128-byte line, the piece's slot within
+// the line XORed with the row's position in its group of eight (the layout a
+// TMA load with a 128-byte swizzle writes at a 1024-byte aligned address).
+__device__ __forceinline__ int vsw_offset(int row, int piece, int plane_bytes) {
+  return (piece >> 3) * plane_bytes + row * 128 + (((piece & 7) ^ (row & 7)) << 4);
+}
 
 // Item decode shared by the builder: item -> (b, c, g).  Items come in two
 // classes: first those of the groups gorder[0 .. n_indep), then those of the
@@ -393,7 +413,8 @@ __global__ void __launch_bounds__((NW + NP) * 32, 1)
   constexpr int ROWB = C::ROWB, PPR = C::PPR, RPI = C::RPI, E = C::E, NS = C::NS;
 
   extern __shared__ __align__(128) unsigned char smem_raw[];
-  unsigned char* smem = smem_raw + ((128u - (smem_u32(smem_raw) & 127u)) & 127u);
+  unsigned char* smem =
+      smem_raw + (((uint32_t)C::ALIGN - (smem_u32(smem_raw) & (C::ALIGN - 1u))) & (C::ALIGN - 1u));
   int4* info = reinterpret_cast<int4*>(smem + C::OFF_INFO);
   int* cum = reinterpret_cast<int*>(smem + C::OFF_CUM);
   // per stage: full (q and K/V rows landed; one arrival per streaming warp),
@@ -709,7 +730,8 @@ __global__ void __launch_bounds__((NW + NP) * 32, 1)
                 const size_t src = (size_t)lpos[t0 + row] * D + piece * E;
                 const int dst = row * ROWB + piece * 16;
                 cp_async16(kd + dst, kbase + src);
-                cp_async16(vd + dst, vbase + src);
+                if constexpr (C::VSW) cp_async16(vd + vsw_offset(row, piece, C::PLANE), vbase + src);
+                else cp_async16(vd + dst, vbase + src);
               }
             }
           }
@@ -718,7 +740,11 @@ __global__ void __launch_bounds__((NW + NP) * 32, 1)
         __syncwarp();
         if (lane == 0 && sw != 0) mbar_arrive(&full[s]);
         if (lane == 0 && sw == 0) {
-          const uint32_t bytes = ((flags & kDense) ? 2u * (uint32_t)nrows * ROWB : 0u) +
+          // swizzled V planes: a dense tile's V comes as whole boxes (TT rows,
+          // or 16-row boxes covering a shorter tile)
+          const uint32_t vrows = !C::VSW ? (uint32_t)nrows
+                                         : (nrows == TT ? (uint32_t)TT : (uint32_t)((nrows + 15) & ~15));
+          const uint32_t bytes = ((flags & kDense) ? ((uint32_t)nrows + vrows) * ROWB : 0u) +
                                  ((flags & kFirst) ? (uint32_t)C::kQBytes : 0u) +
                                  (LYCHEE_ATTN_RUNS ? 2u * (uint32_t)nt * ROWB
                                                    : 2u * (uint32_t)ngrp * 4u * ROWB);
@@ -733,10 +759,23 @@ __global__ void __launch_bounds__((NW + NP) * 32, 1)
           if (flags & kDense) {
             const size_t off = (size_t)(p0 + t0) * D;
             bulk_g2s(kd, kbase + off, (uint32_t)nrows * ROWB, &full[s], pol);
-            bulk_g2s(vd, vbase + off, (uint32_t)nrows * ROWB, &full[s], pol);
+            if constexpr (C::VSW) {
+#pragma unroll
+              for (int pl = 0; pl < C::NPL; ++pl) {
+                unsigned char* vp = vd + pl * C::PLANE;
+                if (nrows == TT) {
+                  tma_load_3d(vp, &p.tmv_tile, 64 * pl, p0 + t0, unit, &full[s], pol);
+                } else {
+                  for (int i = 0; i < nrows; i += 16)
+                    tma_load_3d(vp + i * 128, &p.tmv_rest, 64 * pl, p0 + t0 + i, unit, &full[s], pol);
+                }
+              }
+            } else {
+              bulk_g2s(vd, vbase + off, (uint32_t)nrows * ROWB, &full[s], pol);
+            }
           }
         }
-        if (LYCHEE_ATTN_RUNS && nt > 0 && sw == 0) {
+        if (!C::VSW && LYCHEE_ATTN_RUNS && nt > 0 && sw == 0) {
           // rows [0, nt) as runs of consecutive positions, one bulk copy of K
           // and one of V per run (rows of a run are adjacent in the tile too)
           for (int i0 = 0; i0 < nt; i0 += 32) {
@@ -753,7 +792,7 @@ __global__ void __launch_bounds__((NW + NP) * 32, 1)
             }
           }
         }
-        if (!LYCHEE_ATTN_RUNS && ngrp > 0 && sw == 0) {
+        if (!C::VSW && !LYCHEE_ATTN_RUNS && ngrp > 0 && sw == 0) {
           // four rows per copy; a padded group repeats the range's last row
           const int last = lpos[t0 + nt - 1];
           for (int gi = lane; gi < ngrp; gi += 32) {
@@ -1070,9 +1109,6 @@ __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
   const __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
   return *reinterpret_cast<const uint32_t*>(&v);
 }
-__device__ __forceinline__ uint32_t word_of(const uint4& v, int i) {
-  return i == 0 ? v.x : i == 1 ? v.y : i == 2 ? v.z : v.w;
-}
 
 // Consumer warps of attn_kernel for bf16 caches.  A warp takes whole slabs of
 // 16 rows of a tile (slab sigma of an item, counted over its tiles, goes to warp
@@ -1087,8 +1123,10 @@ __device__ __forceinline__ uint32_t word_of(const uint4& v, int i) {
 //   past the tile and padding heads get score -inf; retrieval heads' raw scores go to the logits;
 //   online softmax per head with the lazy maximum;
 //   O^T (d x 8 heads) += V_slab^T . P on the tensor cores, P rounded to bf16
-//   (the weights summed into l are the rounded ones), V and P brought into
-//   fragment layout by 8x8 transposes in registers.
+//   (the weights summed into l are the rounded ones): V^T's fragments come
+//   from the swizzled V tile by transposing ldmatrix (conflict-free: the eight
+//   rows of a matrix sit in eight different 16-byte slots), P's by two 8x8
+//   transposes in registers.
 // At the end of an item each warp writes one partial state per head of the
 // group into its own slot (slot = warp).
 template <typename T, int D, int G, int NW, int NP, int TT, int STAGES>
@@ -1154,7 +1192,7 @@ __device__ __forceinline__ void consumer_loop_mma(const AttnParams& p, unsigned 
     };
     const uint32_t lane_all = (hx < G ? 1u : 0u) | (hy < G ? 2u : 0u);
     const unsigned char* kt = smem + C::OFF_K + s * C::kStageKV + 16 * t;
-    const unsigned char* vt = smem + C::OFF_V + s * C::kStageKV + 16 * t;
+    const uint32_t vt_u32 = smem_u32(smem + C::OFF_V + s * C::kStageKV);
     const int nsl = (nrows + 15) >> 4;
     int j = (warp - (tt * SPT) % NW) % NW;
     if (j < 0) j += NW;
@@ -1177,13 +1215,20 @@ __device__ __forceinline__ void consumer_loop_mma(const AttnParams& p, unsigned 
         mma_16816(sc[(2 * P + 1) & 3], KA[P].z, KB[P].z, KA[P].w, KB[P].w, qf[P].z, qf[P].w);
       }
       // V of the same rows, loaded while the scores finish
-      const unsigned char* va = vt + (vA ? rA : 0) * ROWB;
-      const unsigned char* vb = vt + (vB ? rB : 0) * ROWB;
-      uint4 VA[NPB], VB[NPB];
+      // straight into A fragments of V^T: block m (dimensions 16m .. 16m + 15)
+      // from four 8x8 matrices, lanes 8i .. 8i + 7 addressing matrix i: rows
+      // 8 (i / 2) .. + 7 of the slab, dimensions 16m + 8 (i % 2) .. + 7 (a row
+      // past the tile reads row 0 instead; its weight is 0)
+      uint32_t VF[2 * NPB][4];
+      {
+        const int lr = 16 * j + ((lane >> 4) << 3) + (lane & 7);
+        const int rr = lr < nrows ? lr : 0;
+        const uint32_t ra = vt_u32 + rr * 128;
+        const int hi = (lane >> 3) & 1;
 #pragma unroll
-      for (int P = 0; P < NPB; ++P) {
-        VA[P] = *reinterpret_cast<const uint4*>(va + 64 * P);
-        VB[P] = *reinterpret_cast<const uint4*>(vb + 64 * P);
+        for (int mb = 0; mb < 2 * NPB; ++mb)
+          ldsm_x4_trans(ra + (mb >> 2) * C::PLANE + (((((2 * mb) & 7) + hi) ^ (rr & 7)) << 4),
+                        VF[mb][0], VF[mb][1], VF[mb][2], VF[mb][3]);
       }
       // raw scores: (rA, hx), (rA, hy), (rB, hx), (rB, hy)
       float sv[4];
@@ -1245,16 +1290,8 @@ __device__ __forceinline__ void consumer_loop_mma(const AttnParams& p, unsigned 
       // P as the B operand (rows x heads), then O^T += V^T P per 16 dimensions
       const uint32_t b0 = transpose8x8(pa), b1 = transpose8x8(pb);
 #pragma unroll
-      for (int P = 0; P < NPB; ++P) {
-#pragma unroll
-        for (int jp = 0; jp < 2; ++jp) {
-          const uint32_t x0 = transpose8x8(word_of(VA[P], 2 * jp));
-          const uint32_t x1 = transpose8x8(word_of(VA[P], 2 * jp + 1));
-          const uint32_t y0 = transpose8x8(word_of(VB[P], 2 * jp));
-          const uint32_t y1 = transpose8x8(word_of(VB[P], 2 * jp + 1));
-          mma_16816(o[2 * P + jp], x0, x1, y0, y1, b0, b1);
-        }
-      }
+      for (int mb = 0; mb < 2 * NPB; ++mb)
+        mma_16816(o[mb], VF[mb][0], VF[mb][1], VF[mb][2], VF[mb][3], b0, b1);
     }
     __syncwarp();
     if (lane == 0) mbar_arrive(&empty[s]);
@@ -1278,14 +1315,13 @@ __device__ __forceinline__ void consumer_loop_mma(const AttnParams& p, unsigned 
         const int h = 2 * t + e;
         if (h < G) {
           const size_t ps = ((size_t)(b * p.Hq + h0 + h) * p.nchunk + c) * kPartSlots + warp;
-          float* dst = p.part_acc + ps * D + 8 * (g >> 1) + (g & 1);
+          // block mb: rows g, g + 8 of O^T are dimensions 16 mb + g, + 8
+          float* dst = p.part_acc + ps * D + g;
 #pragma unroll
-          for (int P = 0; P < NPB; ++P)
-#pragma unroll
-            for (int jp = 0; jp < 2; ++jp) {
-              dst[32 * P + 4 * jp] = o[2 * P + jp][e];
-              dst[32 * P + 4 * jp + 2] = o[2 * P + jp][2 + e];
-            }
+          for (int mb = 0; mb < 2 * NPB; ++mb) {
+            dst[16 * mb] = o[mb][e];
+            dst[16 * mb + 8] = o[mb][2 + e];
+          }
           if (g == 0) *reinterpret_cast<float2*>(p.part_ml + ps * 2) = make_float2(m[e], l[e]);
         }
       }
@@ -1384,6 +1420,11 @@ cudaError_t launch_attn_d(const AttnParams& p, int G, int num_sms, cudaStream_t 
 }
 
 }  // namespace
+
+int attn_tile_rows(int dtype, int D) {
+  if (dtype == 0) return D == 64 ? tile_rows<__nv_bfloat16, 64>() : tile_rows<__nv_bfloat16, 128>();
+  return D == 64 ? tile_rows<float, 64>() : tile_rows<float, 128>();
+}
 
 cudaError_t launch_attn(const AttnParams& p, int dtype, int D, int G, int num_sms,
                         cudaStream_t st) {

@@ -167,6 +167,32 @@ __device__ __forceinline__ void tma_gather4(void* dst, const void* tmap, int x, 
       : "memory");
 }
 
+// ---- 3-D tiled load through a tensor map (TMA, no multicast) ----------------------
+// Copies the box at coordinates (x, y, z) (x innermost, x * element size a
+// multiple of 16 bytes) to dst, in the map's shared-memory layout (with a
+// 128-byte swizzle: dst 1024-byte aligned); elements outside the tensor read as
+// zero.  Completion is signalled as the box's bytes on `bar`.
+__device__ __forceinline__ void tma_load_3d(void* dst, const void* tmap, int x, int y, int z,
+                                            uint64_t* bar, uint64_t policy) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint"
+      " [%0], [%1, {%2, %3, %4}], [%5], %6;" ::"r"(smem_u32(dst)),
+      "l"(reinterpret_cast<uint64_t>(tmap)), "r"(x), "r"(y), "r"(z), "r"(smem_u32(bar)),
+      "l"(policy)
+      : "memory");
+}
+
+// ---- four 8x8 matrices of 16-bit elements from shared memory, transposed ------------
+// Lanes 8i .. 8i + 7 give the addresses of the 8 rows (16 bytes each) of matrix
+// i; lane 4r + c receives, of each matrix, the elements at rows 2c and 2c + 1 of
+// column r (the lower half of the register holding row 2c).
+__device__ __forceinline__ void ldsm_x4_trans(uint32_t addr, uint32_t& r0, uint32_t& r1,
+                                              uint32_t& r2, uint32_t& r3) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0, %1, %2, %3}, [%4];"
+               : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
+               : "r"(addr));
+}
+
 // ---- programmatic dependent launch -------------------------------------------------
 // Every kernel of the library lets the next kernel of its stream start launching
 // at once (its CTAs become resident as SMs free up) and, before touching any

@@ -53,16 +53,25 @@ struct AttnParams {
   // the kernel waits for that kernel before it reads them.
   int n_indep;
   uint8_t gorder[128];
-  int gather_tma;           // 1: sparse rows are gathered through tmk / tmv
+  int gather_tma;           // fp32 caches, 1: part of the sparse rows come through tmk / tmv
   unsigned long long wait_ns;  // a pipeline wait gives up (kErrTimeout) after this long
   int withhold_first;       // test only: the builder never announces its first item
   // K and V caches viewed as [B * Hkv * N_max] rows of D elements, box one row
-  // (TMA tile::gather4); valid when gather_tma is 1
+  // (TMA tile::gather4); valid when gather_tma is 1 (fp32 caches)
   alignas(64) CUtensorMap tmk;
   alignas(64) CUtensorMap tmv;
+  // bf16 caches (tensor-core consumers): V viewed as [B * Hkv][N_max][D],
+  // boxes 64 elements wide with a 128-byte swizzle, attn_tile_rows() rows high
+  // (tmv_tile) and 16 rows high (tmv_rest); the dense tiles' V rows come
+  // through these
+  alignas(64) CUtensorMap tmv_tile;
+  alignas(64) CUtensorMap tmv_rest;
 };
 cudaError_t launch_attn(const AttnParams& p, int dtype, int D, int G, int num_sms,
                         cudaStream_t st);
+// Rows per shared-memory tile of the attention kernel for this element type and
+// head dimension.
+int attn_tile_rows(int dtype, int D);
 
 // argsTopK of retrieval heads (topk.cu).
 struct TopkParams {

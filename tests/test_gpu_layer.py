@@ -183,9 +183,10 @@ def test_graph_capture_replays_identically():
 
 
 def test_sparse_row_copies_without_tensor_maps():
-    """The 16-byte-copy gather path (taken when no tensor map can describe the
-    cache) gives the same parity results: rerun a set of layer cases in a fresh
-    process with the row gathers forced onto that path."""
+    """The 16-byte-copy gather path of fp32 caches (taken when no tensor map
+    can describe the cache; bf16 caches always gather that way) gives the same
+    parity results: rerun a set of layer cases in a fresh process with the row
+    gathers forced onto that path."""
     import os
     import subprocess
     import sys
