@@ -203,11 +203,12 @@ bool encode_row_map(CUtensorMap* m, const void* base, const lychee_shape* s) {
              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-// bf16 V cache [B, Hkv, N_max, d] as a 3-D tensor (d, N_max, B * Hkv), boxes 64
-// elements wide and `rows` high with a 128-byte swizzle: the form in which the
-// attention kernel's tensor-core consumers take dense V tiles.  Rows past N_max
-// read as zero.  False when the driver offers no encoder or refuses the map.
-bool encode_v_tile_map(CUtensorMap* m, const void* base, const lychee_shape* s, int rows) {
+// bf16 K or V cache [B, Hkv, N_max, d] as a 3-D tensor (d, N_max, B * Hkv),
+// boxes 64 elements wide and `rows` high with a 128-byte swizzle: the form in
+// which the attention kernel's tensor-core consumers take dense tiles.  Rows
+// past N_max read as zero.  False when the driver offers no encoder or refuses
+// the map.
+bool encode_tile_map(CUtensorMap* m, const void* base, const lychee_shape* s, int rows) {
   PFN_cuTensorMapEncodeTiled_v12000 enc = tensor_map_encoder();
   if (!enc) return false;
   const cuuint64_t dims[3] = {(cuuint64_t)s->d, (cuuint64_t)s->N_max,
@@ -401,9 +402,10 @@ lychee_status run_layer(const Ctx& c, const void* q, const void* kc, const void*
   // before anything of the layer is launched
   AttnParams ap{};
   if (s->dtype == LYCHEE_BF16) {
-    // dense V tiles through swizzled boxes (sparse rows: 16-byte copies)
-    if (!(encode_v_tile_map(&ap.tmv_tile, vc, s, attn_tile_rows(s->dtype, s->d)) &&
-          encode_v_tile_map(&ap.tmv_rest, vc, s, 16)))
+    // dense K / V tiles through swizzled boxes (sparse rows: 16-byte copies)
+    const int tt = attn_tile_rows(s->dtype, s->d);
+    if (!(encode_tile_map(&ap.tmk_tile, kc, s, tt) && encode_tile_map(&ap.tmk_rest, kc, s, 16) &&
+          encode_tile_map(&ap.tmv_tile, vc, s, tt) && encode_tile_map(&ap.tmv_rest, vc, s, 16)))
       return LYCHEE_ERR_CUDA;
   } else {
     ap.gather_tma = !tma_gathers_disabled() && encode_row_map(&ap.tmk, kc, s) &&

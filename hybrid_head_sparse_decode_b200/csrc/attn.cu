@@ -23,26 +23,29 @@
 //     proportional to its rows.  It fills two alternating item buffers, so the
 //     next item is built while the current one streams and is consumed.
 //   * streaming warps move each built item through a ring of shared-memory
-//     stages in tiles of TT rows of R.  A dense tile (consecutive positions)
-//     arrives as a 1-D bulk copy (cp.async.bulk) of its K rows and, for bf16
-//     caches, TMA tiled loads of its V rows (one box of 64 dimensions per
-//     128-byte half row, 128-byte swizzle; fp32 caches: another 1-D bulk copy),
-//     issued by the first streaming warp.  A sparse tile is gathered row by
-//     row: for bf16 caches by 16-byte cp.async spread over every streaming
-//     warp, V rows written into the same swizzled layout; for fp32 caches over
-//     two paths at once, part of the rows as TMA tile::gather4 copies (four
-//     rows each, through a tensor map over the cache rows) issued by the first
-//     streaming warp, the rest as 16-byte cp.async by the other streaming
-//     warps.  Whole 32-byte sectors either way; no copy uses multicast.
+//     stages in tiles of TT rows of R.
+//     - bf16 caches: a stage holds K and V as planes of 128-byte half rows
+//       (64 dimensions each) with a 128-byte swizzle.  A dense tile
+//       (consecutive positions) arrives as TMA tiled loads, one box per plane
+//       of K and of V, issued by the first streaming warp; a sparse tile is
+//       gathered row by row by 16-byte cp.async spread over every streaming
+//       warp, each piece written to its swizzled slot.
+//     - fp32 caches: a stage holds the rows as they are in HBM.  A dense tile
+//       arrives as two 1-D bulk copies (cp.async.bulk); a sparse tile over
+//       two paths at once, part of the rows as TMA tile::gather4 copies (four
+//       rows each, through a tensor map over the cache rows) issued by the
+//       first streaming warp, the rest as 16-byte cp.async by the others.
+//     Whole 32-byte sectors either way; no copy uses multicast.
 //   * NW consumer warps, in one of two forms.
 //     - bf16 caches (consumer_loop_mma): a warp takes whole slabs of 16 rows
 //       and serves every head of the group on them at once on the tensor cores
 //       (mma.sync m16n8k16, bf16 operands, fp32 accumulation): S^T = K q^T for
 //       the slab, scores of rows a head does not use set to -inf from the
 //       heads' membership words, an online softmax per head with a lazy
-//       maximum, O^T += V^T P with P rounded to bf16 and V^T's fragments read
-//       straight from the swizzled V tile by transposing ldmatrix.  A row of the union
-//       costs the same few instructions whichever heads use it, so the warps
+//       maximum, O^T += V^T P with P rounded to bf16; the fragments of K and
+//       of V^T come straight from the swizzled planes by ldmatrix (transposing
+//       for V).  A row of the union costs the same few instructions whichever
+//       heads use it, so the warps
 //       keep pace with HBM; the arithmetic is a skinny GEMM (at most 8 heads
 //       wide) that the warp-level MMA serves without any staging.
 //     - fp32 caches (consumer_loop): during an item each warp serves one head
@@ -166,15 +169,15 @@ struct AttnCfg {
   static_assert(CPL >= 2 && DL % E == 0 && CPL % 2 == 0, "lane mapping");
   static_assert(TT % kPairsPerBatch == 0 && TT % 4 == 0 && TT <= 255, "tile rows");
   static constexpr bool MMA = mma_path<T>();
-  // tensor-core consumers: V tiles in swizzled planes (below), sparse rows by
-  // 16-byte copies only
-  static constexpr bool VSW = MMA;
+  // tensor-core consumers: K and V tiles in swizzled planes (below), sparse
+  // rows by 16-byte copies only
+  static constexpr bool SWZ = MMA;
   static constexpr int TMA_ROWS = MMA ? 0 : LYCHEE_ATTN_TMA_ROWS;
-  static constexpr int NPL = ROWB / 128;          // V planes (VSW): 64 dimensions each
-  static constexpr int PLANE = TT * 128;          // bytes per plane of a stage
-  static_assert(!VSW || (ROWB % 128 == 0 && TT % 16 == 0 && !LYCHEE_ATTN_RUNS),
-                "swizzled V planes: whole 128-byte half rows, 16-row boxes");
-  static constexpr int ALIGN = VSW ? 1024 : 128;  // the 128-byte swizzle repeats every 1024 bytes
+  static constexpr int NPL = ROWB / 128;          // planes (SWZ): 64 dimensions each
+  static constexpr int PLANE = TT * 128;          // bytes per plane of a stage's K or V
+  static_assert(!SWZ || (ROWB % 128 == 0 && TT % 16 == 0 && !LYCHEE_ATTN_RUNS),
+                "swizzled planes: whole 128-byte half rows, 16-row boxes");
+  static constexpr int ALIGN = SWZ ? 1024 : 128;  // the 128-byte swizzle repeats every 1024 bytes
   static_assert(MMA ? (G <= 8 && NW <= kPartSlots && TT % 16 == 0)
                     : (G <= NW && NW <= kPartSlots && NW <= 16),
                 "warps per head fit the partial slots; tensor-core slabs of 16 rows");
@@ -210,15 +213,16 @@ struct AttnCfg {
   static constexpr int OFF_BAR = (OFF_CUM + (kMaxBatchCompact + 1) * 4 + 15) / 16 * 16;
   static constexpr int NBAR = 2 * STAGES + 4;     // full, empty, ready[2], freeb[2]
   static constexpr int SMEM = OFF_BAR + NBAR * 8 + ALIGN;   // + alignment slack
-  static_assert(!VSW || (OFF_V % 1024 == 0 && kStageKV % 1024 == 0 && PLANE % 1024 == 0),
-                "V planes on 1024-byte boundaries");
+  static_assert(!SWZ || (OFF_V % 1024 == 0 && kStageKV % 1024 == 0 && PLANE % 1024 == 0),
+                "planes on 1024-byte boundaries");
 };
 
-// Byte offset of 16-byte piece `piece` of V row `row` in a stage with swizzled
-// V planes: plane piece / 8, the row's 128-byte line, the piece's slot within
-// the line XORed with the row's position in its group of eight (the layout a
-// TMA load with a 128-byte swizzle writes at a 1024-byte aligned address).
-__device__ __forceinline__ int vsw_offset(int row, int piece, int plane_bytes) {
+// Byte offset of 16-byte piece `piece` of K (or V) row `row` in a stage's
+// swizzled planes: plane piece / 8, the row's 128-byte line, the piece's slot
+// within the line XORed with the row's position in its group of eight (the
+// layout a TMA load with a 128-byte swizzle writes at a 1024-byte aligned
+// address).
+__device__ __forceinline__ int swz_offset(int row, int piece, int plane_bytes) {
   return (piece >> 3) * plane_bytes + row * 128 + (((piece & 7) ^ (row & 7)) << 4);
 }
 
@@ -728,10 +732,9 @@ __global__ void __launch_bounds__((NW + NP) * 32, 1)
               const int piece = PPR >= 32 ? pc2 * 32 + lane : lane % PPR;
               if (row < nrows && piece < PPR) {
                 const size_t src = (size_t)lpos[t0 + row] * D + piece * E;
-                const int dst = row * ROWB + piece * 16;
+                const int dst = C::SWZ ? swz_offset(row, piece, C::PLANE) : row * ROWB + piece * 16;
                 cp_async16(kd + dst, kbase + src);
-                if constexpr (C::VSW) cp_async16(vd + vsw_offset(row, piece, C::PLANE), vbase + src);
-                else cp_async16(vd + dst, vbase + src);
+                cp_async16(vd + dst, vbase + src);
               }
             }
           }
@@ -740,11 +743,11 @@ __global__ void __launch_bounds__((NW + NP) * 32, 1)
         __syncwarp();
         if (lane == 0 && sw != 0) mbar_arrive(&full[s]);
         if (lane == 0 && sw == 0) {
-          // swizzled V planes: a dense tile's V comes as whole boxes (TT rows,
-          // or 16-row boxes covering a shorter tile)
-          const uint32_t vrows = !C::VSW ? (uint32_t)nrows
+          // swizzled planes: a dense tile comes as whole boxes (TT rows, or
+          // 16-row boxes covering a shorter tile)
+          const uint32_t drows = !C::SWZ ? (uint32_t)nrows
                                          : (nrows == TT ? (uint32_t)TT : (uint32_t)((nrows + 15) & ~15));
-          const uint32_t bytes = ((flags & kDense) ? ((uint32_t)nrows + vrows) * ROWB : 0u) +
+          const uint32_t bytes = ((flags & kDense) ? 2u * drows * ROWB : 0u) +
                                  ((flags & kFirst) ? (uint32_t)C::kQBytes : 0u) +
                                  (LYCHEE_ATTN_RUNS ? 2u * (uint32_t)nt * ROWB
                                                    : 2u * (uint32_t)ngrp * 4u * ROWB);
@@ -757,25 +760,29 @@ __global__ void __launch_bounds__((NW + NP) * 32, 1)
                      (uint32_t)C::kQBytes, &full[s], pol);
           }
           if (flags & kDense) {
-            const size_t off = (size_t)(p0 + t0) * D;
-            bulk_g2s(kd, kbase + off, (uint32_t)nrows * ROWB, &full[s], pol);
-            if constexpr (C::VSW) {
+            if constexpr (C::SWZ) {
+              // per plane, K then V: one TT-row box, or 16-row boxes
 #pragma unroll
               for (int pl = 0; pl < C::NPL; ++pl) {
-                unsigned char* vp = vd + pl * C::PLANE;
+                const int po = pl * C::PLANE;
                 if (nrows == TT) {
-                  tma_load_3d(vp, &p.tmv_tile, 64 * pl, p0 + t0, unit, &full[s], pol);
+                  tma_load_3d(kd + po, &p.tmk_tile, 64 * pl, p0 + t0, unit, &full[s], pol);
+                  tma_load_3d(vd + po, &p.tmv_tile, 64 * pl, p0 + t0, unit, &full[s], pol);
                 } else {
-                  for (int i = 0; i < nrows; i += 16)
-                    tma_load_3d(vp + i * 128, &p.tmv_rest, 64 * pl, p0 + t0 + i, unit, &full[s], pol);
+                  for (int i = 0; i < nrows; i += 16) {
+                    tma_load_3d(kd + po + i * 128, &p.tmk_rest, 64 * pl, p0 + t0 + i, unit, &full[s], pol);
+                    tma_load_3d(vd + po + i * 128, &p.tmv_rest, 64 * pl, p0 + t0 + i, unit, &full[s], pol);
+                  }
                 }
               }
             } else {
+              const size_t off = (size_t)(p0 + t0) * D;
+              bulk_g2s(kd, kbase + off, (uint32_t)nrows * ROWB, &full[s], pol);
               bulk_g2s(vd, vbase + off, (uint32_t)nrows * ROWB, &full[s], pol);
             }
           }
         }
-        if (!C::VSW && LYCHEE_ATTN_RUNS && nt > 0 && sw == 0) {
+        if (!C::SWZ && LYCHEE_ATTN_RUNS && nt > 0 && sw == 0) {
           // rows [0, nt) as runs of consecutive positions, one bulk copy of K
           // and one of V per run (rows of a run are adjacent in the tile too)
           for (int i0 = 0; i0 < nt; i0 += 32) {
@@ -792,7 +799,7 @@ __global__ void __launch_bounds__((NW + NP) * 32, 1)
             }
           }
         }
-        if (!C::VSW && !LYCHEE_ATTN_RUNS && ngrp > 0 && sw == 0) {
+        if (!C::SWZ && !LYCHEE_ATTN_RUNS && ngrp > 0 && sw == 0) {
           // four rows per copy; a padded group repeats the range's last row
           const int last = lpos[t0 + nt - 1];
           for (int gi = lane; gi < ngrp; gi += 32) {
@@ -1114,19 +1121,16 @@ __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
 // 16 rows of a tile (slab sigma of an item, counted over its tiles, goes to warp
 // sigma mod NW) and serves every head of the group on them at once:
 //   S^T (16 rows x 8 heads; heads >= G are zero columns) = K_slab . q^T on the
-//   tensor cores, bf16 operands and fp32 accumulation; the head dimension is
-//   visited in a fixed permutation (lane t of a 32-dimension block reads
-//   dimensions 8t..8t+7 and feeds them as k = 2t, 2t+1, 2t+8, 2t+9 of two
-//   16-deep steps), the same for K and q, so every K row is read with plain
-//   16-byte loads;
+//   tensor cores, bf16 operands and fp32 accumulation, K's fragments by
+//   ldmatrix from the swizzled K planes, q's from the stage's q rows;
 //   rows a head does not use (the heads' membership words of the item), rows
 //   past the tile and padding heads get score -inf; retrieval heads' raw scores go to the logits;
 //   online softmax per head with the lazy maximum;
 //   O^T (d x 8 heads) += V_slab^T . P on the tensor cores, P rounded to bf16
 //   (the weights summed into l are the rounded ones): V^T's fragments come
-//   from the swizzled V tile by transposing ldmatrix (conflict-free: the eight
-//   rows of a matrix sit in eight different 16-byte slots), P's by two 8x8
-//   transposes in registers.
+//   from the swizzled V planes by transposing ldmatrix, P's by two 8x8
+//   transposes in registers.  Every ldmatrix is conflict-free: the eight rows
+//   of a matrix sit in eight different 16-byte slots.
 // At the end of an item each warp writes one partial state per head of the
 // group into its own slot (slot = warp).
 template <typename T, int D, int G, int NW, int NP, int TT, int STAGES>
@@ -1144,7 +1148,7 @@ __device__ __forceinline__ void consumer_loop_mma(const AttnParams& p, unsigned 
   const float sl = p.scale_log2;
   const float lazy = kLazyLog2 / sl;
 
-  uint4 qf[NPB];                         // q of head g, dimensions 32P + 8t .. + 7
+  uint32_t qb[2 * NPB][2];               // B fragments of q^T: head g, dims 16kk + 2t (+ 8), + 1
   float o[2 * NPB][4];                   // O^T fragments, block 2P + jp
   float m[2], mth[2], msl[2], l[2];      // per lane head (hx, hy)
   uint32_t rm = 0;
@@ -1165,10 +1169,13 @@ __device__ __forceinline__ void consumer_loop_mma(const AttnParams& p, unsigned 
       c = i0.z;
       buf = i1.w & 1;
       rm = (uint32_t)i1.y;
-      const unsigned char* qs = smem + C::OFF_Q + s * C::QSTRIDE + g * ROWB + 16 * t;
+      const uint32_t* qs =
+          reinterpret_cast<const uint32_t*>(smem + C::OFF_Q + s * C::QSTRIDE + g * ROWB) + t;
 #pragma unroll
-      for (int P = 0; P < NPB; ++P)
-        qf[P] = g < G ? *reinterpret_cast<const uint4*>(qs + 64 * P) : make_uint4(0u, 0u, 0u, 0u);
+      for (int kk = 0; kk < 2 * NPB; ++kk) {
+        qb[kk][0] = g < G ? qs[8 * kk] : 0u;
+        qb[kk][1] = g < G ? qs[8 * kk + 4] : 0u;
+      }
 #pragma unroll
       for (int k = 0; k < 2 * NPB; ++k) o[k][0] = o[k][1] = o[k][2] = o[k][3] = 0.f;
 #pragma unroll
@@ -1191,7 +1198,7 @@ __device__ __forceinline__ void consumer_loop_mma(const AttnParams& p, unsigned 
       return ((w.x >> (po & 31)) & 1u) | (((w.y >> (po & 31)) & 1u) << 1);
     };
     const uint32_t lane_all = (hx < G ? 1u : 0u) | (hy < G ? 2u : 0u);
-    const unsigned char* kt = smem + C::OFF_K + s * C::kStageKV + 16 * t;
+    const uint32_t kt_u32 = smem_u32(smem + C::OFF_K + s * C::kStageKV);
     const uint32_t vt_u32 = smem_u32(smem + C::OFF_V + s * C::kStageKV);
     const int nsl = (nrows + 15) >> 4;
     int j = (warp - (tt * SPT) % NW) % NW;
@@ -1199,21 +1206,26 @@ __device__ __forceinline__ void consumer_loop_mma(const AttnParams& p, unsigned 
     for (; j < nsl; j += NW) {
       const int rA = 16 * j + g, rB = rA + 8;
       const bool vA = rA < nrows, vB = rB < nrows;
-      const unsigned char* ka = kt + (vA ? rA : 0) * ROWB;
-      const unsigned char* kb = kt + (vB ? rB : 0) * ROWB;
-      uint4 KA[NPB], KB[NPB];
+      // A fragments of the K slab, block kk (dimensions 16kk .. + 15) from four
+      // 8x8 matrices, lanes 8i .. 8i + 7 addressing matrix i: rows 8 (i % 2)
+      // .. + 7 of the slab, dimensions 16kk + 8 (i / 2) .. + 7 (a row past the
+      // tile reads row 0 instead; its score is masked)
+      uint32_t KF[2 * NPB][4];
+      {
+        const int lr = 16 * j + (((lane >> 3) & 1) << 3) + (lane & 7);
+        const int rr = lr < nrows ? lr : 0;
+        const uint32_t ra = kt_u32 + rr * 128;
+        const int hi = lane >> 4;
 #pragma unroll
-      for (int P = 0; P < NPB; ++P) {
-        KA[P] = *reinterpret_cast<const uint4*>(ka + 64 * P);
-        KB[P] = *reinterpret_cast<const uint4*>(kb + 64 * P);
+        for (int kk = 0; kk < 2 * NPB; ++kk)
+          ldsm_x4(ra + (kk >> 2) * C::PLANE + (((((2 * kk) & 7) + hi) ^ (rr & 7)) << 4),
+                  KF[kk][0], KF[kk][1], KF[kk][2], KF[kk][3]);
       }
       // ---- S^T = K q^T (four accumulation chains)
       float sc[4][4] = {};
 #pragma unroll
-      for (int P = 0; P < NPB; ++P) {
-        mma_16816(sc[(2 * P) & 3], KA[P].x, KB[P].x, KA[P].y, KB[P].y, qf[P].x, qf[P].y);
-        mma_16816(sc[(2 * P + 1) & 3], KA[P].z, KB[P].z, KA[P].w, KB[P].w, qf[P].z, qf[P].w);
-      }
+      for (int kk = 0; kk < 2 * NPB; ++kk)
+        mma_16816(sc[kk & 3], KF[kk][0], KF[kk][1], KF[kk][2], KF[kk][3], qb[kk][0], qb[kk][1]);
       // V of the same rows, loaded while the scores finish
       // straight into A fragments of V^T: block m (dimensions 16m .. 16m + 15)
       // from four 8x8 matrices, lanes 8i .. 8i + 7 addressing matrix i: rows

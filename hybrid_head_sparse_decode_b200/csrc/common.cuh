@@ -182,6 +182,17 @@ __device__ __forceinline__ void tma_load_3d(void* dst, const void* tmap, int x, 
       : "memory");
 }
 
+// ---- four 8x8 matrices of 16-bit elements from shared memory ------------------------
+// Lanes 8i .. 8i + 7 give the addresses of the 8 rows (16 bytes each) of matrix
+// i; lane 4r + c receives, of each matrix, the elements at columns 2c and
+// 2c + 1 of row r.
+__device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2,
+                                        uint32_t& r3) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0, %1, %2, %3}, [%4];"
+               : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
+               : "r"(addr));
+}
+
 // ---- four 8x8 matrices of 16-bit elements from shared memory, transposed ------------
 // Lanes 8i .. 8i + 7 give the addresses of the 8 rows (16 bytes each) of matrix
 // i; lane 4r + c receives, of each matrix, the elements at rows 2c and 2c + 1 of

@@ -60,10 +60,11 @@ struct AttnParams {
   // (TMA tile::gather4); valid when gather_tma is 1 (fp32 caches)
   alignas(64) CUtensorMap tmk;
   alignas(64) CUtensorMap tmv;
-  // bf16 caches (tensor-core consumers): V viewed as [B * Hkv][N_max][D],
+  // bf16 caches (tensor-core consumers): K and V viewed as [B * Hkv][N_max][D],
   // boxes 64 elements wide with a 128-byte swizzle, attn_tile_rows() rows high
-  // (tmv_tile) and 16 rows high (tmv_rest); the dense tiles' V rows come
-  // through these
+  // (*_tile) and 16 rows high (*_rest); the dense tiles come through these
+  alignas(64) CUtensorMap tmk_tile;
+  alignas(64) CUtensorMap tmk_rest;
   alignas(64) CUtensorMap tmv_tile;
   alignas(64) CUtensorMap tmv_rest;
 };

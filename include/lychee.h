@@ -42,7 +42,7 @@
  *     trap: the offending entry is skipped or clamped, a flag is set in the
  *     workspace, and lychee_check_device_error() reports it.
  *   - Device pointers must be 16-byte aligned (q, caches, out, workspace).
- *     bf16 V caches are also described to the driver as TMA tensor maps
+ *     bf16 K and V caches are also described to the driver as TMA tensor maps
  *     (cuTensorMapEncodeTiled) before the attention launch; if the driver
  *     offers no encoder or refuses the map, the call returns LYCHEE_ERR_CUDA
  *     with nothing of that layer launched.
