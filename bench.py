@@ -175,22 +175,17 @@ def make_workload(name, device, seed_offset=0):
 
 
 def describe(name, prob):
-    from hybrid_head_sparse_decode_b200.inputs import StackProblem
-    if isinstance(prob, StackProblem):
-        L, B, Hq, Hkv, d, N = prob.shape
-        return {"workload": name, "layers": L, "B": B, "Hq": Hq, "Hkv": Hkv, "d": d,
-                "N": N, "seqlens": [int(x) for x in prob.seqlens.cpu()], "k": prob.k,
-                "retrieval_heads": int(prob.roles.sum()), "layer0": "all retrieval",
-                "io_dtype": "bf16", "accumulate": "fp32",
-                "precision": "q.K: bf16 products, fp32 sums (tensor cores); softmax fp32; "
-                             "P rounded to bf16 for P.V (tensor cores, fp32 sums), the "
-                             "normaliser summing the same rounded weights",
-                "l2": "no flush: each step reads %.1f GB of K/V (> 126 MB L2)" % (
-                    2 * L * B * Hkv * N * d * 2 / 1e9)}
-    B, Hq, Hkv, d, N = prob.shape
-    return {"workload": name, "layers": 1, "B": B, "Hq": Hq, "Hkv": Hkv, "d": d, "N": N,
-            "k": prob.k, "retrieval_heads": int(prob.role.sum()), "io_dtype": "bf16",
-            "accumulate": "fp32", "l2": "flushed between steps by writing a 256 MB buffer"}
+    """The config object of a stack workload's bench line."""
+    L, B, Hq, Hkv, d, N = prob.shape
+    return {"workload": name, "layers": L, "B": B, "Hq": Hq, "Hkv": Hkv, "d": d,
+            "N": N, "seqlens": [int(x) for x in prob.seqlens.cpu()], "k": prob.k,
+            "retrieval_heads": int(prob.roles.sum()), "layer0": "all retrieval",
+            "io_dtype": "bf16", "accumulate": "fp32",
+            "precision": "q.K: bf16 products, fp32 sums (tensor cores); softmax fp32; "
+                         "P rounded to bf16 for P.V (tensor cores, fp32 sums), the "
+                         "normaliser summing the same rounded weights",
+            "l2": "no flush: each step reads %.1f GB of K/V (> 126 MB L2)" % (
+                2 * L * B * Hkv * N * d * 2 / 1e9)}
 
 
 def select_name(block):
@@ -523,6 +518,14 @@ def layer_rows(prob, all_retrieval):
     return u, lit
 
 
+def flush_l2(buf):
+    """Evict the caches' lines from L2: write a buffer larger than L2, then
+    read it back, so that the dirty lines of the write are written back here
+    and not during the next timed call."""
+    buf.zero_()
+    buf.sum()
+
+
 def time_layer_call(prob, steps, warmup, flush, all_retrieval):
     """CUDA-event times (ms) of the single-layer call, L2 flushed before every
     call, and the attention kernel's own median launch time from the library's
@@ -542,7 +545,7 @@ def time_layer_call(prob, steps, warmup, flush, all_retrieval):
                                workspace=ws)
 
     for _ in range(warmup):
-        flush.zero_()
+        flush_l2(flush)
         call()
     st, bits = ops.check_device_error(ws)
     if st != 0:
@@ -551,7 +554,7 @@ def time_layer_call(prob, steps, warmup, flush, all_retrieval):
     ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
           for _ in range(steps)]
     for e0, e1 in ev:
-        flush.zero_()
+        flush_l2(flush)
         e0.record(stream)
         call()
         e1.record(stream)
@@ -560,7 +563,7 @@ def time_layer_call(prob, steps, warmup, flush, all_retrieval):
     prof = ops.Profile(max_launches=4 * steps + 8)
     with prof:
         for _ in range(steps):
-            flush.zero_()
+            flush_l2(flush)
             call()
         torch.cuda.synchronize()
     attn = sorted(ms for k, ms in prof.records if k == "attn")
@@ -609,7 +612,7 @@ def run_sweep(args, device):
             "higher_is_better": False, "dtype": "bf16", "data": "synthetic (seeded)",
             "config": {"workload": "qwen3_layer_sweep", "Hq": 32, "Hkv": 8, "d": 128,
                        "retrieval_heads": 4, "incoming_sets": "random",
-                       "l2": "flushed before every call by writing a 256 MB buffer",
+                       "l2": "flushed before every call by writing a 256 MB buffer and reading it back (no dirty lines left to write back during the call)",
                        "timed": "the whole layer call (set bitmaps, attention, top-k + "
                                 "combine); attn_* from the attention kernel's own launch"},
             "peak": {"hbm_gbs": peak, "source": peak_kind}, "points": points}
