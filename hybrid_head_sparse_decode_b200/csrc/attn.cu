@@ -1206,6 +1206,9 @@ __device__ __forceinline__ void consumer_loop_mma(const AttnParams& p, unsigned 
     for (; j < nsl; j += NW) {
       const int rA = 16 * j + g, rB = rA + 8;
       const bool vA = rA < nrows, vB = rB < nrows;
+      // which of the lane's heads use its two rows (looked up while K loads)
+      const uint32_t mkA = vA ? (masked ? lane_heads(rA) : lane_all) : 0u;
+      const uint32_t mkB = vB ? (masked ? lane_heads(rB) : lane_all) : 0u;
       // A fragments of the K slab, block kk (dimensions 16kk .. + 15) from four
       // 8x8 matrices, lanes 8i .. 8i + 7 addressing matrix i: rows 8 (i % 2)
       // .. + 7 of the slab, dimensions 16kk + 8 (i / 2) .. + 7 (a row past the
@@ -1258,20 +1261,20 @@ __device__ __forceinline__ void consumer_loop_mma(const AttnParams& p, unsigned 
           }
         }
       }
-      const uint32_t mkA = vA ? (masked ? lane_heads(rA) : lane_all) : 0u;
-      const uint32_t mkB = vB ? (masked ? lane_heads(rB) : lane_all) : 0u;
       sv[0] = (mkA & 1u) ? sv[0] : -INFINITY;
       sv[1] = (mkA & 2u) ? sv[1] : -INFINITY;
       sv[2] = (mkB & 1u) ? sv[2] : -INFINITY;
       sv[3] = (mkB & 2u) ? sv[3] : -INFINITY;
-      // ---- online softmax per head, lazy maximum (warp-uniform branch)
+      // ---- online softmax per head, lazy maximum (warp-uniform branch): a
+      // head's maximum over the slab exceeds its threshold iff one of its
+      // scores does, so the maximum itself is reduced only when it is used
       float mx[2] = {fmaxf(sv[0], sv[2]), fmaxf(sv[1], sv[3])};
-#pragma unroll
-      for (int o2 = 4; o2 < 32; o2 <<= 1) {
-        mx[0] = fmaxf(mx[0], __shfl_xor_sync(kFull, mx[0], o2));
-        mx[1] = fmaxf(mx[1], __shfl_xor_sync(kFull, mx[1], o2));
-      }
       if (__any_sync(kFull, mx[0] > mth[0] || mx[1] > mth[1])) {
+#pragma unroll
+        for (int o2 = 4; o2 < 32; o2 <<= 1) {
+          mx[0] = fmaxf(mx[0], __shfl_xor_sync(kFull, mx[0], o2));
+          mx[1] = fmaxf(mx[1], __shfl_xor_sync(kFull, mx[1], o2));
+        }
         float al[2];
 #pragma unroll
         for (int e = 0; e < 2; ++e) {

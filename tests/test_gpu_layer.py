@@ -89,6 +89,23 @@ def test_random_shapes(case):
     check_layer(prob)
 
 
+@pytest.mark.parametrize("dt", [torch.bfloat16, torch.float32])
+def test_rows_past_the_sequence_are_never_read(dt):
+    """K and V rows at positions n_b .. N_max - 1 hold NaN: no tile, box or
+    gather may bring them into a result.  Ragged sequences whose ends fall
+    inside a 16-row box, N_max not a multiple of 16 (boxes past N_max), dense
+    and sparse-only groups; outputs, logits and sets against the oracle."""
+    B, Hq, Hkv, d, N_max = 3, 8, 2, 128, 1001
+    prob = inputs.make_layer(B, Hq, Hkv, d, N_max, dtype=dt, roles=[0, 1, 0, 0, 0, 0, 0, 0],
+                             seed=1300, seqlens=[1001, 333, 70], k_frac=0.3,
+                             idx_mode="random")
+    for b in range(B):
+        n = int(prob.seqlens[b])
+        prob.k_cache[b, :, n:, :] = float("nan")
+        prob.v_cache[b, :, n:, :] = float("nan")
+    check_layer(prob)
+
+
 def test_sparse_over_all_positions_equals_retrieval():
     B, Hq, Hkv, d, N_max = 1, 4, 1, 128, 3000
     prob = inputs.make_layer(B, Hq, Hkv, d, N_max, roles=[1, 0, 1, 0], seed=7, k_fixed=N_max)
