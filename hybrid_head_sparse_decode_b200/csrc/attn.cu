@@ -88,10 +88,10 @@ constexpr int ilp_of() {
   return D * (int)sizeof(T) > 256 ? 1 : LYCHEE_ATTN_ILP;
 }
 
-// Register split between the warpgroups (setmaxnreg): the producer warpgroup
-// gives registers back, the consumer warpgroups take them.  The block launches
-// with 128 registers per thread (checked on the host before the launch):
-// 4 * 32 * kProdRegs + NW * 32 * kConsRegs must not exceed 512 * 128.
+// Register split between the warpgroups of the fp32-FMA kernel (setmaxnreg):
+// the producer warpgroup gives registers back, the consumer warpgroups take
+// them.  The block launches with 65536 / threads registers per thread (checked
+// on the host before the launch); the split must fit in them.
 #ifndef LYCHEE_ATTN_REGSPLIT
 #define LYCHEE_ATTN_REGSPLIT 1
 #endif
@@ -164,6 +164,15 @@ struct AttnCfg {
   static constexpr int PPR = ROWB / 16;           // 16-byte pieces per row (gathers)
   static constexpr int RPI = PPR >= 32 ? 1 : 32 / PPR;  // rows per gather instruction
   static constexpr int NT = (NW + NP) * 32;
+  // register split (setmaxnreg, fp32-FMA consumers): the block launches with
+  // LREGS registers per thread, the producer warpgroups drop to PREGS, the
+  // consumer ones rise to CREGS
+  static constexpr bool RSPLIT = !mma_path<T>() && ilp_of<T, D>() > 1 && LYCHEE_ATTN_REGSPLIT;
+  static constexpr int LREGS = (65536 / NT) & ~7;
+  static constexpr int PREGS = kProdRegs;
+  static constexpr int CREGS = kConsRegs;
+  static_assert(!RSPLIT || (NW % 4 == 0 && NP % 4 == 0 && NP * 32 * PREGS + NW * 32 * CREGS <= NT * LREGS),
+                "register split: whole warpgroups, within the launch's registers");
   static constexpr int NS = NP - 1;               // streaming warps (all producers but the builder)
   static constexpr int MAXT = (kChunk + TT - 1) / TT;   // tiles per item at most
   static_assert(CPL >= 2 && DL % E == 0 && CPL % 2 == 0, "lane mapping");
@@ -469,13 +478,9 @@ __global__ void __launch_bounds__((NW + NP) * 32, 1)
   }
   __syncthreads();
 
-  constexpr int ILP = ilp_of<T, D>();
-  if constexpr (!C::MMA && ILP > 1 && LYCHEE_ATTN_REGSPLIT) {
-    static_assert(NW % 4 == 0 && NP == 4, "whole warpgroups: NW consumers, 4 producers");
-    static_assert(4 * 32 * kProdRegs + NW * 32 * kConsRegs <= (NW + NP) * 32 * 128,
-                  "register split within the launch's registers");
-    if (warp >= NW) asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kProdRegs));
-    else asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kConsRegs));
+  if constexpr (C::RSPLIT) {
+    if (warp >= NW) asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(C::PREGS));
+    else asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(C::CREGS));
   }
   if (warp == NW + 1) {
     // ------------------------------------------------------------ builder
@@ -827,10 +832,10 @@ __global__ void __launch_bounds__((NW + NP) * 32, 1)
   }
   __syncthreads();
   if (p.t_heads > 0) {
-    if constexpr (!C::MMA && ILP > 1 && LYCHEE_ATTN_REGSPLIT) {
+    if constexpr (C::RSPLIT) {
       // back to the launch's registers per thread in every warp
-      if (warp >= NW) asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(128));
-      else asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(128));
+      if (warp >= NW) asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(C::LREGS));
+      else asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(C::LREGS));
     }
     pdl_wait();   // the previous layer's partial states are complete
     static_assert((C::NT / 32) * (32 / (D / 4)) * (D + 4) * 4 + 16 + window_smem_floats<D>() * 4 <=
@@ -1353,12 +1358,12 @@ cudaError_t launch_attn_t(const AttnParams& p, int num_sms, cudaStream_t st) {
     cudaError_t e =
         cudaFuncSetAttribute(kfn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)C::SMEM);
     if (e != cudaSuccess) return e;
-    if (!C::MMA && ilp_of<T, D>() > 1 && LYCHEE_ATTN_REGSPLIT) {
-      // the register split assumes 128 registers per thread at launch
+    if (C::RSPLIT) {
+      // the register split assumes LREGS registers per thread at launch
       cudaFuncAttributes fa{};
       e = cudaFuncGetAttributes(&fa, kfn);
       if (e != cudaSuccess) return e;
-      if (fa.numRegs != 128) return cudaErrorInvalidConfiguration;
+      if (fa.numRegs != C::LREGS) return cudaErrorInvalidConfiguration;
     }
     return cudaSuccess;
   });
