@@ -316,13 +316,15 @@ struct LayerPlan {
   int lbuf = 0, pbuf = 0;      // logits / partial-state regions of this layer
   bool build_bits = false;     // single layer: incoming index rows -> bitmaps first
   bool write_bits = false;     // stack: the retrieval heads' sets go to the bitmaps
-  bool fused_combine = true;   // single layer: the combine shares the selection launch
+  bool fused_combine = true;   // the combine shares the selection launch (single layer,
+                               // a stack's last layer)
   const uint8_t* prev_role = nullptr;   // stack: the previous layer's roles (null: none)
   int tail_pbuf = -1;          // stack: partial region of the previous layer, combined
   void* tail_out = nullptr;    //   by this layer's attention CTAs into tail_out
   bool span_start = false;     // profiler span mode: the stack's first / last
   bool span_end = false;       //   attention launch
-  WindowParams win{};          // this layer's window branch (single layer; k null: none)
+  WindowParams win{};          // this layer's window branch, combined with fused_combine
+                               // (k null: none)
   WindowParams tail_win{};     // the previous layer's window branch (stack)
 };
 
@@ -376,8 +378,9 @@ int group_order(const uint8_t* role, const uint8_t* prev_role, int Hq, int Hkv, 
 // plan.write_bits) the sets of retrieval heads out.  The single-layer call
 // (build_bits, fused_combine) waits for the previous kernel before the first
 // work item; in a stack the attention kernel starts on the groups whose sets
-// are final while the previous layer's selection still runs, combines the
-// layer before in its tail, and the selection launch holds no combine.
+// are final while the previous layer's selection still runs and combines the
+// layer before in its tail; only the last layer's selection launch holds a
+// combine.
 lychee_status run_layer(const Ctx& c, const void* q, const void* kc, const void* vc,
                         const int32_t* seqlens, const int32_t* k_per_seq, const uint8_t* role,
                         const int32_t* idx_in, void* out, int32_t* idx_out,
@@ -515,26 +518,6 @@ lychee_status run_layer(const Ctx& c, const void* q, const void* kc, const void*
   return LYCHEE_OK;
 }
 
-// The combine of one layer on its own launch (the stack's last layer).
-lychee_status combine_layer(const Ctx& c, int pbuf, const int32_t* seqlens, void* out,
-                            const WindowParams& win) {
-  const lychee_shape* s = c.s;
-  CombineParams cp{};
-  cp.part_ml = reinterpret_cast<const float*>(c.ws + c.L.part_ml[pbuf]);
-  cp.part_acc = reinterpret_cast<const float*>(c.ws + c.L.part_acc[pbuf]);
-  cp.part_n = reinterpret_cast<const int32_t*>(c.ws + c.L.part_n[pbuf]);
-  cp.seqlens = seqlens;
-  cp.out = out;
-  cp.err = &c.hdr()->err;
-  cp.B = s->B; cp.Hq = s->Hq; cp.N_max = s->N_max; cp.nchunk = c.L.nchunk;
-  cp.chunk = pick_chunk(s, c.sms);
-  cp.scale_log2 = (float)(1.4426950408889634 / std::sqrt((double)s->d));
-  cp.win = win;
-  const cudaError_t e =
-      timed(kKindCombine, c.st, [&] { return launch_combine(cp, s->dtype, s->d, c.st); });
-  return e == cudaSuccess ? LYCHEE_OK : LYCHEE_ERR_CUDA;
-}
-
 lychee_status export_sets(const Ctx& c, const int32_t* seqlens, int32_t* idx) {
   ExportParams xp{};
   xp.bitmaps = reinterpret_cast<const uint32_t*>(c.ws + c.L.bitmaps);
@@ -645,7 +628,10 @@ lychee_status stack_impl(const lychee_shape* s, int32_t L, const void* q,
     plan.lbuf = l % kLogitBufs;
     plan.pbuf = l % kPartBufs;
     plan.write_bits = true;
-    plan.fused_combine = false;
+    // every layer but the last is combined by the next layer's attention; the
+    // last one's combine shares its selection launch
+    plan.fused_combine = l == L - 1;
+    if (plan.fused_combine) plan.win = win_of(l);
     plan.span_start = l == 0;
     plan.span_end = l == L - 1;
     if (l > 0) {
@@ -655,16 +641,14 @@ lychee_status stack_impl(const lychee_shape* s, int32_t L, const void* q,
       plan.tail_win = win_of(l - 1);
     }
     st = run_layer(c, q_of(l), k_caches[l], v_caches[l], seqlens, k_per_seq,
-                   head_role + (size_t)l * s->Hq, nullptr, nullptr, nullptr, plan);
+                   head_role + (size_t)l * s->Hq, nullptr, plan.fused_combine ? out_of(l) : nullptr,
+                   nullptr, plan);
     if (st != LYCHEE_OK) return st;
     if (idx_layers) {
       st = export_sets(c, seqlens, idx_layers + (size_t)l * s->B * s->Hq * s->k);
       if (st != LYCHEE_OK) return st;
     }
   }
-  // the last layer's output (every other layer was combined by the next one)
-  st = combine_layer(c, (L - 1) % kPartBufs, seqlens, out_of(L - 1), win_of(L - 1));
-  if (st != LYCHEE_OK) return st;
   return export_sets(c, seqlens, idx_final);
 }
 

@@ -95,21 +95,26 @@ __global__ void __launch_bounds__(kThreads) build_bits_kernel(const __grid_const
 }
 
 // Bitmaps -> index rows for every head: ascending positions, -1 padded to k.
-// One CTA of kExportThreads per (sequence, head).  Each warp owns a contiguous
-// run of the row's words; the members before its run come from a CTA-wide
-// scan of the warps' member counts.  The warp then takes its words 32 at a
-// time, one per lane, and emits them word by word: the members of one word
-// are written by the lanes of their bits, to consecutive slots, so every store
-// instruction writes one contiguous piece of the output row.
-constexpr int kExportThreads = 1024;
-__global__ void __launch_bounds__(kExportThreads) export_kernel(const __grid_constant__ ExportParams p) {
+// A row is cut into parts of kExportWords bitmap words, one CTA per (sequence,
+// head, part), one word per thread.  A CTA counts the members before its part
+// (the popcounts of the row's earlier words), places its own members by a
+// block-wide prefix sum of the words' counts into a shared-memory list (each
+// thread writes its word's members), and copies the list to the row with
+// consecutive threads on consecutive slots.  The CTA holding the row's last
+// word also writes the -1 padding.
+constexpr int kExportWords = 256;
+__global__ void __launch_bounds__(kExportWords) export_kernel(const __grid_constant__ ExportParams p) {
   pdl_launch_dependents();
   pdl_wait();
-  constexpr int kWarps = kExportThreads / 32;
+  constexpr int kWarps = kExportWords / 32;
   __shared__ uint32_t wsum[kWarps];
+  __shared__ uint32_t s_before;
+  __shared__ int32_t list[kExportWords * 32];
   const int bh = blockIdx.x, b = bh / p.Hq;
   const int n = min(max(p.seqlens[b], 1), p.N_max);
   const int words = (n + 31) >> 5;
+  const int w0 = blockIdx.y * kExportWords;
+  if (w0 >= words) return;                           // past this sequence's row
   const uint32_t* row = p.bitmaps + (size_t)bh * p.nwords;
   int32_t* out = p.idx + (size_t)bh * p.k;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -117,43 +122,49 @@ __global__ void __launch_bounds__(kExportThreads) export_kernel(const __grid_con
   auto word = [&](int w) -> uint32_t {
     return w < words ? __ldcg(&row[w]) & (w == words - 1 ? tail : 0xffffffffu) : 0u;
   };
-  const int wpw = (words + kWarps - 1) / kWarps;   // words per warp
-  const int w0 = min(words, warp * wpw), w1 = min(words, w0 + wpw);
-  uint32_t cnt = 0;
-  for (int w = w0 + lane; w < w1; w += 32) cnt += __popc(word(w));
+  // members in the words before this part
+  uint32_t pre = 0;
+  for (int w = tid; w < w0; w += kExportWords) pre += __popc(word(w));
 #pragma unroll
-  for (int o = 16; o > 0; o >>= 1) cnt += __shfl_xor_sync(0xffffffffu, cnt, o);
-  if (lane == 0) wsum[warp] = cnt;
+  for (int o = 16; o > 0; o >>= 1) pre += __shfl_xor_sync(0xffffffffu, pre, o);
+  if (lane == 0) wsum[warp] = pre;
   __syncthreads();
-  uint32_t before = 0, total = 0;
-  for (int i = 0; i < kWarps; ++i) {
-    before += i < warp ? wsum[i] : 0u;
-    total += wsum[i];
+  if (tid == 0) {
+    uint32_t t = 0;
+    for (int i = 0; i < kWarps; ++i) t += wsum[i];
+    s_before = t;
   }
-  uint32_t run = before;                             // members before the next word
-  for (int g0 = w0; g0 < w1; g0 += 32) {
-    const int w = g0 + lane;
-    const uint32_t bits = w < w1 ? word(w) : 0u;
-    const uint32_t c = __popc(bits);
-    uint32_t incl = c;
+  __syncthreads();
+  const uint32_t before = s_before;
+  // this thread's word and its members' place in the part
+  const int w = w0 + tid;
+  uint32_t bits = word(w);
+  const uint32_t c = __popc(bits);
+  uint32_t incl = c;
 #pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      const uint32_t y = __shfl_up_sync(0xffffffffu, incl, o);
-      if (lane >= o) incl += y;
-    }
-    const uint32_t off = run + incl - c;             // first slot of this lane's word
-    const int nw = min(32, w1 - g0);
-    for (int t = 0; t < nw; ++t) {
-      const uint32_t bt = __shfl_sync(0xffffffffu, bits, t);
-      const uint32_t ot = __shfl_sync(0xffffffffu, off, t);
-      if ((bt >> lane) & 1u) {
-        const uint32_t slot = ot + __popc(bt & ((1u << lane) - 1u));
-        if (slot < (uint32_t)p.k) out[slot] = (g0 + t) * 32 + lane;
-      }
-    }
-    run += __shfl_sync(0xffffffffu, incl, 31);
+  for (int o = 1; o < 32; o <<= 1) {
+    const uint32_t y = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += y;
   }
-  for (int t = (int)total + tid; t < p.k; t += kExportThreads) out[t] = -1;
+  __syncthreads();                                   // wsum is reused
+  if (lane == 31) wsum[warp] = incl;
+  __syncthreads();
+  uint32_t wbase = 0, m = 0;
+  for (int i = 0; i < kWarps; ++i) {
+    wbase += i < warp ? wsum[i] : 0u;
+    m += wsum[i];
+  }
+  uint32_t slot = wbase + incl - c;
+  while (bits) {
+    const int j = __ffs(bits) - 1;
+    bits &= bits - 1u;
+    list[slot++] = w * 32 + j;
+  }
+  __syncthreads();
+  for (uint32_t i = tid; i < m; i += kExportWords)
+    if (before + i < (uint32_t)p.k) out[before + i] = list[i];
+  if (w0 + kExportWords >= words)                    // the row's last part: the padding
+    for (int t = (int)(before + m) + tid; t < p.k; t += kExportWords) out[t] = -1;
 }
 
 }  // namespace
@@ -167,8 +178,9 @@ cudaError_t launch_build_bits(const BuildBitsParams& p, cudaStream_t st) {
 }
 
 cudaError_t launch_export(const ExportParams& p, cudaStream_t st) {
-  const cudaError_t e =
-      launch_pdl(export_kernel, dim3((unsigned)(p.B * p.Hq)), dim3(kExportThreads), 0, st, p);
+  const unsigned parts = (unsigned)((p.nwords + kExportWords - 1) / kExportWords);
+  const cudaError_t e = launch_pdl(export_kernel, dim3((unsigned)(p.B * p.Hq), parts),
+                                   dim3(kExportWords), 0, st, p);
   if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
