@@ -15,21 +15,26 @@ constexpr int kThreads = 256;
 constexpr int kEntriesPerCta = 4 * kThreads;   // set entries one build_bits CTA covers
 
 // Index rows of the listed sparse heads -> bitmaps (and, when asked, a bit-exact
-// copy of the rows: a sparse head hands its set on unchanged).  One thread per
-// entry, loads coalesced along the row.  Every bitmap word has exactly one
-// writer, so the row needs no clearing pass and no atomics: the thread holding
-// the first entry of a word ORs that word's entries (at most 32, contiguous in
-// the ascending row) and also writes the empty words between the previous
-// entry's word and its own.  A set ends at its first -1 (or at the row's k-th
-// entry; the budget k_b does not bound what a sparse head reads).  The empty
-// words before the first member and after the last one can be thousands; the
-// CTA holding that entry clears them together after its entries.  An entry
-// outside [0, n_b), not strictly above its predecessor, or after the end of the
-// set sets kErrBadIndex; the row is then not a set and its bitmap is
-// unspecified, but every store still stays inside the row.
+// copy of the rows: a sparse head hands its set on unchanged).  Each warp takes
+// 32 consecutive entries at a time, loads coalesced along the row.  Every
+// bitmap word has exactly one writer, so the row needs no clearing pass and no
+// atomics: the lane holding the first entry of a word (the word's leader)
+// writes it, with the OR of the word's entries among the warp's 32 (a
+// segmented OR over the run of lanes holding that word) and, when the run
+// reaches the warp's last lane, of the entries after them; it also writes the
+// empty words between the previous entry's word and its own.  A set ends at its
+// first -1 (or at the row's k-th entry; the budget k_b does not bound what a
+// sparse head reads).  The empty words before the first member and after the
+// last one can be thousands; the CTA holding that entry clears them together
+// after its entries.  An entry outside [0, n_b), not strictly above its
+// predecessor, or after the end of the set sets kErrBadIndex; the row is then
+// not a set and its bitmap is unspecified, but every store still stays inside
+// the row.
 __global__ void __launch_bounds__(kThreads) build_bits_kernel(const __grid_constant__ BuildBitsParams p) {
   pdl_launch_dependents();
   pdl_wait();
+  constexpr uint32_t kAllLanes = 0xffffffffu;
+  constexpr int kWarps = kThreads / 32;
   // word ranges this CTA clears together: [0] before the first member, [1]
   // after the last (each written by the one thread that finds it)
   __shared__ int s_lo[2], s_hi[2];
@@ -41,39 +46,68 @@ __global__ void __launch_bounds__(kThreads) build_bits_kernel(const __grid_const
   uint32_t* row = p.bitmaps + bh * p.nwords;
   const int words = (n + 31) >> 5;
   const int32_t* idx = p.idx_in + bh * p.k;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int base = blockIdx.x * kEntriesPerCta;
+  constexpr int R = kEntriesPerCta / kThreads;         // chunks of 32 entries per warp
+  // every chunk's entries (and the entry before each chunk) loaded up front
+  int jr[R], pr[R];
 #pragma unroll
-  for (int r = 0; r < kEntriesPerCta / kThreads; ++r) {
-    const int t = base + r * kThreads + threadIdx.x;
-    if (t >= p.k) break;
-    const int j = idx[t];
-    if (p.idx_out) p.idx_out[bh * p.k + t] = j;
-    const int prev = t > 0 ? idx[t - 1] : -1;
-    if (j < 0) {
-      // the set ends at its first -1: the words after the last member (all of
-      // them for an empty set) are cleared below
-      if (t == 0 || prev >= 0) {
-        s_lo[1] = t == 0 ? 0 : (prev >> 5) + 1;
-        s_hi[1] = words;
+  for (int r = 0; r < R; ++r) {
+    const int t = base + (r * kWarps + warp) * 32 + lane;
+    jr[r] = t < p.k ? idx[t] : -1;
+    pr[r] = (lane == 0 && t > 0 && t <= p.k) ? idx[t - 1] : -1;
+  }
+#pragma unroll
+  for (int r = 0; r < R; ++r) {
+    const int t0 = base + (r * kWarps + warp) * 32;
+    if (t0 >= p.k) break;                              // warp-uniform
+    const int t = t0 + lane;
+    const bool in = t < p.k;
+    const int j = jr[r];
+    if (in && p.idx_out) p.idx_out[bh * p.k + t] = j;
+    int prev = __shfl_up_sync(kAllLanes, j, 1);
+    if (lane == 0) prev = pr[r];
+    bool member = false;
+    if (in) {
+      if (j < 0) {
+        // the set ends at its first -1: the words after the last member (all
+        // of them for an empty set) are cleared below
+        if (t == 0 || prev >= 0) {
+          s_lo[1] = t == 0 ? 0 : (prev >> 5) + 1;
+          s_hi[1] = words;
+        }
+      } else if ((t > 0 && prev < 0) || j >= n || j <= prev) {
+        flag_error(p.err, kErrBadIndex);   // after the end, out of range, or not ascending
+      } else {
+        member = true;
       }
-      continue;
     }
-    if (t > 0 && prev < 0) {   // a member after the end of the set
-      flag_error(p.err, kErrBadIndex);
-      continue;
-    }
-    if (j >= n || j <= prev) {
-      flag_error(p.err, kErrBadIndex);
-      continue;
-    }
+    // runs of lanes holding members of one word: a run starts where a lane's
+    // key differs from the previous lane's (every non-member has a key of its own)
     const int w = j >> 5;
-    const int pw = prev >> 5;   // -1 for the first entry (arithmetic shift)
-    if (w != pw) {
-      uint32_t bits = 1u << (j & 31);
-      for (int u = t + 1; u < p.k; ++u) {
-        const int ju = idx[u];
-        if ((ju >> 5) != w || ju <= j) break;
-        bits |= 1u << (ju & 31);
+    const int key = member ? w : -2 - lane;
+    const int key_prev = __shfl_up_sync(kAllLanes, key, 1);
+    const uint32_t starts = __ballot_sync(kAllLanes, lane == 0 || key != key_prev);
+    const uint32_t later = starts & ~((2u << lane) - 1u);   // runs starting after this lane
+    const int run_end = later ? __ffs(later) - 1 : 32;      // first lane past this lane's run
+    uint32_t bits = member ? 1u << (j & 31) : 0u;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const uint32_t y = __shfl_down_sync(kAllLanes, bits, o);
+      if (lane + o < run_end) bits |= y;
+    }
+    const int j_last = __shfl_sync(kAllLanes, j, 31);
+    const int pw = prev >> 5;                          // -1 for the first entry (arithmetic shift)
+    if (member && w != pw) {
+      if (run_end == 32) {
+        // the word's entries may go on past the warp's 32
+        int last = j_last;
+        for (int u = t0 + 32; u < p.k; ++u) {
+          const int ju = idx[u];
+          if ((ju >> 5) != w || ju <= last) break;
+          bits |= 1u << (ju & 31);
+          last = ju;
+        }
       }
       row[w] = bits;
       if (pw < 0) {            // the first member: the words before it, below
@@ -83,7 +117,7 @@ __global__ void __launch_bounds__(kThreads) build_bits_kernel(const __grid_const
         for (int g = pw + 1; g < w; ++g) row[g] = 0u;
       }
     }
-    if (t == p.k - 1) {        // a full row: the words after its last member
+    if (member && t == p.k - 1) {   // a full row: the words after its last member
       s_lo[1] = w + 1;
       s_hi[1] = words;
     }
