@@ -8,7 +8,9 @@ layers of the workload (per layer: hybrid attention, top-k of the retrieval
 heads, combine; the sets chained layer to layer), on seeded synthetic inputs
 already resident in HBM.  The default workload is the Qwen3-8B-shaped 36-layer
 stack at 128K context (19.3 GB of K/V per step, far larger than L2, so no L2
-flush is needed between steps).  Rank 0 prints one JSON line.
+flush is needed between steps).  The timed steps replay the step captured once
+into a CUDA graph; the same steps as direct calls are reported beside them.
+Rank 0 prints one JSON line.
 
 Under torchrun (N > 1) every rank runs an independent replica (its own sequence,
 seeded by rank); there is no collective on the data path.  Ranks meet at a
@@ -279,19 +281,38 @@ def run_lychee(args, rank, world, device):
             torch.distributed.barrier()
 
     stream = torch.cuda.current_stream()
+    # the step captured once into a CUDA graph (the stack's launches, with their
+    # programmatic dependencies) and replayed once per decode step
+    gstream = torch.cuda.Stream()
+    sgraph = torch.cuda.CUDAGraph()
+    with torch.cuda.stream(gstream):
+        with torch.cuda.graph(sgraph, stream=gstream):
+            ops.decode_stack(prob.q, prob.k_caches, prob.v_caches, prob.seqlens, roles, prob.k,
+                             k_per_seq=prob.k_per_seq, out=out, idx_final=fin, workspace=ws,
+                             block=blk, stream=gstream)
+    for _ in range(args.warmup):
+        sgraph.replay()
     t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     sampler = ClockSampler(device.index)
-    # timed region: the steps alone (the reported value)
+    # timed region: the steps alone (the reported value), graph replays
     barrier()
     torch.cuda.synchronize()
     with sampler:
         t0.record(stream)
         for _ in range(args.steps):
-            step()
+            sgraph.replay()
         t1.record(stream)
         torch.cuda.synchronize()
     barrier()
     ms_total = t0.elapsed_time(t1)
+    # the same steps as direct calls of the library (host work per call included)
+    torch.cuda.synchronize()
+    t0.record(stream)
+    for _ in range(args.steps):
+        step()
+    t1.record(stream)
+    torch.cuda.synchronize()
+    direct_ms = max_over_ranks(t0.elapsed_time(t1), world, device) / args.steps
     # the same steps again with every library launch bracketed by CUDA events on
     # its stream: per-kernel durations for the roofline of the attention kernel
     prof = ops.Profile(max_launches=args.steps * (4 * L + 2) + 16)
@@ -300,14 +321,15 @@ def run_lychee(args, rank, world, device):
         for _ in range(args.steps):
             step()
         torch.cuda.synchronize()
-    # per-step spread: an event after every step of another pass of the same steps
+    # per-step spread: an event after every replay of another pass of the same steps
     ev = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps + 1)]
     torch.cuda.synchronize()
     ev[0].record(stream)
     for i in range(args.steps):
-        step()
+        sgraph.replay()
         ev[i + 1].record(stream)
     torch.cuda.synchronize()
+    del sgraph
     per_step = sorted(ev[i].elapsed_time(ev[i + 1]) for i in range(args.steps))
     ms_total = max_over_ranks(ms_total, world, device)
     ms_step = ms_total / args.steps
@@ -481,6 +503,9 @@ def run_lychee(args, rank, world, device):
                              "kernels_ms_per_step": {k: round(v, 4) for k, v in dkinds.items()}},
         "e2e": {"value": round(job_us_per_step(e_ms / args.steps, world), 3), "unit": UNIT,
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+        "timing": "value: the step captured once into a CUDA graph, replayed once per step",
+        "direct_call": {"ms_per_step": round(direct_ms, 5),
+                        "note": "the same steps as direct calls of lychee_decode_stack"},
         "append_kv": {"ms_per_step": round(append_ms, 4), "launches_per_step": L,
                       "note": "the current token's K/V rows into all layers' caches, one launch "
                               "per layer, replayed from a CUDA graph; the step above starts from "
