@@ -122,12 +122,6 @@ constexpr bool mma_path() {
   return LYCHEE_ATTN_MMA && std::is_same<T, __nv_bfloat16>::value;
 }
 
-// 1: the TMA part of a sparse tile goes as 1-D bulk copies of runs of
-// consecutive positions instead of tile::gather4 copies
-#ifndef LYCHEE_ATTN_RUNS
-#define LYCHEE_ATTN_RUNS 0
-#endif
-
 template <typename T>
 struct Vec;
 template <>
@@ -184,7 +178,7 @@ struct AttnCfg {
   static constexpr int TMA_ROWS = MMA ? 0 : LYCHEE_ATTN_TMA_ROWS;
   static constexpr int NPL = ROWB / 128;          // planes (SWZ): 64 dimensions each
   static constexpr int PLANE = TT * 128;          // bytes per plane of a stage's K or V
-  static_assert(!SWZ || (ROWB % 128 == 0 && TT % 16 == 0 && !LYCHEE_ATTN_RUNS),
+  static_assert(!SWZ || (ROWB % 128 == 0 && TT % 16 == 0),
                 "swizzled planes: whole 128-byte half rows, 16-row boxes");
   static constexpr int ALIGN = SWZ ? 1024 : 128;  // the 128-byte swizzle repeats every 1024 bytes
   static_assert(MMA ? (G <= 8 && NW <= kPartSlots && TT % 16 == 0)
@@ -754,8 +748,7 @@ __global__ void __launch_bounds__((NW + NP) * 32, 1)
                                          : (nrows == TT ? (uint32_t)TT : (uint32_t)((nrows + 15) & ~15));
           const uint32_t bytes = ((flags & kDense) ? 2u * drows * ROWB : 0u) +
                                  ((flags & kFirst) ? (uint32_t)C::kQBytes : 0u) +
-                                 (LYCHEE_ATTN_RUNS ? 2u * (uint32_t)nt * ROWB
-                                                   : 2u * (uint32_t)ngrp * 4u * ROWB);
+                                 2u * (uint32_t)ngrp * 4u * ROWB;
           fence_proxy_async_smem();
           if (bytes) mbar_arrive_expect_tx(&full[s], bytes);
           else mbar_arrive(&full[s]);
@@ -787,24 +780,7 @@ __global__ void __launch_bounds__((NW + NP) * 32, 1)
             }
           }
         }
-        if (!C::SWZ && LYCHEE_ATTN_RUNS && nt > 0 && sw == 0) {
-          // rows [0, nt) as runs of consecutive positions, one bulk copy of K
-          // and one of V per run (rows of a run are adjacent in the tile too)
-          for (int i0 = 0; i0 < nt; i0 += 32) {
-            const int i = i0 + lane;
-            if (i < nt) {
-              const int pos = lpos[t0 + i];
-              if (i == 0 || lpos[t0 + i - 1] != pos - 1) {
-                int len = 1;
-                while (i + len < nt && lpos[t0 + i + len] == pos + len) ++len;
-                const size_t off = (size_t)pos * D;
-                bulk_g2s(kd + i * ROWB, kbase + off, (uint32_t)len * ROWB, &full[s], pol);
-                bulk_g2s(vd + i * ROWB, vbase + off, (uint32_t)len * ROWB, &full[s], pol);
-              }
-            }
-          }
-        }
-        if (!C::SWZ && !LYCHEE_ATTN_RUNS && ngrp > 0 && sw == 0) {
+        if (!C::SWZ && ngrp > 0 && sw == 0) {
           // four rows per copy; a padded group repeats the range's last row
           const int last = lpos[t0 + nt - 1];
           for (int gi = lane; gi < ngrp; gi += 32) {
