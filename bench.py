@@ -751,7 +751,7 @@ def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=50)
-    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", default="lychee", choices=["lychee", "reference"])
     ap.add_argument("--workload", default="qwen3_stack_128k")
     ap.add_argument("--no-cpu-baseline", action="store_true")
