@@ -467,10 +467,16 @@ cudaError_t launch_tc(const TopkParams& p, const CombineParams& cp, cudaStream_t
 
 template <typename T, int D>
 cudaError_t launch_tc_d(const TopkParams& p, const CombineParams& cp, cudaStream_t st) {
+  // With the combine in the same launch (a single layer, a stack's last layer):
   // 16 CTAs per head when the rows are long (more than 32768 logits), the GPU
   // can hold such clusters and the heads' CTAs fit one wave (two CTAs per SM);
   // else 8: many heads (a layer of retrieval heads) are then selected in one
-  // wave instead of two, and short rows need fewer histogram exchanges
+  // wave instead of two, and short rows need fewer histogram exchanges.
+  // A selection-only launch (a stack's other layers) always takes 8: it runs
+  // beside the next layer's attention kernel, and a cluster of 8 needs 4 free
+  // SMs at once where one of 16 needs 8 (measured: the 36-layer 128K step is
+  // about 50 us shorter).
+  if (cp.B == 0) return launch_tc<8, T, D>(p, cp, st);
   const long long ctas16 = 16LL * p.B * p.nheads;
   const bool one_wave = p.sms <= 0 || ctas16 <= 2LL * p.sms;
   const bool long_rows = p.N_max > 32768;
