@@ -180,3 +180,36 @@ def test_equal_block_maxima_straddle_the_cut():
     assert np.array_equal(gi[0, 0], oracle.block_select(raw, kb, block, prob.k))
     chosen = sorted({int(x) // block for x in gi[0, 0] if x >= 0} & set(tie))
     assert chosen == tie[:2], (chosen, tie)
+
+
+def test_stack_zero_query_takes_the_lowest_positions():
+    """A stack (its selection-only launches on 8-CTA clusters): with every
+    logit 0, every retrieval head of every layer selects positions 0 .. k_b - 1
+    and every sparse head passes on what it inherits, so every layer's sets are
+    those; a sparse head's output is the mean of its group's V rows over them,
+    a retrieval head's the mean over all n_b rows."""
+    prob = inputs.make_stack(4, 2, 8, 2, 128, 40000, seed=3300, seqlens=[40000, 23457],
+                             k_frac=0.3, n_extra_retrieval=3)
+    L, B, Hq, Hkv, d, N_max = prob.shape
+    q = torch.zeros_like(prob.q).to(DEV)
+    kc = [t.to(DEV) for t in prob.k_caches]
+    vc = [t.to(DEV) for t in prob.v_caches]
+    out, fin, lay = ops.decode_stack(q, kc, vc, prob.seqlens.to(DEV), prob.roles, prob.k,
+                                     k_per_seq=prob.k_per_seq.to(DEV), want_layers=True)
+    torch.cuda.synchronize()
+    lay = lay.cpu().numpy()
+    G = Hq // Hkv
+    for b in range(B):
+        kb = int(prob.meta["kb"][b])
+        want = np.concatenate([np.arange(kb), np.full(prob.k - kb, -1)]).astype(np.int32)
+        for l in range(L):
+            for h in range(Hq):
+                assert np.array_equal(lay[l, b, h], want), (l, b, h)
+            n = int(prob.seqlens[b])
+            mean_set = prob.v_caches[l][b, :, :kb].double().mean(1).numpy()   # [Hkv, d]
+            mean_all = prob.v_caches[l][b, :, :n].double().mean(1).numpy()
+            got = out[l, b].double().cpu().numpy()
+            for h in range(Hq):
+                ref = mean_all if int(prob.roles[l, h]) == N.ROLE_RETRIEVAL else mean_set
+                assert np.abs(got[h] - ref[h // G]).max() <= compare_tol(torch.bfloat16), (l, b, h)
+    assert np.array_equal(fin.cpu().numpy(), lay[-1])
