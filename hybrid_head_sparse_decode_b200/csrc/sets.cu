@@ -40,14 +40,14 @@ __global__ void __launch_bounds__(kThreads) build_bits_kernel(const __grid_const
   __shared__ int s_lo[2], s_hi[2];
   if (threadIdx.x < 2) s_lo[threadIdx.x] = s_hi[threadIdx.x] = 0;
   __syncthreads();
-  const int b = blockIdx.y / p.nheads, h = p.heads[blockIdx.y % p.nheads];
+  const int b = blockIdx.x / p.nheads, h = p.heads[blockIdx.x % p.nheads];
   const int n = min(max(p.seqlens[b], 1), p.N_max);
   const size_t bh = (size_t)b * p.Hq + h;
   uint32_t* row = p.bitmaps + bh * p.nwords;
   const int words = (n + 31) >> 5;
   const int32_t* idx = p.idx_in + bh * p.k;
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  const int base = blockIdx.x * kEntriesPerCta;
+  const int base = blockIdx.y * kEntriesPerCta;
   constexpr int R = kEntriesPerCta / kThreads;         // chunks of 32 entries per warp
   // every chunk's entries (and the entry before each chunk) loaded up front
   int jr[R], pr[R];
@@ -205,7 +205,8 @@ __global__ void __launch_bounds__(kExportWords) export_kernel(const __grid_const
 
 cudaError_t launch_build_bits(const BuildBitsParams& p, cudaStream_t st) {
   if (p.nheads <= 0) return cudaSuccess;
-  const dim3 grid((unsigned)((p.k + kEntriesPerCta - 1) / kEntriesPerCta), (unsigned)(p.B * p.nheads));
+  // (sequence, head) pairs on x (up to 2^31 - 1), parts of the row on y (up to 65535)
+  const dim3 grid((unsigned)(p.B * p.nheads), (unsigned)((p.k + kEntriesPerCta - 1) / kEntriesPerCta));
   const cudaError_t e = launch_pdl(build_bits_kernel, grid, dim3(kThreads), 0, st, p);
   if (e != cudaSuccess) return e;
   return cudaGetLastError();

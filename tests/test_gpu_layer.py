@@ -217,6 +217,33 @@ def test_sparse_row_copies_without_tensor_maps():
     assert r.returncode == 0, r.stdout[-3000:] + r.stderr[-3000:]
 
 
+def test_more_sparse_rows_than_a_grid_column_holds():
+    """More (sequence, sparse head) pairs than 65535 (the limit of a grid's y
+    and z dimensions): the bitmap builder puts them on x.  Outputs against the
+    oracle, pass-through sets bit for bit, the retrieval head's sets checked on
+    a sample of sequences."""
+    B = 9400
+    g = torch.Generator().manual_seed(1401)
+    seqlens = torch.randint(1, 41, (B,), generator=g).tolist()
+    prob = inputs.make_layer(B, 8, 2, 64, 40, roles=[0, 0, 0, 1, 0, 0, 0, 0], seed=1402,
+                             seqlens=seqlens, k_fixed=12, idx_mode="random")
+    assert B * 7 > 65535
+    out, idx_out, logits, st, bits = run_gpu(prob)
+    assert st == N.OK, (st, bits)
+    ref_out, ref_idx, ref_logits = oracle_layer(prob)
+    compare_outputs(out, ref_out, prob.q.dtype)
+    gi = idx_out.cpu().numpy()
+    sparse = [h for h in range(8) if h != 3]
+    assert np.array_equal(gi[:, sparse], prob.idx_in.numpy()[:, sparse])
+    lg = logits.cpu().numpy()
+    rep = SetReport()
+    for b in range(0, B, 97):
+        n = int(prob.seqlens[b])
+        check_set(rep, (b, 3), gi[b, 3], int(prob.meta["kb"][b]), prob.k, ref_logits[b, 3, :n],
+                  gpu_raw=lg[b, 3, :n], d=64)
+    assert not rep.failures, rep.failures[:5]
+
+
 def test_large_batch_item_space():
     """More than 1024 sequences: the attention kernel enumerates every (sequence,
     chunk) pair and skips chunks past n_b instead of keeping per-sequence chunk
