@@ -464,6 +464,12 @@ def run_lychee(args, rank, world, device):
         "config": dict(describe(args.workload, prob),
                        select=select_name(blk)),
         "us_per_layer": round(ms_step * 1e3 / L, 3),
+        # the attention launches of layer 0 (all retrieval heads) and of the
+        # other layers, from the events around every launch (serialised)
+        "attn_us_by_layer": {
+            "layer0_median": round(statistics.median(attn[0::L]) * 1e3, 2) if attn else None,
+            "others_median": round(statistics.median([a for i, a in enumerate(attn) if i % L])
+                                   * 1e3, 2) if attn and L > 1 else None},
         "step_ms_spread": {"p10": round(nearest_rank(per_step, 0.1), 5),
                            "median": round(nearest_rank(per_step, 0.5), 5),
                            "p90": round(nearest_rank(per_step, 0.9), 5),
