@@ -54,10 +54,12 @@
 //       accumulator; eight pairs are in flight per warp.  q.K with packed
 //       fp32x2 FMA and two shuffles to finish the dot product, the same lazy
 //       online softmax per pair slot, P.V on the same lanes and rows.
-//     At the end of an item each warp writes its partial state (m, l, acc[d])
-//     for each head it served to its own slot of the workspace; the combine
-//     kernel merges the warps and chunks in a fixed order, so the result does
-//     not depend on scheduling and no warp waits for another.
+//     At the end of an item the fp32 consumers write each warp's partial state
+//     (m, l, acc[d]) for each head it served to its own slot of the workspace;
+//     the tensor-core consumers first merge their warps' states of each head
+//     in shared memory (a fixed order) and write one.  The combine merges the
+//     states and chunks in a fixed order, so the result does not depend on
+//     scheduling.
 // Logits of retrieval heads (raw q.k in fp32, not divided by sqrt(d)) are
 // written to the workspace for the top-k kernel.
 #include <type_traits>
@@ -213,8 +215,14 @@ struct AttnCfg {
   static constexpr int OFF_INFO = OFF_Q + STAGES * QSTRIDE;             // [STAGES][2] int4
   static constexpr int OFF_ITEM = OFF_INFO + STAGES * 32;               // [2][IBUF]
   static constexpr int OFF_CUM = OFF_ITEM + 2 * IBUF;
-  static constexpr int OFF_BAR = (OFF_CUM + (kMaxBatchCompact + 1) * 4 + 15) / 16 * 16;
-  static constexpr int NBAR = 2 * STAGES + 4;     // full, empty, ready[2], freeb[2]
+  // tensor-core consumers: the warps' states of an item's heads, merged into
+  // one per head before they go out ([NW][MRGH][D + 2] fp32, up to four heads
+  // a round)
+  static constexpr int MRGH = G < 4 ? G : 4;
+  static constexpr int OFF_MRG = (OFF_CUM + (kMaxBatchCompact + 1) * 4 + 15) / 16 * 16;
+  static constexpr int MRGB = MMA ? NW * MRGH * (D + 2) * 4 : 0;
+  static constexpr int OFF_BAR = (OFF_MRG + MRGB + 15) / 16 * 16;
+  static constexpr int NBAR = 2 * STAGES + 6;     // full, empty, ready[2], freeb[2], mrg[2]
   static constexpr int SMEM = OFF_BAR + NBAR * 8 + ALIGN;   // + alignment slack
   static_assert(!SWZ || (OFF_V % 1024 == 0 && kStageKV % 1024 == 0 && PLANE % 1024 == 0),
                 "planes on 1024-byte boundaries");
@@ -322,7 +330,8 @@ __device__ __forceinline__ void consumer_loop(const AttnParams& p, unsigned char
                                               uint64_t* full, uint64_t* empty, uint64_t* freeb);
 template <typename T, int D, int G, int NW, int NP, int TT, int STAGES>
 __device__ __forceinline__ void consumer_loop_mma(const AttnParams& p, unsigned char* smem,
-                                                  uint64_t* full, uint64_t* empty, uint64_t* freeb);
+                                                  uint64_t* full, uint64_t* empty, uint64_t* freeb,
+                                                  uint64_t* mrg);
 
 // The tail of a stack layer's attention kernel: the combine of the previous
 // layer (its partial states are complete once the previous kernel of the stream
@@ -431,6 +440,7 @@ __global__ void __launch_bounds__((NW + NP) * 32, 1)
   uint64_t* empty = full + STAGES;
   uint64_t* ready = empty + STAGES;
   uint64_t* freeb = ready + 2;
+  uint64_t* mrg = freeb + 2;   // consumers' item-end merge: [0] states written, [1] states read
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int Hq = p.Hq, Hkv = p.Hkv, N_max = p.N_max, B = p.B;
@@ -449,6 +459,7 @@ __global__ void __launch_bounds__((NW + NP) * 32, 1)
     for (int i = 0; i < 2; ++i) {
       mbar_init(&ready[i], 1);
       mbar_init(&freeb[i], NS + NW);
+      mbar_init(&mrg[i], NW);
     }
     fence_mbar_init();
   }
@@ -599,8 +610,8 @@ __global__ void __launch_bounds__((NW + NP) * 32, 1)
               hw[0] = make_uint4(hv[0], hv[1], hv[2], hv[3]);
               hw[1] = make_uint4(hv[4], hv[5], hv[6], hv[7]);
             }
-            // every consumer warp writes a partial state for every head
-            if (lane < G) p.part_n[(size_t)(b * Hq + h0 + lane) * p.nchunk + c] = NW;
+            // the consumer warps' states are merged into one per head
+            if (lane < G) p.part_n[(size_t)(b * Hq + h0 + lane) * p.nchunk + c] = 1;
           } else {
             // each sparse head's rows as union indices, in order (lane w places
             // the rows of word w), and where each tile starts in that list: a
@@ -803,7 +814,7 @@ __global__ void __launch_bounds__((NW + NP) * 32, 1)
       if (lane == 0) mbar_arrive(&freeb[buf]);   // done reading this item's positions
     }
   } else if (warp < NW) {
-    if constexpr (C::MMA) consumer_loop_mma<T, D, G, NW, NP, TT, STAGES>(p, smem, full, empty, freeb);
+    if constexpr (C::MMA) consumer_loop_mma<T, D, G, NW, NP, TT, STAGES>(p, smem, full, empty, freeb, mrg);
     else consumer_loop<T, D, G, NW, NP, TT, STAGES>(p, smem, full, empty, freeb);
   }
   __syncthreads();
@@ -1112,11 +1123,13 @@ __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
 //   from the swizzled V planes by transposing ldmatrix, P's by two 8x8
 //   transposes in registers.  Every ldmatrix is conflict-free: the eight rows
 //   of a matrix sit in eight different 16-byte slots.
-// At the end of an item each warp writes one partial state per head of the
-// group into its own slot (slot = warp).
+// At the end of an item the warps' states of each head are merged in shared
+// memory (a fixed order: warp 0 first) and one state per head goes to slot 0
+// of the workspace, a quarter of the partial-state traffic of one per warp.
 template <typename T, int D, int G, int NW, int NP, int TT, int STAGES>
 __device__ __forceinline__ void consumer_loop_mma(const AttnParams& p, unsigned char* smem,
-                                                  uint64_t* full, uint64_t* empty, uint64_t* freeb) {
+                                                  uint64_t* full, uint64_t* empty, uint64_t* freeb,
+                                                  uint64_t* mrg) {
   using C = AttnCfg<T, D, G, NW, NP, TT, STAGES>;
   constexpr int ROWB = C::ROWB;
   constexpr int NPB = D / 32;            // 32-dimension blocks
@@ -1135,7 +1148,7 @@ __device__ __forceinline__ void consumer_loop_mma(const AttnParams& p, unsigned 
   uint32_t rm = 0;
   int b = 0, h0 = 0, c = 0, buf = 0;
 
-  uint32_t s = 0, ph = 0;
+  uint32_t s = 0, ph = 0, mph = 0;   // ring stage and phase; merge barriers' phase
   for (;;) {
     if (!mbar_wait(&full[s], ph, p.err, p.wait_ns)) break;
     const int4 i0 = info[2 * s], i1 = info[2 * s + 1];
@@ -1299,28 +1312,74 @@ __device__ __forceinline__ void consumer_loop_mma(const AttnParams& p, unsigned 
     if (flags & kLast) {
       if (lane == 0) mbar_arrive(&freeb[buf]);   // done with this item's buffer
       // the warp's state for each head of the group: l summed over the rows
-      // (lanes g), acc held once (block 2P + jp, rows g / g + 8 of O^T are
-      // dimensions 32P + 8(g/2) + 4jp + (g%2) and that + 2)
+      // (lanes g)
 #pragma unroll
       for (int o2 = 4; o2 < 32; o2 <<= 1) {
         l[0] += __shfl_xor_sync(kFull, l[0], o2);
         l[1] += __shfl_xor_sync(kFull, l[1], o2);
       }
+      // The warps' states of a head are merged into one before it goes to the
+      // workspace, up to four heads a round: every warp writes its states to
+      // the merge scratch; once all have (mrg[0]), warp w merges the round's
+      // head w and writes it (slot 0); every warp then marks the scratch read
+      // (mrg[1]) before the next round or item writes it again.
+      float* scr = reinterpret_cast<float*>(smem + C::OFF_MRG);
+      bool ok = true;
+      for (int r0 = 0; r0 < G; r0 += C::MRGH) {
 #pragma unroll
-      for (int e = 0; e < 2; ++e) {
-        const int h = 2 * t + e;
-        if (h < G) {
-          const size_t ps = ((size_t)(b * p.Hq + h0 + h) * p.nchunk + c) * kPartSlots + warp;
-          // block mb: rows g, g + 8 of O^T are dimensions 16 mb + g, + 8
-          float* dst = p.part_acc + ps * D + g;
+        for (int e = 0; e < 2; ++e) {
+          const int h = 2 * t + e;
+          if (h >= r0 && h < r0 + C::MRGH) {
+            // block mb: rows g, g + 8 of O^T are dimensions 16 mb + g, + 8
+            float* dst = scr + (warp * C::MRGH + (h - r0)) * (D + 2);
 #pragma unroll
-          for (int mb = 0; mb < 2 * NPB; ++mb) {
-            dst[16 * mb] = o[mb][e];
-            dst[16 * mb + 8] = o[mb][2 + e];
+            for (int mb = 0; mb < 2 * NPB; ++mb) {
+              dst[16 * mb + g] = o[mb][e];
+              dst[16 * mb + 8 + g] = o[mb][2 + e];
+            }
+            if (g == 0) {
+              dst[D] = m[e];
+              dst[D + 1] = l[e];
+            }
           }
-          if (g == 0) *reinterpret_cast<float2*>(p.part_ml + ps * 2) = make_float2(m[e], l[e]);
         }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&mrg[0]);
+        if (!mbar_wait(&mrg[0], mph, p.err, p.wait_ns)) {
+          ok = false;
+          break;
+        }
+        if (warp < C::MRGH) {
+          const int hr = warp, h = r0 + hr;
+          float M = -INFINITY;
+#pragma unroll
+          for (int i = 0; i < NW; ++i) M = fmaxf(M, scr[(i * C::MRGH + hr) * (D + 2) + D]);
+          float L = 0.f, acc[D / 32];
+#pragma unroll
+          for (int q = 0; q < D / 32; ++q) acc[q] = 0.f;
+#pragma unroll
+          for (int i = 0; i < NW; ++i) {
+            const float* src = scr + (i * C::MRGH + hr) * (D + 2);
+            const float mi = src[D];
+            const float w = (mi == -INFINITY) ? 0.f : fast_exp2((mi - M) * sl);
+            L += w * src[D + 1];
+#pragma unroll
+            for (int q = 0; q < D / 32; ++q) acc[q] += w * src[lane + 32 * q];
+          }
+          const size_t ps = ((size_t)(b * p.Hq + h0 + h) * p.nchunk + c) * kPartSlots;
+#pragma unroll
+          for (int q = 0; q < D / 32; ++q) p.part_acc[ps * D + lane + 32 * q] = acc[q];
+          if (lane == 0) *reinterpret_cast<float2*>(p.part_ml + ps * 2) = make_float2(M, L);
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&mrg[1]);
+        if (!mbar_wait(&mrg[1], mph, p.err, p.wait_ns)) {
+          ok = false;
+          break;
+        }
+        mph ^= 1u;
       }
+      if (!ok) break;
     }
   }
 }
