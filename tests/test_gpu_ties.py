@@ -11,7 +11,9 @@ must equal the oracle's, bit for bit:
   * signed zeros (fp32 caches, positive query): rows of +0.0 and of -0.0 give
     logits +0.0 and -0.0, which are equal; the set takes the lowest positions
     among them whatever their signs;
-  * equal block maxima straddling the block cut (block = 64).
+  * equal block maxima straddling the block cut (block = 64);
+  * a zero query through a four-layer stack: every layer's sets are positions
+    0 .. k_b - 1.
 """
 import math
 
