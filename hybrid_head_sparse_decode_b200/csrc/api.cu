@@ -296,10 +296,11 @@ struct Ctx {
 // full-length sequences, (items per SM, rounded up) x positions per item; ties
 // go to the longer chunk (fewer partial states).  Items are claimed
 // dynamically, so this only evens out the last wave (and, for a small layer,
-// spreads its rows over more SMs).  A stack's layer (`overlapped`): the next
-// layer's CTAs take the SMs this one's last wave leaves, so the longest chunk
-// that still gives every SM an item (fewer items: fewer item ends and partial
-// states; measured at 128K, 960 positions against 896: 20 us less per step).
+// spreads its rows over more SMs).  A stack's middle layer (`overlapped`): the
+// next layer's CTAs take the SMs this one's last wave leaves, so the longest
+// chunk that still gives every SM an item (fewer items: fewer item ends and
+// partial states; measured at 128K, 960 positions against 896: 20 us less per
+// step).
 int pick_chunk(const lychee_shape* s, int sms, bool overlapped) {
   if (overlapped) {
     for (int cs = kChunk; cs >= chunk_lo(s); cs -= 32)
@@ -328,6 +329,8 @@ struct LayerPlan {
   const uint8_t* prev_role = nullptr;   // stack: the previous layer's roles (null: none)
   int tail_pbuf = -1;          // stack: partial region of the previous layer, combined
   void* tail_out = nullptr;    //   by this layer's attention CTAs into tail_out
+  int chunk = 0;               // positions per work item (0: the single-layer rule)
+  int tail_chunk = 0;          // stack: the previous layer's
   bool span_start = false;     // profiler span mode: the stack's first / last
   bool span_end = false;       //   attention launch
   WindowParams win{};          // this layer's window branch, combined with fused_combine
@@ -450,7 +453,7 @@ lychee_status run_layer(const Ctx& c, const void* q, const void* kc, const void*
   ap.t_counter = ctr + 2;
   ap.B = s->B; ap.Hq = Hq; ap.Hkv = s->Hkv; ap.N_max = s->N_max;
   ap.nwords = c.L.nwords; ap.nchunk = c.L.nchunk;
-  ap.chunk = pick_chunk(s, c.sms, plan.write_bits);
+  ap.chunk = plan.chunk > 0 ? plan.chunk : pick_chunk(s, c.sms, false);
   ap.nchunk_run = (s->N_max + ap.chunk - 1) / ap.chunk;
   ap.n_items = s->B * s->Hkv * ap.nchunk_run;
   ap.scale_log2 = (float)(1.4426950408889634 / std::sqrt((double)s->d));
@@ -467,6 +470,7 @@ lychee_status run_layer(const Ctx& c, const void* q, const void* kc, const void*
     ap.t_part_acc = reinterpret_cast<const float*>(c.ws + c.L.part_acc[plan.tail_pbuf]);
     ap.t_part_n = reinterpret_cast<const int32_t*>(c.ws + c.L.part_n[plan.tail_pbuf]);
     ap.t_out = plan.tail_out;
+    ap.t_chunk = plan.tail_chunk;
     ap.t_heads = s->B * Hq;
     ap.t_win = plan.tail_win;
   }
@@ -630,8 +634,15 @@ lychee_status stack_impl(const lychee_shape* s, int32_t L, const void* q,
                              gate + (size_t)l * s->B * s->Hq, head_role + (size_t)l * s->Hq)
                  : WindowParams{};
   };
+  // Work-item length per layer: a middle layer's last wave is overlapped by the
+  // next layer's attention, so it takes the longest items; layer 0 (whose
+  // successor waits for all of its sets) and the last layer (whose combine
+  // waits for it) take the single-layer rule, which evens out the last wave.
+  auto chunk_of = [&](int l) { return pick_chunk(s, c.sms, l > 0 && l < L - 1); };
   for (int l = 0; l < L; ++l) {
     LayerPlan plan;
+    plan.chunk = chunk_of(l);
+    if (l > 0) plan.tail_chunk = chunk_of(l - 1);
     plan.lbuf = l % kLogitBufs;
     plan.pbuf = l % kPartBufs;
     plan.write_bits = true;

@@ -362,7 +362,7 @@ __device__ __forceinline__ void tail_combine(const AttnParams& p, unsigned char*
     if (bh >= p.t_heads) break;
     const int b = bh / p.Hq;
     const int n = min(max(__ldg(&p.seqlens[b]), 1), p.N_max);
-    const int nc = (n + p.chunk - 1) / p.chunk;
+    const int nc = (n + p.t_chunk - 1) / p.t_chunk;
     const int32_t* pn = p.t_part_n + (size_t)bh * p.nchunk;
     const float2* ml = reinterpret_cast<const float2*>(p.t_part_ml) + (size_t)bh * p.nchunk * kPartSlots;
     const float* pa = p.t_part_acc + (size_t)bh * p.nchunk * kPartSlots * D;

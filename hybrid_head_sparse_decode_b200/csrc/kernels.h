@@ -44,6 +44,7 @@ struct AttnParams {
   WindowParams t_win;       // the previous layer's window branch (t_win.k null: none)
   int B, Hq, Hkv, N_max, nwords, nchunk, n_items;
   int chunk;                // positions per work item (multiple of 32, kChunkMin..kChunk)
+  int t_chunk;              // the previous layer's (the chunks of the tail's partial states)
   int nchunk_run;           // chunks of N_max at that length (<= nchunk, the partials' stride)
   float scale_log2;         // log2(e) / sqrt(D)
   uint32_t role[4];         // bit h set: head h is a retrieval head
