@@ -1431,7 +1431,7 @@ cudaError_t launch_attn_t(const AttnParams& p, int num_sms, cudaStream_t st) {
 #endif
 
 #ifndef LYCHEE_ATTN_TT
-#define LYCHEE_ATTN_TT 96
+#define LYCHEE_ATTN_TT 128
 #endif
 
 // Tile rows: LYCHEE_ATTN_TT rows of up to 256 bytes, half as many of 512 bytes
