@@ -288,3 +288,21 @@ def test_stack_device_errors_are_reported_not_trapped():
                      k_per_seq=prob.k_per_seq.to(DEV), workspace=ws)
     st, bits = ops.check_device_error(ws)
     assert st == N.OK, (st, bits)
+
+
+@pytest.mark.parametrize("L", [1, 2, 3])
+def test_short_stacks_at_128k(L):
+    """Stacks of one, two and three 128K layers: the first and last layers keep
+    the single-layer work-item length (896 positions on 148 SMs) and a middle
+    layer takes the longest (960), so the tail combine reads the previous
+    layer's partial states at another length than its own; a one-layer stack
+    has no tail at all.  Every layer teacher-forced on sampled heads."""
+    prob = inputs.make_stack(L, 1, 32, 8, 128, 131072, seed=4900 + L, k_frac=0.3, n_planted=64,
+                             n_extra_retrieval=max(1, L - 1) if L > 1 else 0)
+    out, idx_final, idx_layers = run_stack(prob)
+    rep = SetReport()
+    heads = [0, 5, 13, 31]
+    for l in range(L):
+        teacher_forced_layer(prob, l, out, idx_layers, rep, nthreads=8, heads=heads)
+    assert not rep.failures, rep.failures[:5]
+    assert torch.equal(idx_final, idx_layers[-1])
